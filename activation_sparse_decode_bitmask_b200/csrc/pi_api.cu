@@ -1,0 +1,450 @@
+// The C ABI: argument validation, library-owned layer and workspace objects, and the
+// launches of the fused kernel for pi_predict / pi_sparse_ffn / pi_decode_stack.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "pi_internal.h"
+#include "pi_layout.h"
+
+using namespace pi;
+
+namespace {
+
+constexpr long long kDefaultWaitNs = 1000LL * 1000 * 1000;   // 1 s: any legitimate wait is far shorter
+static_assert(sizeof(FusedParams) <= 4000, "kernel parameter block too large");
+
+int family_of(const pi_layer_desc& d) {
+  if (d.w_dtype == PI_F32 && d.x_dtype == PI_F32 && d.p_dtype == PI_F32) return FAM_F32;
+  if (d.w_dtype == PI_F16 && d.x_dtype == PI_F16 && d.p_dtype == PI_F16) return FAM_F16;
+  if (d.w_dtype == PI_Q4_0 && d.x_dtype == PI_F16 && d.p_dtype == PI_F16) return FAM_Q4;
+  return -1;
+}
+int wbytes(int fam) { return fam == FAM_F32 ? 4 : 2; }   // fp element size (weights / predictor)
+int x_elem(const pi_layer_desc& d) { return d.x_dtype == PI_F32 ? 4 : 2; }
+int round16(long long v) { return (int)((v + 15) / 16 * 16); }
+
+int sm_count(int dev) {
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+int smem_optin(int dev) {
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+pi_status check_desc(const pi_layer_desc& d) {
+  if (d.act != PI_RELU && d.act != PI_REGLU) return PI_ERR_ARG;
+  if ((unsigned)d.w_dtype > PI_Q4_0 || (unsigned)d.x_dtype > PI_Q4_0 || (unsigned)d.p_dtype > PI_Q4_0) return PI_ERR_ARG;
+  if (d.d_model <= 0 || d.d_ff < 32 || d.rank <= 0) return PI_ERR_ARG;
+  if (d.d_ff % 32 || d.d_model % 64 || d.rank % 8 || d.rank > d.d_model) return PI_ERR_ARG;
+  const int fam = family_of(d);
+  if (fam < 0) return PI_ERR_UNSUPPORTED;
+  if (fam == FAM_Q4 && d.d_model % 256) return PI_ERR_ARG;
+  return PI_OK;
+}
+
+pi_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return PI_OK;
+  if (e == cudaErrorMemoryAllocation) { cudaGetLastError(); return PI_ERR_OOM; }
+  cudaGetLastError();
+  return PI_ERR_CUDA;
+}
+
+#define PI_TRY(expr)                              \
+  do {                                            \
+    pi_status _s = cuda_status(expr);             \
+    if (_s != PI_OK) return _s;                   \
+  } while (0)
+
+template <typename T>
+cudaError_t dmalloc(T** p, size_t bytes) {
+  return cudaMalloc(reinterpret_cast<void**>(p), bytes ? bytes : 16);
+}
+
+void free_layer_buffers(pi_layer* L) {
+  cudaFree(L->rec); cudaFree(L->p1t); cudaFree(L->p2n); cudaFree(L->bias);
+  cudaFree(L->thresh); cudaFree(L->perm); cudaFree(L->freq_sorted);
+}
+
+// Geometry of the fused kernel for one layer shape.
+pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedParams& p, size_t& smem) {
+  const pi_layer_desc& d = L->desc;
+  std::memset(&p, 0, sizeof(p));
+  p.B = B; p.d = d.d_model; p.f = d.d_ff; p.r = d.rank;
+  p.grid = ws->grid;
+  p.row_bytes = L->row_bytes; p.rec_stride = L->rec_stride;
+  p.gate_off = L->gate_off; p.up_off = L->up_off; p.down_off = L->down_off;
+  p.p1_row = L->p1_row; p.p2_stride = L->p2_stride;
+  p.slot_bytes = std::max({L->row_bytes, L->p1_row, L->p2_stride});
+  p.rows_per_p2slot = p.slot_bytes / L->p2_stride;
+  const int ngroups = d.d_model / 32;
+  p.nslices = std::min(ws->grid, ngroups);
+  if ((ngroups + p.nslices - 1) / p.nslices > 4) return PI_ERR_UNSUPPORTED;
+  if ((d.d_ff + ws->grid - 1) / ws->grid > kMaxOwn) return PI_ERR_UNSUPPORTED;
+  if (!fused_supported(L->family, B, d.d_model)) return PI_ERR_UNSUPPORTED;
+  const size_t budget = (size_t)smem_optin(ws->device);
+  const size_t fixed = fused_fixed_smem(B, d.rank);
+  if (budget <= fixed + 3 * (size_t)p.slot_bytes) return PI_ERR_UNSUPPORTED;
+  p.nslots = (int)std::min<size_t>(kMaxSlots, (budget - fixed) / p.slot_bytes);
+  smem = fused_smem_bytes(p);
+  // ws fields
+  p.u = ws->u; p.maskbuf = ws->maskbuf; p.partials = ws->partials; p.v = ws->v; p.xb = ws->xb;
+  p.ssq = ws->ssq; p.bar = ws->bar; p.err = ws->err; p.active_total = ws->active_total;
+  p.layer_count = nullptr;
+  p.barrier_timeout_ns = kDefaultWaitNs;
+  p.barrier_extra = 0;
+  return PI_OK;
+}
+
+pi_status check_ws(const pi_workspace* ws, const pi_layer_desc& d, int B, int L) {
+  if (!ws) return PI_ERR_ARG;
+  if (d.d_model > ws->d_max || d.d_ff > ws->f_max || d.rank > ws->r_max || B > ws->B_max || L > ws->L_max)
+    return PI_ERR_ARG;
+  return PI_OK;
+}
+
+LayerDev dev_view(const pi_layer* L) { return LayerDev{L->rec, L->p1t, L->p2n}; }
+
+bool same_desc(const pi_layer_desc& a, const pi_layer_desc& b) {
+  return a.d_model == b.d_model && a.d_ff == b.d_ff && a.rank == b.rank && a.act == b.act &&
+         a.w_dtype == b.w_dtype && a.x_dtype == b.x_dtype && a.p_dtype == b.p_dtype;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pi_abi_version(void) { return 10000; }
+
+const char* pi_status_str(pi_status s) {
+  switch (s) {
+    case PI_OK: return "ok";
+    case PI_ERR_ARG: return "invalid argument";
+    case PI_ERR_UNSUPPORTED: return "unsupported shape, batch or dtype combination";
+    case PI_ERR_OOM: return "device allocation failed";
+    case PI_ERR_CUDA: return "CUDA runtime error";
+    case PI_ERR_TIMEOUT: return "a device-side wait timed out";
+    case PI_ERR_DEVICE: return "a device-side check failed";
+  }
+  return "unknown status";
+}
+
+// ------------------------------------------------------------------ layers
+pi_status pi_load_layer(const pi_layer_desc* desc, const pi_layer_weights* w, cudaStream_t stream,
+                        pi_layer** out) {
+  if (!desc || !w || !out) return PI_ERR_ARG;
+  *out = nullptr;
+  pi_status st = check_desc(*desc);
+  if (st != PI_OK) return st;
+  const pi_layer_desc& d = *desc;
+  const int fam = family_of(d);
+  const bool reglu = d.act == PI_REGLU;
+  if (!w->w_up || !w->w_down || !w->bias || !w->p1 || !w->p2 || !w->thresh) return PI_ERR_ARG;
+  if (reglu != (w->w_gate != nullptr)) return PI_ERR_ARG;
+  if (fam == FAM_Q4 && (!w->s_up || !w->s_down || (reglu && !w->s_gate))) return PI_ERR_ARG;
+  if (fam != FAM_Q4 && (w->s_up || w->s_gate || w->s_down)) return PI_ERR_ARG;
+
+  pi_layer* L = new (std::nothrow) pi_layer;
+  if (!L) return PI_ERR_OOM;
+  std::memset(L, 0, sizeof(*L));
+  L->desc = d;
+  L->family = fam;
+  L->hot_count = -1;
+  cudaGetDevice(&L->device);
+  const int D = d.d_model, F = d.d_ff, R = d.rank;
+  const int pb = wbytes(fam == FAM_Q4 ? FAM_F16 : fam);
+  L->row_bytes = fam == FAM_Q4 ? round16((long long)D / 2 + D / 16) : D * wbytes(fam);
+  const int nrows = reglu ? 3 : 2;
+  L->rec_stride = L->row_bytes * nrows;
+  L->gate_off = reglu ? 0 : -1;
+  L->up_off = reglu ? L->row_bytes : 0;
+  L->down_off = L->up_off + L->row_bytes;
+  L->p1_row = D * pb;
+  L->p2_stride = round16((long long)R * pb + 8);
+
+  auto fail = [&](pi_status s) { free_layer_buffers(L); delete L; return s; };
+  if (dmalloc(&L->rec, (size_t)F * L->rec_stride) != cudaSuccess) return fail(PI_ERR_OOM);
+  if (dmalloc(&L->p1t, (size_t)R * L->p1_row) != cudaSuccess) return fail(PI_ERR_OOM);
+  if (dmalloc(&L->p2n, (size_t)F * L->p2_stride) != cudaSuccess) return fail(PI_ERR_OOM);
+  if (dmalloc(&L->bias, (size_t)F * 4) != cudaSuccess) return fail(PI_ERR_OOM);
+  if (dmalloc(&L->thresh, (size_t)F * 4) != cudaSuccess) return fail(PI_ERR_OOM);
+  if (dmalloc(&L->perm, (size_t)F * 4) != cudaSuccess) return fail(PI_ERR_OOM);
+
+  cudaError_t e = cudaSuccess;
+  auto step = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
+  step(cudaMemsetAsync(L->rec, 0, (size_t)F * L->rec_stride, stream));
+  step(cudaMemsetAsync(L->p2n, 0, (size_t)F * L->p2_stride, stream));
+  if (fam == FAM_Q4) {
+    const int nb = D / 32;
+    const void* nib[3] = {w->w_gate, w->w_up, w->w_down};
+    const void* scl[3] = {w->s_gate, w->s_up, w->s_down};
+    const int off[3] = {L->gate_off, L->up_off, L->down_off};
+    for (int m = reglu ? 0 : 1; m < 3; ++m) {
+      step(relayout_copy_rows(nib[m], nb * 16, 0, L->rec, L->rec_stride, off[m], F, nb * 16, nullptr, stream));
+      step(relayout_copy_rows(scl[m], nb * 2, 0, L->rec, L->rec_stride, off[m] + D / 2, F, nb * 2, nullptr, stream));
+    }
+  } else {
+    const int wb = wbytes(fam);
+    if (reglu) step(relayout_copy_rows(w->w_gate, (long long)D * wb, 0, L->rec, L->rec_stride, L->gate_off, F, D * wb, nullptr, stream));
+    step(relayout_copy_rows(w->w_up, (long long)D * wb, 0, L->rec, L->rec_stride, L->up_off, F, D * wb, nullptr, stream));
+    // down: caller's [d x f] row-major -> neuron-major rows
+    step(relayout_transpose(w->w_down, wb, D, F, F, L->rec, L->rec_stride, L->down_off, stream));
+  }
+  // P1 [d x r] -> P1^T [r x d];  P2 [r x f] -> per-neuron rows [f][r] + (t, b)
+  step(relayout_transpose(w->p1, pb, D, R, R, L->p1t, L->p1_row, 0, stream));
+  step(relayout_transpose(w->p2, pb, R, F, F, L->p2n, L->p2_stride, 0, stream));
+  step(relayout_p2_header(w->thresh, w->bias, F, L->p2n, L->p2_stride, R * pb, stream));
+  step(cudaMemcpyAsync(L->bias, w->bias, (size_t)F * 4, cudaMemcpyDeviceToDevice, stream));
+  step(cudaMemcpyAsync(L->thresh, w->thresh, (size_t)F * 4, cudaMemcpyDeviceToDevice, stream));
+  step(iota_i32(L->perm, F, stream));
+  step(cudaStreamSynchronize(stream));
+  if (e != cudaSuccess) return fail(cuda_status(e));
+  *out = L;
+  return PI_OK;
+}
+
+void pi_free_layer(pi_layer* L) {
+  if (!L) return;
+  free_layer_buffers(L);
+  delete L;
+}
+
+pi_status pi_layer_get_desc(const pi_layer* L, pi_layer_desc* out) {
+  if (!L || !out) return PI_ERR_ARG;
+  *out = L->desc;
+  return PI_OK;
+}
+
+pi_status pi_get_perm(const pi_layer* L, int32_t* perm_out, cudaStream_t stream) {
+  if (!L || !perm_out) return PI_ERR_ARG;
+  return cuda_status(cudaMemcpyAsync(perm_out, L->perm, (size_t)L->desc.d_ff * 4, cudaMemcpyDeviceToDevice, stream));
+}
+
+pi_status pi_reorder_hot_prefix(pi_layer* L, const float* freq, int hot_count, cudaStream_t stream) {
+  if (!L || !freq) return PI_ERR_ARG;
+  const int F = L->desc.d_ff;
+  if (hot_count < -1 || hot_count > F) return PI_ERR_ARG;
+  int32_t* order = nullptr;
+  int* bad = nullptr;
+  uint8_t *rec = nullptr, *p2n = nullptr;
+  float *bias = nullptr, *thresh = nullptr, *fs = nullptr;
+  int32_t* perm = nullptr;
+  auto cleanup = [&]() {
+    cudaFree(order); cudaFree(bad); cudaFree(rec); cudaFree(p2n); cudaFree(bias); cudaFree(thresh);
+    cudaFree(fs); cudaFree(perm);
+  };
+  if (dmalloc(&order, (size_t)F * 4) || dmalloc(&bad, 4) || dmalloc(&rec, (size_t)F * L->rec_stride) ||
+      dmalloc(&p2n, (size_t)F * L->p2_stride) || dmalloc(&bias, (size_t)F * 4) || dmalloc(&thresh, (size_t)F * 4) ||
+      dmalloc(&fs, (size_t)F * 4) || dmalloc(&perm, (size_t)F * 4)) {
+    cleanup();
+    return PI_ERR_OOM;
+  }
+  cudaError_t e = cudaSuccess;
+  auto step = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
+  step(cudaMemsetAsync(bad, 0, 4, stream));
+  step(hot_order(freq, F, order, bad, stream));
+  int hbad = 0;
+  step(cudaMemcpyAsync(&hbad, bad, 4, cudaMemcpyDeviceToHost, stream));
+  step(cudaStreamSynchronize(stream));
+  if (e != cudaSuccess) { cleanup(); return cuda_status(e); }
+  if (hbad) { cleanup(); return PI_ERR_ARG; }
+  step(relayout_copy_rows(L->rec, L->rec_stride, 0, rec, L->rec_stride, 0, F, L->rec_stride, order, stream));
+  step(relayout_copy_rows(L->p2n, L->p2_stride, 0, p2n, L->p2_stride, 0, F, L->p2_stride, order, stream));
+  step(gather_f32(L->bias, order, F, bias, stream));
+  step(gather_f32(L->thresh, order, F, thresh, stream));
+  step(gather_f32(freq, order, F, fs, stream));
+  step(gather_i32(L->perm, order, F, perm, stream));
+  step(cudaStreamSynchronize(stream));
+  if (e != cudaSuccess) { cleanup(); return cuda_status(e); }
+  std::swap(L->rec, rec);
+  std::swap(L->p2n, p2n);
+  std::swap(L->bias, bias);
+  std::swap(L->thresh, thresh);
+  std::swap(L->freq_sorted, fs);
+  std::swap(L->perm, perm);
+  L->hot_count = hot_count;
+  cleanup();   // frees the old buffers now held in the temporaries
+  return PI_OK;
+}
+
+// ------------------------------------------------------------------ workspace
+pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_max, pi_workspace** out) {
+  if (!out) return PI_ERR_ARG;
+  *out = nullptr;
+  if (d_max <= 0 || f_max <= 0 || r_max <= 0 || B_max < 1 || B_max > PI_MAX_BATCH || L_max < 1 || L_max > kMaxLayers)
+    return PI_ERR_ARG;
+  if (d_max % 64 || f_max % 32) return PI_ERR_ARG;
+  pi_workspace* ws = new (std::nothrow) pi_workspace;
+  if (!ws) return PI_ERR_OOM;
+  std::memset(ws, 0, sizeof(*ws));
+  ws->d_max = d_max; ws->f_max = f_max; ws->r_max = r_max; ws->B_max = B_max; ws->L_max = L_max;
+  cudaGetDevice(&ws->device);
+  ws->grid = sm_count(ws->device);
+  if (ws->grid <= 0) { delete ws; return PI_ERR_CUDA; }
+  const size_t G = ws->grid, Bm = B_max;
+  bool ok = dmalloc(&ws->u, Bm * r_max * 4) == cudaSuccess &&
+            dmalloc(&ws->maskbuf, 2 * Bm * (f_max / 32) * 4) == cudaSuccess &&
+            dmalloc(&ws->partials, G * Bm * d_max * 4) == cudaSuccess &&
+            dmalloc(&ws->v, Bm * d_max * 4) == cudaSuccess &&
+            dmalloc(&ws->xb, 2 * Bm * d_max * 4) == cudaSuccess &&
+            dmalloc(&ws->ssq, Bm * G * 4) == cudaSuccess &&
+            dmalloc(&ws->bar, 64) == cudaSuccess &&
+            dmalloc(&ws->err, 16) == cudaSuccess &&
+            dmalloc(&ws->active_total, 16) == cudaSuccess &&
+            dmalloc(&ws->layer_count, (size_t)L_max * 4) == cudaSuccess &&
+            dmalloc(&ws->x_dev, Bm * d_max * 4) == cudaSuccess;
+  if (ok) {
+    ok = cudaMemset(ws->bar, 0, 64) == cudaSuccess && cudaMemset(ws->err, 0, 16) == cudaSuccess &&
+         cudaMemset(ws->active_total, 0, 16) == cudaSuccess &&
+         cudaMemset(ws->layer_count, 0, (size_t)L_max * 4) == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
+  }
+  if (!ok) {
+    cudaGetLastError();
+    pi_workspace_free(ws);
+    return PI_ERR_OOM;
+  }
+  *out = ws;
+  return PI_OK;
+}
+
+void pi_workspace_free(pi_workspace* ws) {
+  if (!ws) return;
+  cudaFree(ws->u); cudaFree(ws->maskbuf); cudaFree(ws->partials); cudaFree(ws->v); cudaFree(ws->xb);
+  cudaFree(ws->ssq); cudaFree(ws->bar); cudaFree(ws->err); cudaFree(ws->active_total);
+  cudaFree(ws->layer_count); cudaFree(ws->x_dev);
+  delete ws;
+}
+
+pi_status pi_stream_status(pi_workspace* ws, cudaStream_t stream) {
+  if (!ws) return PI_ERR_ARG;
+  PI_TRY(cudaStreamSynchronize(stream));
+  int err = 0;
+  PI_TRY(cudaMemcpy(&err, ws->err, 4, cudaMemcpyDeviceToHost));
+  if (err == 0) return PI_OK;
+  PI_TRY(cudaMemset(ws->err, 0, 16));
+  PI_TRY(cudaMemset(ws->bar, 0, 64));
+  PI_TRY(cudaDeviceSynchronize());
+  return (err == DEV_ERR_GRID_TIMEOUT || err == DEV_ERR_RING_TIMEOUT) ? PI_ERR_TIMEOUT : PI_ERR_DEVICE;
+}
+
+pi_status pi_workspace_active_total(pi_workspace* ws, unsigned long long* out) {
+  if (!ws || !out) return PI_ERR_ARG;
+  PI_TRY(cudaMemcpy(out, ws->active_total, 8, cudaMemcpyDeviceToHost));
+  return PI_OK;
+}
+
+pi_status pi_workspace_layer_counts(pi_workspace* ws, int32_t* host_out, int L) {
+  if (!ws || !host_out || L < 1 || L > ws->L_max) return PI_ERR_ARG;
+  PI_TRY(cudaMemcpy(host_out, ws->layer_count, (size_t)L * 4, cudaMemcpyDeviceToHost));
+  return PI_OK;
+}
+
+// ------------------------------------------------------------------ hot path
+pi_status pi_predict(const pi_layer* L, const void* x, int B, uint32_t* mask, float* logits, pi_workspace* ws,
+                     cudaStream_t stream) {
+  if (!L || !x || !mask || B < 1 || B > PI_MAX_BATCH) return PI_ERR_ARG;
+  pi_status st = check_ws(ws, L->desc, B, 1);
+  if (st != PI_OK) return st;
+  FusedParams p;
+  size_t smem = 0;
+  st = plan_fused(L, B, ws, p, smem);
+  if (st != PI_OK) return st;
+  p.mode = MODE_PREDICT;
+  p.L = 1;
+  p.layers[0] = dev_view(L);
+  p.x_in = x;
+  p.mask_out = mask;
+  p.logits_out = logits;
+  PI_TRY(cudaMemsetAsync(mask, 0, (size_t)B * (L->desc.d_ff / 32) * 4, stream));
+  PI_TRY(launch_fused(L->family, L->desc.act, B, p, smem, stream));
+  return PI_OK;
+}
+
+pi_status pi_compact_active(const uint32_t* mask, int B, int d_ff, int32_t* idx, int32_t* count, cudaStream_t stream) {
+  if (!mask || !idx || !count || B < 1 || B > PI_MAX_BATCH || d_ff < 32 || d_ff % 32) return PI_ERR_ARG;
+  PI_TRY(launch_compact(mask, B, d_ff, idx, count, stream));
+  return PI_OK;
+}
+
+pi_status pi_sparse_ffn(const pi_layer* L, const void* x, int B, const uint32_t* mask, const int32_t* idx,
+                        const int32_t* count, float* y, pi_workspace* ws, cudaStream_t stream) {
+  if (!L || !x || !mask || !idx || !count || !y || B < 1 || B > PI_MAX_BATCH) return PI_ERR_ARG;
+  pi_status st = check_ws(ws, L->desc, B, 1);
+  if (st != PI_OK) return st;
+  FusedParams p;
+  size_t smem = 0;
+  st = plan_fused(L, B, ws, p, smem);
+  if (st != PI_OK) return st;
+  if ((L->desc.d_ff + ws->grid - 1) / ws->grid > kMaxList) return PI_ERR_UNSUPPORTED;
+  p.mode = MODE_FFN;
+  p.L = 1;
+  p.layers[0] = dev_view(L);
+  p.x_in = x;
+  p.mask_in = mask;
+  p.idx_in = idx;
+  p.count_in = count;
+  p.y_out = y;
+  PI_TRY(launch_fused(L->family, L->desc.act, B, p, smem, stream));
+  return PI_OK;
+}
+
+pi_status pi_decode_stack(pi_layer* const* layers, int Lc, void* x_inout, int B, const pi_trace* trace,
+                          pi_workspace* ws, cudaStream_t stream) {
+  if (!layers || Lc < 1 || Lc > kMaxLayers || !x_inout || B < 1 || B > PI_MAX_BATCH) return PI_ERR_ARG;
+  for (int l = 0; l < Lc; ++l) {
+    if (!layers[l]) return PI_ERR_ARG;
+    if (!same_desc(layers[l]->desc, layers[0]->desc)) return PI_ERR_ARG;
+  }
+  const pi_layer* L0 = layers[0];
+  pi_status st = check_ws(ws, L0->desc, B, Lc);
+  if (st != PI_OK) return st;
+  FusedParams p;
+  size_t smem = 0;
+  st = plan_fused(L0, B, ws, p, smem);
+  if (st != PI_OK) return st;
+  p.mode = MODE_PREDICT | MODE_FFN | MODE_GLUE;
+  p.L = Lc;
+  for (int l = 0; l < Lc; ++l) p.layers[l] = dev_view(layers[l]);
+  p.x_in = x_inout;
+  p.x_out = x_inout;
+  if (trace) p.trace = *trace;
+  p.layer_count = ws->layer_count;
+  PI_TRY(cudaMemsetAsync(ws->layer_count, 0, (size_t)Lc * 4, stream));
+  PI_TRY(launch_fused(L0->family, L0->desc.act, B, p, smem, stream));
+  return PI_OK;
+}
+
+pi_status pi_decode_stack_host(pi_layer* const* layers, int Lc, const void* x_host, void* x_out_host, int B,
+                               pi_workspace* ws, cudaStream_t stream) {
+  if (!layers || Lc < 1 || !layers[0] || !x_host || !x_out_host || !ws || B < 1 || B > ws->B_max) return PI_ERR_ARG;
+  const size_t bytes = (size_t)B * layers[0]->desc.d_model * x_elem(layers[0]->desc);
+  if (layers[0]->desc.d_model > ws->d_max) return PI_ERR_ARG;
+  PI_TRY(cudaMemcpyAsync(ws->x_dev, x_host, bytes, cudaMemcpyHostToDevice, stream));
+  pi_status st = pi_decode_stack(layers, Lc, ws->x_dev, B, nullptr, ws, stream);
+  if (st != PI_OK) return st;
+  PI_TRY(cudaMemcpyAsync(x_out_host, ws->x_dev, bytes, cudaMemcpyDeviceToHost, stream));
+  return pi_stream_status(ws, stream);
+}
+
+pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaStream_t stream) {
+  if (!ws || timeout_ns <= 0) return PI_ERR_ARG;
+  FusedParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.grid = ws->grid;
+  p.bar = ws->bar;
+  p.err = ws->err;
+  p.barrier_timeout_ns = timeout_ns;
+  p.barrier_extra = 1;   // one arrival more than the grid has: no wait can complete
+  PI_TRY(launch_barrier_probe(p, 2, stream));
+  return PI_OK;
+}
+
+}  // extern "C"
