@@ -25,7 +25,8 @@ STATUS = {0: "PI_OK", 1: "PI_ERR_ARG", 2: "PI_ERR_UNSUPPORTED", 3: "PI_ERR_OOM",
 # every entry point the header declares, in declaration order
 EXPORTS = ["pi_load_layer", "pi_reorder_hot_prefix", "pi_get_perm", "pi_layer_get_desc", "pi_free_layer",
            "pi_workspace_create", "pi_workspace_free", "pi_stream_status", "pi_workspace_active_total",
-           "pi_workspace_layer_counts", "pi_diag_barrier_timeout", "pi_predict", "pi_compact_active",
+           "pi_workspace_layer_counts", "pi_diag_phase_clocks_enable", "pi_diag_phase_clocks_read",
+           "pi_device_grid", "pi_diag_barrier_timeout", "pi_predict", "pi_compact_active",
            "pi_sparse_ffn", "pi_decode_stack", "pi_decode_stack_host", "pi_status_str", "pi_abi_version"]
 
 
@@ -66,6 +67,9 @@ def _load() -> ctypes.CDLL:
         "pi_workspace_active_total": (i, [vp, POINTER(c_ulonglong)]),
         "pi_workspace_layer_counts": (i, [vp, vp, i]),
         "pi_diag_barrier_timeout": (i, [vp, c_longlong, vp]),
+        "pi_diag_phase_clocks_enable": (i, [vp, i]),
+        "pi_diag_phase_clocks_read": (i, [vp, vp, ctypes.c_size_t]),
+        "pi_device_grid": (i, [vp]),
         "pi_predict": (i, [vp, vp, i, vp, vp, vp, vp]),
         "pi_compact_active": (i, [vp, i, i, vp, vp, vp]),
         "pi_sparse_ffn": (i, [vp, vp, i, vp, vp, vp, vp, vp, vp]),
@@ -156,6 +160,21 @@ class Workspace:
         v = c_ulonglong()
         _check(_lib.pi_workspace_active_total(self.handle, byref(v)), "pi_workspace_active_total")
         return int(v.value)
+
+    def grid(self) -> int:
+        return _lib.pi_device_grid(self.handle)
+
+    def phase_clocks(self, on=True) -> None:
+        """on: False/0 off, True/1 SM cycle stamps, 2 global-timer nanosecond stamps."""
+        _check(_lib.pi_diag_phase_clocks_enable(self.handle, int(on)), "pi_diag_phase_clocks_enable")
+
+    def read_phase_clocks(self, L_max: int):
+        """[grid, L_max, 12] int64 SM cycle stamps of the last stack call."""
+        import numpy as np
+        g = self.grid()
+        out = np.zeros((g, L_max, 12), dtype=np.int64)
+        _check(_lib.pi_diag_phase_clocks_read(self.handle, out.ctypes.data, out.size), "pi_diag_phase_clocks_read")
+        return out
 
     def layer_counts(self, L: int):
         out = (c_int32 * L)()

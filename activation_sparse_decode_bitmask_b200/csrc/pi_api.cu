@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -70,8 +71,10 @@ cudaError_t dmalloc(T** p, size_t bytes) {
 }
 
 void free_layer_buffers(pi_layer* L) {
-  cudaFree(L->rec); cudaFree(L->p1t); cudaFree(L->p2n); cudaFree(L->bias);
+  cudaFree(L->rec); cudaFree(L->p1t); cudaFree(L->p2o); cudaFree(L->bias);
   cudaFree(L->thresh); cudaFree(L->perm); cudaFree(L->freq_sorted);
+  delete[] L->freq_host;
+  L->freq_host = nullptr;
 }
 
 // Geometry of the fused kernel for one layer shape.
@@ -81,23 +84,34 @@ pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedPara
   p.B = B; p.d = d.d_model; p.f = d.d_ff; p.r = d.rank;
   p.grid = ws->grid;
   p.row_bytes = L->row_bytes; p.rec_stride = L->rec_stride;
-  p.gate_off = L->gate_off; p.up_off = L->up_off; p.down_off = L->down_off;
+  p.gate_off = L->gate_off; p.up_off = L->up_off; p.down_off = L->down_off; p.bias_off = L->bias_off;
   p.p1_row = L->p1_row; p.p2_stride = L->p2_stride;
-  p.slot_bytes = std::max({L->row_bytes, L->p1_row, L->p2_stride});
-  p.rows_per_p2slot = p.slot_bytes / L->p2_stride;
+  p.nown_max = L->nown_max;
   const int ngroups = d.d_model / 32;
   p.nslices = std::min(ws->grid, ngroups);
   if ((ngroups + p.nslices - 1) / p.nslices > 4) return PI_ERR_UNSUPPORTED;
-  if ((d.d_ff + ws->grid - 1) / ws->grid > kMaxOwn) return PI_ERR_UNSUPPORTED;
+  if (L->G != ws->grid) return PI_ERR_ARG;   // layer laid out for another device
+  if (L->nown_max > kMaxOwn) return PI_ERR_UNSUPPORTED;
   if (!fused_supported(L->family, B, d.d_model)) return PI_ERR_UNSUPPORTED;
+  // ring items: whole neuron records, and predictor rows grouped into ~32 KB copies
+  const int cap = std::max(L->rec_stride, 32 * 1024);
+  p.p1_rows_per_item = std::max(1, cap / L->p1_row);
+  p.p2_rows_per_item = std::max(1, cap / L->p2_stride);
+  const long long max_item = std::max({(long long)L->rec_stride, (long long)p.p1_rows_per_item * L->p1_row,
+                                       (long long)p.p2_rows_per_item * L->p2_stride});
   const size_t budget = (size_t)smem_optin(ws->device);
-  const size_t fixed = fused_fixed_smem(B, d.rank);
-  if (budget <= fixed + 3 * (size_t)p.slot_bytes) return PI_ERR_UNSUPPORTED;
-  p.nslots = (int)std::min<size_t>(kMaxSlots, (budget - fixed) / p.slot_bytes);
-  smem = fused_smem_bytes(p);
+  const size_t fixed = fused_fixed_smem(B, d.d_model, d.rank, ws->grid, L->nown_max, L->family);
+  if (budget <= fixed) return PI_ERR_UNSUPPORTED;
+  p.ring_bytes = (int)((budget - fixed) / 128 * 128);
+  if (p.ring_bytes < 2 * max_item || max_item >= (1 << 20)) return PI_ERR_UNSUPPORTED;
+  // records per F batch: the whole batch must sit in the ring at once (one record of
+  // slack for the placement that never wraps an item)
+  p.batch = std::min(fused_max_batch(), p.ring_bytes / L->rec_stride - 1);
+  if (p.batch < 1) return PI_ERR_UNSUPPORTED;
+  smem = fixed + (size_t)p.ring_bytes;
   // ws fields
-  p.u = ws->u; p.maskbuf = ws->maskbuf; p.partials = ws->partials; p.v = ws->v; p.xb = ws->xb;
-  p.ssq = ws->ssq; p.bar = ws->bar; p.err = ws->err; p.active_total = ws->active_total;
+  p.ux = ws->ux; p.px = ws->px; p.vx = ws->vx; p.sx = ws->sx; p.bx = ws->bx;
+  p.bar = ws->bar; p.err = ws->err; p.active_total = ws->active_total;
   p.layer_count = nullptr;
   p.barrier_timeout_ns = kDefaultWaitNs;
   p.barrier_extra = 0;
@@ -111,7 +125,18 @@ pi_status check_ws(const pi_workspace* ws, const pi_layer_desc& d, int B, int L)
   return PI_OK;
 }
 
-LayerDev dev_view(const pi_layer* L) { return LayerDev{L->rec, L->p1t, L->p2n}; }
+// Hot-prefix length at batch B: the neurons (in hot order) whose union firing probability
+// 1 - (1 - f)^B is at least 1/2, or the count fixed by pi_reorder_hot_prefix.
+int hot_len(const pi_layer* L, int B) {
+  if (!L->freq_host) return 0;
+  if (L->hot_count >= 0) return L->hot_count;
+  int n = 0;
+  const int F = L->desc.d_ff;
+  while (n < F && 1.0 - std::pow(1.0 - (double)L->freq_host[n], (double)B) >= 0.5) ++n;
+  return n;
+}
+
+LayerDev dev_view(const pi_layer* L, int B = 0) { return LayerDev{L->rec, L->p1t, L->p2o, B > 0 ? hot_len(L, B) : 0, 0}; }
 
 bool same_desc(const pi_layer_desc& a, const pi_layer_desc& b) {
   return a.d_model == b.d_model && a.d_ff == b.d_ff && a.rank == b.rank && a.act == b.act &&
@@ -163,17 +188,21 @@ pi_status pi_load_layer(const pi_layer_desc* desc, const pi_layer_weights* w, cu
   const int pb = wbytes(fam == FAM_Q4 ? FAM_F16 : fam);
   L->row_bytes = fam == FAM_Q4 ? round16((long long)D / 2 + D / 16) : D * wbytes(fam);
   const int nrows = reglu ? 3 : 2;
-  L->rec_stride = L->row_bytes * nrows;
+  L->rec_stride = L->row_bytes * nrows + 16;   // rows, then a 16-byte header with the bias
   L->gate_off = reglu ? 0 : -1;
   L->up_off = reglu ? L->row_bytes : 0;
   L->down_off = L->up_off + L->row_bytes;
+  L->bias_off = L->down_off + L->row_bytes;
   L->p1_row = D * pb;
   L->p2_stride = round16((long long)R * pb + 8);
+  L->G = sm_count(L->device);
+  if (L->G <= 0) { delete L; return PI_ERR_CUDA; }
+  L->nown_max = (F + L->G - 1) / L->G;
 
   auto fail = [&](pi_status s) { free_layer_buffers(L); delete L; return s; };
   if (dmalloc(&L->rec, (size_t)F * L->rec_stride) != cudaSuccess) return fail(PI_ERR_OOM);
   if (dmalloc(&L->p1t, (size_t)R * L->p1_row) != cudaSuccess) return fail(PI_ERR_OOM);
-  if (dmalloc(&L->p2n, (size_t)F * L->p2_stride) != cudaSuccess) return fail(PI_ERR_OOM);
+  if (dmalloc(&L->p2o, (size_t)L->G * L->nown_max * L->p2_stride) != cudaSuccess) return fail(PI_ERR_OOM);
   if (dmalloc(&L->bias, (size_t)F * 4) != cudaSuccess) return fail(PI_ERR_OOM);
   if (dmalloc(&L->thresh, (size_t)F * 4) != cudaSuccess) return fail(PI_ERR_OOM);
   if (dmalloc(&L->perm, (size_t)F * 4) != cudaSuccess) return fail(PI_ERR_OOM);
@@ -181,7 +210,7 @@ pi_status pi_load_layer(const pi_layer_desc* desc, const pi_layer_weights* w, cu
   cudaError_t e = cudaSuccess;
   auto step = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
   step(cudaMemsetAsync(L->rec, 0, (size_t)F * L->rec_stride, stream));
-  step(cudaMemsetAsync(L->p2n, 0, (size_t)F * L->p2_stride, stream));
+  step(cudaMemsetAsync(L->p2o, 0, (size_t)L->G * L->nown_max * L->p2_stride, stream));
   if (fam == FAM_Q4) {
     const int nb = D / 32;
     const void* nib[3] = {w->w_gate, w->w_up, w->w_down};
@@ -200,8 +229,9 @@ pi_status pi_load_layer(const pi_layer_desc* desc, const pi_layer_weights* w, cu
   }
   // P1 [d x r] -> P1^T [r x d];  P2 [r x f] -> per-neuron rows [f][r] + (t, b)
   step(relayout_transpose(w->p1, pb, D, R, R, L->p1t, L->p1_row, 0, stream));
-  step(relayout_transpose(w->p2, pb, R, F, F, L->p2n, L->p2_stride, 0, stream));
-  step(relayout_p2_header(w->thresh, w->bias, F, L->p2n, L->p2_stride, R * pb, stream));
+  step(relayout_transpose(w->p2, pb, R, F, F, L->p2o, L->p2_stride, 0, stream, L->G, L->nown_max));
+  step(relayout_p2_header(w->thresh, w->bias, F, L->p2o, L->p2_stride, R * pb, L->G, L->nown_max, stream));
+  step(relayout_row_scalar(w->bias, F, L->rec, L->rec_stride, L->bias_off, stream));
   step(cudaMemcpyAsync(L->bias, w->bias, (size_t)F * 4, cudaMemcpyDeviceToDevice, stream));
   step(cudaMemcpyAsync(L->thresh, w->thresh, (size_t)F * 4, cudaMemcpyDeviceToDevice, stream));
   step(iota_i32(L->perm, F, stream));
@@ -234,15 +264,16 @@ pi_status pi_reorder_hot_prefix(pi_layer* L, const float* freq, int hot_count, c
   if (hot_count < -1 || hot_count > F) return PI_ERR_ARG;
   int32_t* order = nullptr;
   int* bad = nullptr;
-  uint8_t *rec = nullptr, *p2n = nullptr;
+  uint8_t *rec = nullptr, *p2o = nullptr;
+  const size_t p2_bytes = (size_t)L->G * L->nown_max * L->p2_stride;
   float *bias = nullptr, *thresh = nullptr, *fs = nullptr;
   int32_t* perm = nullptr;
   auto cleanup = [&]() {
-    cudaFree(order); cudaFree(bad); cudaFree(rec); cudaFree(p2n); cudaFree(bias); cudaFree(thresh);
+    cudaFree(order); cudaFree(bad); cudaFree(rec); cudaFree(p2o); cudaFree(bias); cudaFree(thresh);
     cudaFree(fs); cudaFree(perm);
   };
   if (dmalloc(&order, (size_t)F * 4) || dmalloc(&bad, 4) || dmalloc(&rec, (size_t)F * L->rec_stride) ||
-      dmalloc(&p2n, (size_t)F * L->p2_stride) || dmalloc(&bias, (size_t)F * 4) || dmalloc(&thresh, (size_t)F * 4) ||
+      dmalloc(&p2o, p2_bytes) || dmalloc(&bias, (size_t)F * 4) || dmalloc(&thresh, (size_t)F * 4) ||
       dmalloc(&fs, (size_t)F * 4) || dmalloc(&perm, (size_t)F * 4)) {
     cleanup();
     return PI_ERR_OOM;
@@ -257,7 +288,8 @@ pi_status pi_reorder_hot_prefix(pi_layer* L, const float* freq, int hot_count, c
   if (e != cudaSuccess) { cleanup(); return cuda_status(e); }
   if (hbad) { cleanup(); return PI_ERR_ARG; }
   step(relayout_copy_rows(L->rec, L->rec_stride, 0, rec, L->rec_stride, 0, F, L->rec_stride, order, stream));
-  step(relayout_copy_rows(L->p2n, L->p2_stride, 0, p2n, L->p2_stride, 0, F, L->p2_stride, order, stream));
+  step(cudaMemsetAsync(p2o, 0, p2_bytes, stream));
+  step(gather_owner_rows(L->p2o, p2o, order, F, L->G, L->nown_max, L->p2_stride, stream));
   step(gather_f32(L->bias, order, F, bias, stream));
   step(gather_f32(L->thresh, order, F, thresh, stream));
   step(gather_f32(freq, order, F, fs, stream));
@@ -265,12 +297,19 @@ pi_status pi_reorder_hot_prefix(pi_layer* L, const float* freq, int hot_count, c
   step(cudaStreamSynchronize(stream));
   if (e != cudaSuccess) { cleanup(); return cuda_status(e); }
   std::swap(L->rec, rec);
-  std::swap(L->p2n, p2n);
+  std::swap(L->p2o, p2o);
   std::swap(L->bias, bias);
   std::swap(L->thresh, thresh);
   std::swap(L->freq_sorted, fs);
   std::swap(L->perm, perm);
   L->hot_count = hot_count;
+  float* fh = new (std::nothrow) float[F];
+  if (fh && cudaMemcpy(fh, L->freq_sorted, (size_t)F * 4, cudaMemcpyDeviceToHost) == cudaSuccess) {
+    delete[] L->freq_host;
+    L->freq_host = fh;
+  } else {
+    delete[] fh;
+  }
   cleanup();   // frees the old buffers now held in the temporaries
   return PI_OK;
 }
@@ -289,21 +328,28 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
   cudaGetDevice(&ws->device);
   ws->grid = sm_count(ws->device);
   if (ws->grid <= 0) { delete ws; return PI_ERR_CUDA; }
+  if (ws->grid > kMaxGrid) { delete ws; return PI_ERR_UNSUPPORTED; }
   const size_t G = ws->grid, Bm = B_max;
-  bool ok = dmalloc(&ws->u, Bm * r_max * 4) == cudaSuccess &&
-            dmalloc(&ws->maskbuf, 2 * Bm * (f_max / 32) * 4) == cudaSuccess &&
-            dmalloc(&ws->partials, G * Bm * d_max * 4) == cudaSuccess &&
-            dmalloc(&ws->v, Bm * d_max * 4) == cudaSuccess &&
-            dmalloc(&ws->xb, 2 * Bm * d_max * 4) == cudaSuccess &&
-            dmalloc(&ws->ssq, Bm * G * 4) == cudaSuccess &&
+  const size_t Wm = ((f_max + G - 1) / G + 31) / 32;   // bitmap words per block and token
+  bool ok = dmalloc(&ws->ux, Bm * r_max * 8) == cudaSuccess &&
+            dmalloc(&ws->px, G * Bm * d_max * 8) == cudaSuccess &&
+            dmalloc(&ws->vx, Bm * d_max * 8) == cudaSuccess &&
+            dmalloc(&ws->sx, Bm * G * 8) == cudaSuccess &&
+            dmalloc(&ws->bx, Bm * G * Wm * 8) == cudaSuccess &&
             dmalloc(&ws->bar, 64) == cudaSuccess &&
             dmalloc(&ws->err, 16) == cudaSuccess &&
             dmalloc(&ws->active_total, 16) == cudaSuccess &&
             dmalloc(&ws->layer_count, (size_t)L_max * 4) == cudaSuccess &&
             dmalloc(&ws->x_dev, Bm * d_max * 4) == cudaSuccess;
   if (ok) {
-    ok = cudaMemset(ws->bar, 0, 64) == cudaSuccess && cudaMemset(ws->err, 0, 16) == cudaSuccess &&
-         cudaMemset(ws->active_total, 0, 16) == cudaSuccess &&
+    // tagged words start with tag 0; launch epochs start at 1, so no stale word matches
+    const uint32_t bar0[4] = {0u, 0u, 1u, 0u};
+    ok = cudaMemset(ws->ux, 0, Bm * r_max * 8) == cudaSuccess && cudaMemset(ws->px, 0, G * Bm * d_max * 8) == cudaSuccess &&
+         cudaMemset(ws->vx, 0, Bm * d_max * 8) == cudaSuccess && cudaMemset(ws->sx, 0, Bm * G * 8) == cudaSuccess &&
+         cudaMemset(ws->bx, 0, Bm * G * Wm * 8) == cudaSuccess &&
+         cudaMemset(ws->bar, 0, 64) == cudaSuccess &&
+         cudaMemcpy(ws->bar, bar0, sizeof(bar0), cudaMemcpyHostToDevice) == cudaSuccess &&
+         cudaMemset(ws->err, 0, 16) == cudaSuccess && cudaMemset(ws->active_total, 0, 16) == cudaSuccess &&
          cudaMemset(ws->layer_count, 0, (size_t)L_max * 4) == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
   }
   if (!ok) {
@@ -317,9 +363,9 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
 
 void pi_workspace_free(pi_workspace* ws) {
   if (!ws) return;
-  cudaFree(ws->u); cudaFree(ws->maskbuf); cudaFree(ws->partials); cudaFree(ws->v); cudaFree(ws->xb);
-  cudaFree(ws->ssq); cudaFree(ws->bar); cudaFree(ws->err); cudaFree(ws->active_total);
-  cudaFree(ws->layer_count); cudaFree(ws->x_dev);
+  cudaFree(ws->ux); cudaFree(ws->px); cudaFree(ws->vx); cudaFree(ws->sx); cudaFree(ws->bx);
+  cudaFree(ws->bar); cudaFree(ws->err); cudaFree(ws->active_total);
+  cudaFree(ws->layer_count); cudaFree(ws->x_dev); cudaFree(ws->phase_clk);
   delete ws;
 }
 
@@ -329,8 +375,13 @@ pi_status pi_stream_status(pi_workspace* ws, cudaStream_t stream) {
   int err = 0;
   PI_TRY(cudaMemcpy(&err, ws->err, 4, cudaMemcpyDeviceToHost));
   if (err == 0) return PI_OK;
+  uint32_t bar[4];
+  PI_TRY(cudaMemcpy(bar, ws->bar, sizeof(bar), cudaMemcpyDeviceToHost));
+  bar[0] = 0u;
+  bar[1] = 0u;
+  bar[2] += 1u;   // fresh tags: nothing an aborted launch left behind can match
+  PI_TRY(cudaMemcpy(ws->bar, bar, sizeof(bar), cudaMemcpyHostToDevice));
   PI_TRY(cudaMemset(ws->err, 0, 16));
-  PI_TRY(cudaMemset(ws->bar, 0, 64));
   PI_TRY(cudaDeviceSynchronize());
   return (err == DEV_ERR_GRID_TIMEOUT || err == DEV_ERR_RING_TIMEOUT) ? PI_ERR_TIMEOUT : PI_ERR_DEVICE;
 }
@@ -363,7 +414,6 @@ pi_status pi_predict(const pi_layer* L, const void* x, int B, uint32_t* mask, fl
   p.x_in = x;
   p.mask_out = mask;
   p.logits_out = logits;
-  PI_TRY(cudaMemsetAsync(mask, 0, (size_t)B * (L->desc.d_ff / 32) * 4, stream));
   PI_TRY(launch_fused(L->family, L->desc.act, B, p, smem, stream));
   return PI_OK;
 }
@@ -412,11 +462,13 @@ pi_status pi_decode_stack(pi_layer* const* layers, int Lc, void* x_inout, int B,
   if (st != PI_OK) return st;
   p.mode = MODE_PREDICT | MODE_FFN | MODE_GLUE;
   p.L = Lc;
-  for (int l = 0; l < Lc; ++l) p.layers[l] = dev_view(layers[l]);
+  for (int l = 0; l < Lc; ++l) p.layers[l] = dev_view(layers[l], B);
   p.x_in = x_inout;
   p.x_out = x_inout;
   if (trace) p.trace = *trace;
   p.layer_count = ws->layer_count;
+  p.phase_clk = ws->phase_clk;
+  p.phase_global = ws->phase_global;
   PI_TRY(cudaMemsetAsync(ws->layer_count, 0, (size_t)Lc * 4, stream));
   PI_TRY(launch_fused(L0->family, L0->desc.act, B, p, smem, stream));
   return PI_OK;
@@ -433,6 +485,31 @@ pi_status pi_decode_stack_host(pi_layer* const* layers, int Lc, const void* x_ho
   PI_TRY(cudaMemcpyAsync(x_out_host, ws->x_dev, bytes, cudaMemcpyDeviceToHost, stream));
   return pi_stream_status(ws, stream);
 }
+
+pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on) {
+  if (!ws) return PI_ERR_ARG;
+  if (!on) {
+    cudaFree(ws->phase_clk);
+    ws->phase_clk = nullptr;
+    return PI_OK;
+  }
+  ws->phase_global = on == 2;
+  if (ws->phase_clk) return PI_OK;
+  const size_t n = (size_t)ws->grid * ws->L_max * 12;
+  if (dmalloc(&ws->phase_clk, n * sizeof(long long)) != cudaSuccess) return PI_ERR_OOM;
+  PI_TRY(cudaMemset(ws->phase_clk, 0, n * sizeof(long long)));
+  return PI_OK;
+}
+
+pi_status pi_diag_phase_clocks_read(pi_workspace* ws, long long* host_out, size_t n) {
+  if (!ws || !host_out || !ws->phase_clk) return PI_ERR_ARG;
+  const size_t total = (size_t)ws->grid * ws->L_max * 12;
+  if (n > total) return PI_ERR_ARG;
+  PI_TRY(cudaMemcpy(host_out, ws->phase_clk, n * sizeof(long long), cudaMemcpyDeviceToHost));
+  return PI_OK;
+}
+
+int pi_device_grid(pi_workspace* ws) { return ws ? ws->grid : 0; }
 
 pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaStream_t stream) {
   if (!ws || timeout_ns <= 0) return PI_ERR_ARG;

@@ -25,16 +25,18 @@ enum Family : int { FAM_F32 = 0, FAM_F16 = 1, FAM_Q4 = 2 };
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;
-constexpr int kMaxSlots = 48;
 constexpr int kMaxOwn = 512;          // owned neurons per block (d_ff <= 512 * grid)
 constexpr int kMaxList = 512;         // active neurons a block may process in one layer
-constexpr int kMaxLayers = 128;       // layers of one pi_decode_stack call
+constexpr int kMaxLayers = 100;       // layers of one pi_decode_stack call
+constexpr int kMaxGrid = 256;         // blocks of the fused kernel (SMs)
 
 // Library-owned, re-laid-out layer.
 struct LayerDev {
   const uint8_t* rec;     // [f][rec_stride]   per-neuron record [gate][up][down]
   const uint8_t* p1t;     // [r][p1_row]       P1 transposed, p_dtype
-  const uint8_t* p2n;     // [f][p2_stride]    per-neuron predictor row + (t, b) header
+  const uint8_t* p2o;     // [G][nown_max][p2_stride] predictor row + (t, b) of neuron c + m*G
+  int hot;                // hot-prefix length at this call's batch (L2 warm-up), 0 = none
+  int pad;
 };
 
 }  // namespace pi
@@ -45,15 +47,19 @@ struct pi_layer {
   int row_bytes;    // one weight row (d elements) in the record
   int rec_stride;   // bytes per neuron record (gate? + up + down), multiple of 16
   int gate_off, up_off, down_off;   // byte offsets of the rows in a record (gate_off -1 for ReLU)
+  int bias_off;     // byte offset of the record's 16-byte header holding the bias (f32)
   int p1_row;       // bytes of one P1^T row (d * p_bytes)
   int p2_stride;    // bytes per neuron predictor row (r * p_bytes + 8, rounded to 16)
+  int G;            // blocks the owner-major predictor layout was built for (the SM count)
+  int nown_max;     // ceil(f / G): predictor rows per block, padded
   uint8_t* rec;
   uint8_t* p1t;
-  uint8_t* p2n;
+  uint8_t* p2o;
   float* bias;      // [f] stored order
   float* thresh;    // [f] stored order
   int32_t* perm;    // [f] stored position -> original id
   float* freq_sorted;  // [f] firing frequency in stored order (after a reorder), else null
+  float* freq_host;    // host copy of freq_sorted (descending), or null
   int hot_count;    // -1: derived per batch from freq_sorted
   int device;
 };
@@ -62,17 +68,18 @@ struct pi_workspace {
   int d_max, f_max, r_max, B_max, L_max;
   int grid;          // blocks of the fused kernel (one per SM)
   int device;
-  float* u;          // [B_max][r_max]
-  uint32_t* maskbuf; // [2][B_max][f_max/32]
-  float* partials;   // [grid][B_max][d_max]
-  float* v;          // [B_max][d_max]
-  float* xb;         // [2][B_max][d_max]
-  float* ssq;        // [B_max][grid]
-  uint32_t* bar;     // [0] arrive counter, [1] exit counter (reset by the last block out)
+  uint64_t* ux;      // [B_max][r_max]          tagged u
+  uint64_t* px;      // [grid][B_max][d_max]    tagged y partials
+  uint64_t* vx;      // [B_max][d_max]          tagged x + y
+  uint64_t* sx;      // [B_max][grid]           tagged slice sums of squares
+  uint64_t* bx;      // [B_max][grid][W_max]    tagged own-neuron bitmaps
+  uint32_t* bar;     // [0] probe barrier count, [1] exit count, [2] launch epoch (tags)
   int* err;          // device error word
   unsigned long long* active_total;  // running sum of active-list lengths (all calls)
   int32_t* layer_count;              // [L_max] per-layer union active count of the last stack
   void* x_dev;       // [B_max][d_max] staging for pi_decode_stack_host (fp32 size)
+  long long* phase_clk;  // diagnostics: [grid][L_max][12] stamps, or null when off
+  int phase_global;      // 1: stamps from the global ns timer
   void* x_host_pinned;
 };
 
@@ -83,8 +90,8 @@ struct FusedParams {
   int mode;            // bit 1: predictor, bit 2: FFN, bit 4: stack glue (layer loop)
   int L, B, d, f, r;
   int grid;
-  int row_bytes, rec_stride, gate_off, up_off, down_off, p1_row, p2_stride;
-  int slot_bytes, nslots, rows_per_p2slot;
+  int row_bytes, rec_stride, gate_off, up_off, down_off, bias_off, p1_row, p2_stride;
+  int ring_bytes, p1_rows_per_item, p2_rows_per_item, nown_max, batch;
   int nslices;
   LayerDev layers[kMaxLayers];
   // inputs / outputs
@@ -98,26 +105,27 @@ struct FusedParams {
   float* y_out;              // [B][d] (ffn)
   pi_trace trace;            // (stack)
   // workspace
-  float* u;
-  uint32_t* maskbuf;
-  float* partials;
-  float* v;            // [B][d] x + y of the current layer
-  float* xb;           // [2][B][d] fp32 layer inputs, by layer parity
-  float* ssq;
+  uint64_t* ux;
+  uint64_t* px;
+  uint64_t* vx;
+  uint64_t* sx;
+  uint64_t* bx;              // [B][G][W] tagged bitmaps of the blocks' own neurons
   uint32_t* bar;
   int* err;
   unsigned long long* active_total;
   int32_t* layer_count;
   long long barrier_timeout_ns;
   int barrier_extra;   // added to the barrier target (diagnostics: forces a timeout)
+  long long* phase_clk;  // diagnostics: SM cycle stamps per block, layer and phase, or null
+  int phase_global;      // stamps from the global ns timer instead of the SM cycle counter
 };
 
 enum : int { MODE_PREDICT = 1, MODE_FFN = 2, MODE_GLUE = 4 };
 
 cudaError_t launch_fused(int family, int act, int B, const FusedParams& p, size_t smem_bytes,
                          cudaStream_t stream);
-size_t fused_smem_bytes(const FusedParams& p);
-size_t fused_fixed_smem(int B, int r);
+size_t fused_fixed_smem(int B, int d, int r, int grid, int nown_max, int family);
+int fused_max_batch();
 bool fused_supported(int family, int B, int d);
 cudaError_t launch_barrier_probe(const FusedParams& p, int rounds, cudaStream_t stream);
 

@@ -11,10 +11,17 @@ namespace pi {
 
 namespace {
 
-// dst row c gets src column c: dst[c * dst_stride + dst_off + r * sizeof(T)] = src[r * src_ld + c]
+// Row of neuron n in the owner-major predictor layout: block n % G, position n / G.
+__device__ __forceinline__ long long owner_row(int n, int G, int nmax) {
+  return G > 0 ? (long long)(n % G) * nmax + n / G : (long long)n;
+}
+
+// dst row c gets src column c: dst[row(c) * dst_stride + dst_off + r * sizeof(T)] = src[r * src_ld + c]
+// (row(c) = c, or the owner-major row when G > 0)
 template <typename T>
 __global__ void transpose_kernel(const T* __restrict__ src, int rows, int cols, long long src_ld,
-                                 uint8_t* __restrict__ dst, long long dst_stride, long long dst_off) {
+                                 uint8_t* __restrict__ dst, long long dst_stride, long long dst_off,
+                                 int G, int nmax) {
   __shared__ T tile[32][33];
   const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
   for (int k = threadIdx.y; k < 32; k += blockDim.y) {
@@ -25,7 +32,8 @@ __global__ void transpose_kernel(const T* __restrict__ src, int rows, int cols, 
   for (int k = threadIdx.y; k < 32; k += blockDim.y) {
     const int c = c0 + k, r = r0 + threadIdx.x;
     if (r < rows && c < cols)
-      *reinterpret_cast<T*>(dst + (long long)c * dst_stride + dst_off + (long long)r * sizeof(T)) = tile[threadIdx.x][k];
+      *reinterpret_cast<T*>(dst + owner_row(c, G, nmax) * dst_stride + dst_off + (long long)r * sizeof(T)) =
+          tile[threadIdx.x][k];
   }
 }
 
@@ -49,12 +57,29 @@ __global__ void copy_rows_kernel(const uint8_t* __restrict__ src, long long src_
 
 // per-neuron predictor header: (t_i, b_i) after the r predictor values
 __global__ void p2_header_kernel(const float* __restrict__ thresh, const float* __restrict__ bias, int f,
-                                 uint8_t* __restrict__ p2n, int p2_stride, int hdr_off) {
+                                 uint8_t* __restrict__ p2o, int p2_stride, int hdr_off, int G, int nmax) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= f) return;
-  float* h = reinterpret_cast<float*>(p2n + (long long)i * p2_stride + hdr_off);
+  float* h = reinterpret_cast<float*>(p2o + owner_row(i, G, nmax) * p2_stride + hdr_off);
   h[0] = thresh[i];
   h[1] = bias[i];
+}
+
+// one float per row: dst + i*stride + off <- v[i]
+__global__ void row_scalar_kernel(const float* __restrict__ v, int f, uint8_t* __restrict__ dst, long long stride,
+                                  long long off) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < f) *reinterpret_cast<float*>(dst + (long long)i * stride + off) = v[i];
+}
+
+// owner-major rows permuted by neuron: dst row(n) <- src row(order[n])
+__global__ void gather_owner_rows_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst,
+                                         const int32_t* __restrict__ order, int f, int G, int nmax, int stride) {
+  const int n = blockIdx.x;
+  if (n >= f) return;
+  const uint4* s = reinterpret_cast<const uint4*>(src + owner_row(order[n], G, nmax) * stride);
+  uint4* d = reinterpret_cast<uint4*>(dst + owner_row(n, G, nmax) * stride);
+  for (int k = threadIdx.x; k < stride / 16; k += blockDim.x) d[k] = s[k];
 }
 
 __global__ void gather_f32_kernel(const float* __restrict__ src, const int32_t* __restrict__ order, int n,
@@ -149,14 +174,15 @@ __global__ void __launch_bounds__(1024) compact_kernel(const uint32_t* __restric
 static dim3 tgrid(int rows, int cols) { return dim3((cols + 31) / 32, (rows + 31) / 32); }
 
 cudaError_t relayout_transpose(const void* src, int esize, int rows, int cols, long long src_ld,
-                               uint8_t* dst, long long dst_stride, long long dst_off, cudaStream_t s) {
+                               uint8_t* dst, long long dst_stride, long long dst_off, cudaStream_t s,
+                               int G, int nmax) {
   const dim3 blk(32, 8);
   if (esize == 4)
     transpose_kernel<uint32_t><<<tgrid(rows, cols), blk, 0, s>>>(static_cast<const uint32_t*>(src), rows, cols,
-                                                                  src_ld, dst, dst_stride, dst_off);
+                                                                  src_ld, dst, dst_stride, dst_off, G, nmax);
   else if (esize == 2)
     transpose_kernel<uint16_t><<<tgrid(rows, cols), blk, 0, s>>>(static_cast<const uint16_t*>(src), rows, cols,
-                                                                  src_ld, dst, dst_stride, dst_off);
+                                                                  src_ld, dst, dst_stride, dst_off, G, nmax);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
@@ -171,9 +197,20 @@ cudaError_t relayout_copy_rows(const void* src, long long src_stride, long long 
   return cudaGetLastError();
 }
 
-cudaError_t relayout_p2_header(const float* thresh, const float* bias, int f, uint8_t* p2n, int p2_stride,
-                               int hdr_off, cudaStream_t s) {
-  p2_header_kernel<<<(f + 255) / 256, 256, 0, s>>>(thresh, bias, f, p2n, p2_stride, hdr_off);
+cudaError_t relayout_p2_header(const float* thresh, const float* bias, int f, uint8_t* p2o, int p2_stride,
+                               int hdr_off, int G, int nmax, cudaStream_t s) {
+  p2_header_kernel<<<(f + 255) / 256, 256, 0, s>>>(thresh, bias, f, p2o, p2_stride, hdr_off, G, nmax);
+  return cudaGetLastError();
+}
+
+cudaError_t relayout_row_scalar(const float* v, int f, uint8_t* dst, long long stride, long long off, cudaStream_t s) {
+  row_scalar_kernel<<<(f + 255) / 256, 256, 0, s>>>(v, f, dst, stride, off);
+  return cudaGetLastError();
+}
+
+cudaError_t gather_owner_rows(const uint8_t* src, uint8_t* dst, const int32_t* order, int f, int G, int nmax,
+                              int stride, cudaStream_t s) {
+  gather_owner_rows_kernel<<<f, 128, 0, s>>>(src, dst, order, f, G, nmax, stride);
   return cudaGetLastError();
 }
 

@@ -195,6 +195,22 @@ pi_status pi_workspace_layer_counts(pi_workspace* ws, int32_t* host_out, int L);
  * device-side wait ends without hanging the GPU. */
 pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaStream_t stream);
 
+/* Diagnostic: with `on`, every later pi_decode_stack on this workspace records each
+ * block's SM cycle counter at 12 points of every layer. The consumer warps record 0-8:
+ * layer start, predictor rows done, after the first grid barrier, own active list ready,
+ * FFN done, after the second barrier, slice reduce done, after the third barrier, and
+ * glue done. The producer warp records 9-11: waiting for the active list, list
+ * received, and all of the layer's weight rows issued. With `on` = 2 the stamps come from
+ * the GPU's global nanosecond timer instead, so blocks can be compared with one another.
+ * With `on` = 0 recording stops and the buffer is freed. */
+pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on);
+
+/* Copy the first n stamps ([grid][L_max][12], int64 cycles) to host memory (synchronous). */
+pi_status pi_diag_phase_clocks_read(pi_workspace* ws, long long* host_out, size_t n);
+
+/* Blocks per launch of the fused kernel on this workspace's device (its SM count). */
+int pi_device_grid(pi_workspace* ws);
+
 /* ---------------------------------------------------------------- hot path */
 
 /* Predictor. x: device [B][d] in x_dtype. mask: device u32 [B][f/32].
