@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 
@@ -114,7 +115,18 @@ pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedPara
   p.bar = ws->bar; p.err = ws->err; p.active_total = ws->active_total;
   p.layer_count = nullptr;
   p.barrier_timeout_ns = kDefaultWaitNs;
+  p.wait_cycles = kDefaultWaitNs * 3;   // cycles at up to 3 GHz: at least the nominal budget
   p.barrier_extra = 0;
+  static const unsigned poll_ns = [] {
+    const char* e = std::getenv("PI_POLL_NS");   // tuning knob for the exchange back-off
+    return e ? (unsigned)std::strtoul(e, nullptr, 10) : 64u;
+  }();
+  p.poll_ns = poll_ns;
+  static const int gate = [] {
+    const char* e = std::getenv("PI_GATE_PRODUCER");
+    return e ? std::atoi(e) : 0;
+  }();
+  p.gate_producer = gate;
   return PI_OK;
 }
 
@@ -334,7 +346,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
   bool ok = dmalloc(&ws->ux, Bm * r_max * 8) == cudaSuccess &&
             dmalloc(&ws->px, G * Bm * d_max * 8) == cudaSuccess &&
             dmalloc(&ws->vx, Bm * d_max * 8) == cudaSuccess &&
-            dmalloc(&ws->sx, Bm * G * 8) == cudaSuccess &&
+            dmalloc(&ws->sx, Bm * G * 16) == cudaSuccess &&
             dmalloc(&ws->bx, Bm * G * Wm * 8) == cudaSuccess &&
             dmalloc(&ws->bar, 64) == cudaSuccess &&
             dmalloc(&ws->err, 16) == cudaSuccess &&
@@ -345,7 +357,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
     // tagged words start with tag 0; launch epochs start at 1, so no stale word matches
     const uint32_t bar0[4] = {0u, 0u, 1u, 0u};
     ok = cudaMemset(ws->ux, 0, Bm * r_max * 8) == cudaSuccess && cudaMemset(ws->px, 0, G * Bm * d_max * 8) == cudaSuccess &&
-         cudaMemset(ws->vx, 0, Bm * d_max * 8) == cudaSuccess && cudaMemset(ws->sx, 0, Bm * G * 8) == cudaSuccess &&
+         cudaMemset(ws->vx, 0, Bm * d_max * 8) == cudaSuccess && cudaMemset(ws->sx, 0, Bm * G * 16) == cudaSuccess &&
          cudaMemset(ws->bx, 0, Bm * G * Wm * 8) == cudaSuccess &&
          cudaMemset(ws->bar, 0, 64) == cudaSuccess &&
          cudaMemcpy(ws->bar, bar0, sizeof(bar0), cudaMemcpyHostToDevice) == cudaSuccess &&
@@ -495,7 +507,7 @@ pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on) {
   }
   ws->phase_global = on == 2;
   if (ws->phase_clk) return PI_OK;
-  const size_t n = (size_t)ws->grid * ws->L_max * 12;
+  const size_t n = (size_t)ws->grid * ws->L_max * 16;
   if (dmalloc(&ws->phase_clk, n * sizeof(long long)) != cudaSuccess) return PI_ERR_OOM;
   PI_TRY(cudaMemset(ws->phase_clk, 0, n * sizeof(long long)));
   return PI_OK;
@@ -503,7 +515,7 @@ pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on) {
 
 pi_status pi_diag_phase_clocks_read(pi_workspace* ws, long long* host_out, size_t n) {
   if (!ws || !host_out || !ws->phase_clk) return PI_ERR_ARG;
-  const size_t total = (size_t)ws->grid * ws->L_max * 12;
+  const size_t total = (size_t)ws->grid * ws->L_max * 16;
   if (n > total) return PI_ERR_ARG;
   PI_TRY(cudaMemcpy(host_out, ws->phase_clk, n * sizeof(long long), cudaMemcpyDeviceToHost));
   return PI_OK;
@@ -519,6 +531,7 @@ pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaSt
   p.bar = ws->bar;
   p.err = ws->err;
   p.barrier_timeout_ns = timeout_ns;
+  p.wait_cycles = timeout_ns * 2;   // SM cycles, about 2 per ns
   p.barrier_extra = 1;   // one arrival more than the grid has: no wait can complete
   PI_TRY(launch_barrier_probe(p, 2, stream));
   return PI_OK;

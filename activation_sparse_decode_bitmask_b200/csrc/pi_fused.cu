@@ -20,8 +20,9 @@
 //        then all threads add h * w_down_i into y (registers, fp32, one thread per 16 B)
 //        -> partial exchange
 //   R    block s < nslices owns a column slice: v = x + sum_c partial_c in ascending c,
-//        and the slice's sum of squares -> v / ssq exchange
-//   glue x' = v / sqrt(sum_s ssq_s / d + 1e-6), rounded to the activation dtype
+//        and the slice's sum and sum of squares -> v / moments exchange
+//   glue x' = (v - mean(v)) / sqrt(var(v) + 1e-6) from the slices' sums and sums of
+//        squares, rounded to the activation dtype
 // Cross-block exchanges use 64-bit words {tag, value}: a reader polls the words
 // themselves until every tag matches, so data and completion arrive together and no grid
 // barrier is needed.  Tags are unique per launch (a device epoch advanced by the last
@@ -55,8 +56,10 @@ struct Smem {
   int pad;
   uint32_t item_pos[kItems];   // producer bookkeeping of items in flight
   uint32_t item_size[kItems];
-  float rms[4];
-  float hbuf[2][kMaxBatch][4];
+  float gmean[4];   // glue: mean and standard deviation of v per token
+  float gsd[4];
+  float hbuf[kMaxList][4];      // h of the layer's records, by list position
+  int hflag[kMaxList];          // = layer + 1 once hbuf[e] is written
   int32_t list[kMaxList];
   uint8_t list_bits[kMaxList];
   uint8_t own_bits[kMaxOwn];
@@ -65,7 +68,7 @@ struct Smem {
 };
 
 // Diagnostics: SM cycle stamps at phase boundaries, [block][layer][kPhases].
-constexpr int kPhases = 12;
+constexpr int kPhases = 16;
 __device__ __forceinline__ long long stamp_now(const FusedParams& p) {
   return p.phase_global ? (long long)globaltimer_ns() : clock64();
 }
@@ -77,8 +80,11 @@ __device__ __forceinline__ void pstamp(const FusedParams& p, int l, int ph) {
   if (p.phase_clk) p.phase_clk[((size_t)blockIdx.x * p.L + l) * kPhases + ph] = stamp_now(p);
 }
 
+// Bounded waits count SM cycles (clock64 is cheap to read; the global timer is not):
+// `limit` is the wait budget converted to cycles at an upper bound of the SM clock.
+__device__ __forceinline__ uint64_t wait_start() { return (uint64_t)clock64(); }
 __device__ __forceinline__ bool timed_out(uint64_t t0, long long limit) {
-  return (long long)(globaltimer_ns() - t0) > limit;
+  return (long long)((uint64_t)clock64() - t0) > limit;
 }
 __device__ __forceinline__ void set_abort(Smem& sm, int* err, int code) {
   atomicExch(err, code);
@@ -133,12 +139,13 @@ __device__ __forceinline__ void poll_words(const uint64_t* base, int first, int 
       }
     if (!need || aborted(sm)) break;
     if (!started) {
-      t0 = globaltimer_ns();
+      t0 = wait_start();
       started = true;
-    } else if (timed_out(t0, p.barrier_timeout_ns)) {
+    } else if (timed_out(t0, p.wait_cycles)) {
       set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT);
       break;
     }
+    if (p.poll_ns) __nanosleep(p.poll_ns);   // back off: many blocks poll the same lines
   }
 }
 
@@ -164,10 +171,10 @@ __device__ __forceinline__ void ring_wait_item(uint32_t item, Smem& sm, const Fu
   uint64_t* bar = &sm.full[item % kItems];
   const uint32_t par = (item / kItems) & 1u;
   if (!aborted(sm) && !mbar_try_wait(bar, par)) {
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = wait_start();
     while (!mbar_try_wait(bar, par)) {
       if (aborted(sm)) break;
-      if (timed_out(t0, p.barrier_timeout_ns)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); break; }
+      if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); break; }
     }
   }
 }
@@ -233,6 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     }
     mbar_init(&sm.list_ready, 1);
     mbar_init(&sm.layer_start, 1);
+    for (int e = 0; e < kMaxList; ++e) sm.hflag[e] = 0;
     sm.abort_flag = 0;
     sm.nlist = 0;
     mbar_fence_init();
@@ -259,10 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           uint64_t* eb = &sm.empty[oldest % kItems];
           const uint32_t par = (oldest / kItems) & 1u;
           if (!mbar_try_wait(eb, par)) {
-            const uint64_t t0 = globaltimer_ns();
+            const uint64_t t0 = wait_start();
             while (!mbar_try_wait(eb, par)) {
               if (aborted(sm)) return false;
-              if (timed_out(t0, p.barrier_timeout_ns)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); return false; }
+              if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); return false; }
             }
           }
           ++oldest;
@@ -285,6 +293,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         const LayerDev Ld = p.layers[l];
         uint8_t* dst;
         uint64_t* fb;
+        if (do_pred && p.gate_producer && l > 0) {
+          // experiment: keep the producer quiet until the consumers start this layer
+          const uint64_t t0 = wait_start();
+          while (!mbar_try_wait(&sm.layer_start, (uint32_t)(l & 1))) {
+            if (aborted(sm)) { ok = false; break; }
+            if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
+          }
+        }
         if (do_pred) {
           for (int k = k0; k < k1 && ok; k += p.p1_rows_per_item) {
             const int n = min(p.p1_rows_per_item, k1 - k);
@@ -300,26 +316,36 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
             bulk_g2s(dst, own + (size_t)m * p.p2_stride, bytes, fb);
           }
         }
-        if (do_ffn && ok && Ld.hot > 0) {
-          // When the consumers start this layer, the HBM is idle until the active list is
-          // known: warm L2 with this block's own hot-prefix records, which most likely fire.
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(&sm.layer_start, (uint32_t)(l & 1))) {
-            if (aborted(sm)) { ok = false; break; }
-            if (timed_out(t0, p.barrier_timeout_ns)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
-          }
-          for (int i = c; i < Ld.hot && ok; i += G) prefetch_l2_bulk(Ld.rec + (size_t)i * p.rec_stride, (uint32_t)p.rec_stride);
-        }
         if (do_ffn && ok) {
           pstamp(p, l, 9);
-          const uint64_t t0 = globaltimer_ns();
+          const uint64_t t0 = wait_start();
           while (!mbar_try_wait(&sm.list_ready, (uint32_t)(l & 1))) {
             if (aborted(sm)) { ok = false; break; }
-            if (timed_out(t0, p.barrier_timeout_ns)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
+            if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
           }
           pstamp(p, l, 10);
           const int n = ok ? sm.nlist : 0;
-          for (int e = 0; e < n && ok; ++e) {
+          // Ask HBM for every record of the block at once (L2 prefetch needs no shared
+          // memory); the ring copies below then find them in L2 as space frees up.
+          for (int e = 0; e < n && ok; ++e)
+            prefetch_l2_bulk(Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride);
+          // Warm L2 with the next layer's predictor rows of this block while this layer's
+          // records stream: that bulk traffic then lands in the F phase instead of slowing
+          // the cross-block exchanges that follow it, and the ring copies of those rows
+          // later come from L2.  The prefetches are issued after the first records.
+          const bool warm = do_pred && l + 1 < p.L;
+          const int first_recs = min(n, 2);
+          for (int e = 0; e < first_recs && ok; ++e) {
+            if (!(ok = begin_item((uint32_t)p.rec_stride, dst, fb))) break;
+            bulk_g2s(dst, Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride, fb);
+          }
+          if (warm && ok) {
+            const LayerDev Ln = p.layers[l + 1];
+            if (k1 > k0) prefetch_l2_bulk(Ln.p1t + (size_t)k0 * p.p1_row, (uint32_t)(k1 - k0) * p.p1_row);
+            if (nown > 0)
+              prefetch_l2_bulk(Ln.p2o + (size_t)c * p.nown_max * p.p2_stride, (uint32_t)nown * p.p2_stride);
+          }
+          for (int e = first_recs; e < n && ok; ++e) {
             if (!(ok = begin_item((uint32_t)p.rec_stride, dst, fb))) break;
             bulk_g2s(dst, Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride, fb);
           }
@@ -331,9 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       for (uint32_t s = first; s < issued; ++s) {
         uint64_t* fb = &sm.full[s % kItems];
         const uint32_t par = (s / kItems) & 1u;
-        const uint64_t t0 = globaltimer_ns();
+        const uint64_t t0 = wait_start();
         while (!mbar_try_wait(fb, par)) {
-          if (timed_out(t0, p.barrier_timeout_ns)) { atomicExch(p.err, DEV_ERR_RING_TIMEOUT); break; }
+          if (timed_out(t0, p.wait_cycles)) { atomicExch(p.err, DEV_ERR_RING_TIMEOUT); break; }
         }
       }
     }
@@ -382,6 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         const int n = min(p.p1_rows_per_item, k1 - k);
         const uint8_t* item = ring_next(ring, (uint32_t)n * p.p1_row);
         ring_wait_item(ring.item, sm, p);
+        if (k == k0) stamp(p, l, 13);
         for (int kk = warp; kk < n; kk += kConsumerWarps) {
           float acc[NB];
           warp_dot_p<FAM, NB>(item + (size_t)kk * p.p1_row, xs, d, acc);
@@ -413,6 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         const int n = min(p.p2_rows_per_item, nown - m0);
         const uint8_t* item = ring_next(ring, (uint32_t)n * p.p2_stride);
         ring_wait_item(ring.item, sm, p);
+        if (m0 == 0) stamp(p, l, 12);
         for (int mb = warp * 4; mb < n; mb += kConsumerWarps * 4) {
           float acc[4][NB];
 #pragma unroll
@@ -647,7 +675,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       for (int j = 0; j < NU; ++j)
 #pragma unroll
         for (int e = 0; e < UE; ++e) y[b][j][e] = 0.f;
-    int hb = 0;
+    // Records stream through the ring in windows of p.batch; warp k of a window forms the
+    // dot products of its record and flags h, and every warp adds each record's down row
+    // as soon as that record's h is flagged (no block-wide barrier in between).
+    const int hval = l + 1;
     for (int e0 = 0; e0 < nlist; e0 += p.batch) {
       const int nb = min(p.batch, nlist - e0);
       uint32_t rpos[kMaxBatch];
@@ -655,7 +686,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
 #pragma unroll
       for (int k = 0; k < kMaxBatch; ++k)
         rpos[k] = (k < nb) ? (uint32_t)(ring_next(ring, (uint32_t)p.rec_stride) - ring.base) : 0u;
-      // dots: warp k handles record k of the batch
       if (warp < nb) {
         uint32_t pos = rpos[0];
 #pragma unroll
@@ -678,25 +708,34 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
             float a;
             if constexpr (ACT == PI_REGLU) a = fmaxf(ga[b] + bi, 0.f) * ua[b];
             else a = fmaxf(ua[b] + bi, 0.f);
-            sm.hbuf[hb][warp][b] = ((bits >> b) & 1u) ? a : 0.f;
+            sm.hbuf[e][b] = ((bits >> b) & 1u) ? a : 0.f;
           }
+          __threadfence_block();
+          *(volatile int*)&sm.hflag[e] = hval;
         }
+        __syncwarp();
       }
-      named_bar_sync(kRedBar, kConsumerThreads);
-      // down: every thread adds h * w_down for its units, records in list order
       for (int k = 0; k < nb; ++k) {
         uint32_t pos = rpos[0];
 #pragma unroll
         for (int kk = 1; kk < kMaxBatch; ++kk) if (k == kk) pos = rpos[kk];
+        const int e = e0 + k;
+        if (*(volatile int*)&sm.hflag[e] != hval) {
+          const uint64_t t0 = wait_start();
+          while (*(volatile int*)&sm.hflag[e] != hval) {
+            if (aborted(sm)) break;
+            if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); break; }
+          }
+        }
+        __threadfence_block();
         ring_wait_item(item0 + k, sm, p);   // completed already: makes the data visible here
         float h[NB];
 #pragma unroll
-        for (int b = 0; b < NB; ++b) h[b] = sm.hbuf[hb][k][b];
+        for (int b = 0; b < NB; ++b) h[b] = sm.hbuf[e][b];
         axpy_units<FAM, NB, NU>(ring.base + pos + p.down_off, nunits, d, h, y);
         ring_release_item(item0 + k, sm);
       }
       ring.item = item0 + nb;
-      hb ^= 1;
     }
     // publish the partial y of this block as tagged words
     {
@@ -725,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       for (int b = 0; b < NB; ++b)
 #pragma unroll
         for (int gq = 0; gq < kMaxColGroups; ++gq) acc[b][gq] = 0.f;
-      const uint64_t t0 = globaltimer_ns();
+      const uint64_t t0 = wait_start();
       for (int gq = 0; gq < ng; ++gq) {
         for (int cc0 = warp; cc0 < G; cc0 += kConsumerWarps * KU) {
           float tmp[KU][NB];
@@ -748,7 +787,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
                   if (tag_ok(w, tag_p)) { tmp[k][b] = tag_val(w); need &= ~(1u << (k * NB + b)); }
                 }
             if (need && aborted(sm)) break;
-            if (need && timed_out(t0, p.barrier_timeout_ns)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+            if (need && timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+            if (need && p.poll_ns) __nanosleep(p.poll_ns);
           }
 #pragma unroll
           for (int k = 0; k < KU; ++k)
@@ -765,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       // warp b finishes token b's columns, summing the warps' parts in a fixed order
       if (warp < NB && warp < B) {
         const int b = warp;
-        float sq = 0.f;
+        float sq = 0.f, sv = 0.f;
 #pragma unroll
         for (int gq = 0; gq < kMaxColGroups; ++gq) {
           if (gq < ng) {
@@ -777,6 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
               const float vv = xsl[gq] + yv;
               xsl[gq] = vv;   // holds v until the glue turns it into the next input
               sq += vv * vv;
+              sv += vv;
               st_tag(p.vx + (size_t)b * d + j, vv, tag_v);
               if (p.trace.y) p.trace.y[((size_t)l * B + b) * d + j] = yv;
             } else {
@@ -786,7 +827,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         }
         if (do_glue) {
           sq = warp_sum(sq);
-          if (lane == 0) st_tag(p.sx + (size_t)b * G + c, sq, tag_v);
+          sv = warp_sum(sv);
+          if (lane == 0) {
+            st_tag(p.sx + ((size_t)b * G + c) * 2, sv, tag_v);
+            st_tag(p.sx + ((size_t)b * G + c) * 2 + 1, sq, tag_v);
+          }
         }
       }
     }
@@ -797,15 +842,24 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     {
       if (warp < NB) {
         float s = 0.f;
+        float s2 = 0.f;
         if (warp < B) {
-          uint64_t w[kMaxGrid / 32];
-          poll_words<kMaxGrid / 32>(p.sx + (size_t)warp * G, lane, 32, nslices, tag_v, w, sm, p);
+          // words (sum, sum of squares) of every slice, interleaved: even lanes read sums,
+          // odd lanes sums of squares (32 is even, so a lane keeps its parity)
+          uint64_t w[2 * kMaxGrid / 32];
+          poll_words<2 * kMaxGrid / 32>(p.sx + (size_t)warp * G * 2, lane, 32, 2 * nslices, tag_v, w, sm, p);
 #pragma unroll
-          for (int k = 0; k < kMaxGrid / 32; ++k)
-            if (lane + 32 * k < nslices) s += tag_val(w[k]);
+          for (int k = 0; k < 2 * kMaxGrid / 32; ++k)
+            if (lane + 32 * k < 2 * nslices) s += tag_val(w[k]);
         }
-        s = warp_sum(s);
-        if (lane == 0) sm.rms[warp] = sqrtf(s / (float)d + kRmsEps);
+        const float sum = warp_sum((lane & 1) ? 0.f : s);
+        s2 = warp_sum((lane & 1) ? s : 0.f);
+        if (lane == 0) {
+          const float mean = sum / (float)d;
+          const float var = fmaxf(s2 / (float)d - mean * mean, 0.f);
+          sm.gmean[warp] = mean;
+          sm.gsd[warp] = sqrtf(var + kRmsEps);
+        }
       }
       named_bar_sync(kRedBar, kConsumerThreads);   // rms known; every warp is done reading xs
       {
@@ -828,17 +882,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
                 if (tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
               }
             if (!need || aborted(sm)) break;
-            if (!started) { tp = globaltimer_ns(); started = true; }
-            else if (timed_out(tp, p.barrier_timeout_ns)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+            if (!started) { tp = wait_start(); started = true; }
+            else if (timed_out(tp, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+            if (p.poll_ns) __nanosleep(p.poll_ns);
           }
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const int pr = base + t + k * kConsumerThreads;
             if (pr < npairs) {
               const int idx = 2 * pr, b = idx / d;
-              const float rms = sm.rms[b];
-              xs[idx] = XT(round_act<FAM>(tag_val(w0[k]) / rms));
-              xs[idx + 1] = XT(round_act<FAM>(tag_val(w1[k]) / rms));
+              const float mean = sm.gmean[b], sd = sm.gsd[b];
+              xs[idx] = XT(round_act<FAM>((tag_val(w0[k]) - mean) / sd));
+              xs[idx + 1] = XT(round_act<FAM>((tag_val(w1[k]) - mean) / sd));
             }
           }
         }
@@ -846,12 +901,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       // slice owners: the new input of their slice, the trace, and the output
       if (slice_owner && warp < NB && warp < B) {
         const int b = warp;
-        const float rms = sm.rms[b];
+        const float mean = sm.gmean[b], sd = sm.gsd[b];
 #pragma unroll
         for (int gq = 0; gq < kMaxColGroups; ++gq)
           if (gq < ng) {
             const size_t j = (size_t)b * d + col0 + 32 * gq + lane;
-            xsl[gq] = round_act<FAM>(xsl[gq] / rms);
+            xsl[gq] = round_act<FAM>((xsl[gq] - mean) / sd);
             if (p.trace.x) store_act<FAM>(p.trace.x, (size_t)(l + 1) * B * d + j, xsl[gq]);
             if (l == p.L - 1) store_act<FAM>(p.x_out, j, xsl[gq]);
           }
@@ -888,9 +943,9 @@ __global__ void __launch_bounds__(kThreads, 1) barrier_probe_kernel(const FusedP
     if (threadIdx.x == 0 && !abort_flag) {
       const uint32_t target = epoch * (uint32_t)gridDim.x + (uint32_t)p.barrier_extra;
       red_release_gpu_add(p.bar, 1u);
-      const uint64_t t0 = globaltimer_ns();
+      const uint64_t t0 = wait_start();
       while (ld_acquire_gpu(p.bar) < target) {
-        if (timed_out(t0, p.barrier_timeout_ns)) {
+        if (timed_out(t0, p.wait_cycles)) {
           atomicExch(p.err, DEV_ERR_GRID_TIMEOUT);
           abort_flag = 1;
           break;

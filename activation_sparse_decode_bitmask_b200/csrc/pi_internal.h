@@ -71,7 +71,7 @@ struct pi_workspace {
   uint64_t* ux;      // [B_max][r_max]          tagged u
   uint64_t* px;      // [grid][B_max][d_max]    tagged y partials
   uint64_t* vx;      // [B_max][d_max]          tagged x + y
-  uint64_t* sx;      // [B_max][grid]           tagged slice sums of squares
+  uint64_t* sx;      // [B_max][grid][2]        tagged slice sums and sums of squares
   uint64_t* bx;      // [B_max][grid][W_max]    tagged own-neuron bitmaps
   uint32_t* bar;     // [0] probe barrier count, [1] exit count, [2] launch epoch (tags)
   int* err;          // device error word
@@ -114,10 +114,13 @@ struct FusedParams {
   int* err;
   unsigned long long* active_total;
   int32_t* layer_count;
-  long long barrier_timeout_ns;
+  long long barrier_timeout_ns;   // grid-barrier probe wait budget (global timer)
+  long long wait_cycles;          // fused-kernel wait budget in SM cycles
   int barrier_extra;   // added to the barrier target (diagnostics: forces a timeout)
   long long* phase_clk;  // diagnostics: SM cycle stamps per block, layer and phase, or null
   int phase_global;      // stamps from the global ns timer instead of the SM cycle counter
+  unsigned poll_ns;      // back-off between polling rounds of the cross-block exchanges
+  int gate_producer;     // 1: the producer starts a layer's copies only when the consumers do
 };
 
 enum : int { MODE_PREDICT = 1, MODE_FFN = 2, MODE_GLUE = 4 };

@@ -25,9 +25,9 @@
  *   ReGLU:  a_i = max(0, w_gate_i . x + b_i) * (w_up_i . x)
  *   a[b,i] = 0 where token b's own bit is 0
  *   y_j     = sum over active i of W_down[j,i] * a_i          (fp32 accumulation)
- *   stack:  x' = (x + y) / sqrt(mean((x + y)^2) + 1e-6), in fp32, stored in the
- *           activation dtype. The pages have no layer stack; this residual + RMS
- *           normalisation is this library's reading.
+ *   stack:  v = x + y;  x' = (v - mean(v)) / sqrt(var(v) + 1e-6), in fp32, stored in
+ *           the activation dtype. The pages have no layer stack; this residual plus a
+ *           mean-centred normalisation is this library's reading.
  *
  * Conventions
  *   - Every call returns a pi_status. PI_OK is 0.
@@ -123,7 +123,7 @@ typedef struct pi_workspace pi_workspace;
  *   mask   [L][B][f/32] u32
  *   idx    [L][f] i32; only the first count[l] entries of layer l are written
  *   count  [L] i32
- *   y      [L][B][d] f32, the FFN output before the residual and normalisation */
+ *   y      [L][B][d] f32, the FFN output before the residual and the normalisation */
 typedef struct {
   void* x;
   float* logits;
@@ -196,16 +196,17 @@ pi_status pi_workspace_layer_counts(pi_workspace* ws, int32_t* host_out, int L);
 pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaStream_t stream);
 
 /* Diagnostic: with `on`, every later pi_decode_stack on this workspace records each
- * block's SM cycle counter at 12 points of every layer. The consumer warps record 0-8:
+ * block's SM cycle counter at 16 points of every layer. The consumer warps record 0-8:
  * layer start, predictor rows done, after the first grid barrier, own active list ready,
  * FFN done, after the second barrier, slice reduce done, after the third barrier, and
  * glue done. The producer warp records 9-11: waiting for the active list, list
- * received, and all of the layer's weight rows issued. With `on` = 2 the stamps come from
+ * received, and all of the layer's weight rows issued; 12 and 13 mark the first
+ * predictor item landing (P2, P1). With `on` = 2 the stamps come from
  * the GPU's global nanosecond timer instead, so blocks can be compared with one another.
  * With `on` = 0 recording stops and the buffer is freed. */
 pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on);
 
-/* Copy the first n stamps ([grid][L_max][12], int64 cycles) to host memory (synchronous). */
+/* Copy the first n stamps ([grid][L_max][16], int64) to host memory (synchronous). */
 pi_status pi_diag_phase_clocks_read(pi_workspace* ws, long long* host_out, size_t n);
 
 /* Blocks per launch of the fused kernel on this workspace's device (its SM count). */

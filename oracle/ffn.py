@@ -20,7 +20,7 @@ What it computes, for one layer and tokens x[b, :]:
              ReGLU: a_i = max(0, w_gate_i . x + b_i) * (w_up_i . x)
              a[b, i] = 0 where token b's own mask bit is 0
   down       y_j = sum over idx ascending of W_down[j, i] * a_i
-  glue       x' = (x + y) / sqrt(mean((x + y)^2) + 1e-6), rounded to the activation dtype
+  glue       v = x + y ; x' = (v - mean(v)) / sqrt(var(v) + 1e-6), rounded to the activation dtype
 All arithmetic is fp64; stored values (fp16, Q4_0) are widened exactly.
 """
 from __future__ import annotations
@@ -201,12 +201,15 @@ def _round_act(v: np.ndarray, x_dtype: str) -> np.ndarray:
 
 
 def stack_glue(x: np.ndarray, y: np.ndarray, x_dtype: str) -> np.ndarray:
-    """x' = (x + y) / sqrt(mean((x + y)^2) + 1e-6), per token, rounded to the
-    activation dtype (through fp32, the glue's precision).  The pages have no layer
-    stack; this residual + RMS normalisation keeps every layer input ~ N(0, I)."""
+    """x' = (v - mean(v)) / sqrt(var(v) + 1e-6) with v = x + y, per token, rounded to the
+    activation dtype (through fp32, the glue's precision).  The pages have no layer stack;
+    this residual + mean-centred normalisation keeps every layer input centred with unit
+    variance, so the firing law of the next layer holds even when the weights have a
+    nonzero mean (Q4_0 codes q - 8 have mean -1/2)."""
     v = np.atleast_2d(np.asarray(x, np.float64)) + y
-    rms = np.sqrt(np.mean(v * v, axis=1, keepdims=True) + RMS_EPS)
-    return _round_act(v / rms, x_dtype)
+    mu = np.mean(v, axis=1, keepdims=True)
+    var = np.mean((v - mu) * (v - mu), axis=1, keepdims=True)
+    return _round_act((v - mu) / np.sqrt(var + RMS_EPS), x_dtype)
 
 
 def layer_step(x: np.ndarray, w: Dict[str, np.ndarray], act: str, x_dtype: str):

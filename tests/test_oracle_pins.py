@@ -230,16 +230,22 @@ def test_q4_0_scale_is_fp16():
 
 # ----------------------------------------------------------------- glue, hot order
 def test_stack_glue_closed_form():
-    x = np.array([[3.0, -4.0, 0.0, 0.0]], np.float32)
+    x = np.array([[3.0, -4.0, 0.0, 1.0]], np.float32)
     y = np.zeros((1, 4))
     out = O.stack_glue(x, y, "f32")
-    rms = np.sqrt((9 + 16) / 4 + 1e-6)
-    assert np.array_equal(out, np.array([[3 / rms, -4 / rms, 0, 0]], np.float32))
-    # residual: x + y enters, not y alone; scale-invariant up to eps
-    y2 = np.array([[1.0, 0.0, 0.0, 2.0]])
-    v = np.array([4.0, -4.0, 0.0, 2.0])
-    assert np.allclose(O.stack_glue(x, y2, "f32")[0], v / np.sqrt(np.mean(v * v) + 1e-6), rtol=1e-6)
+    # mean 0, var = (9 + 16 + 0 + 1) / 4 = 6.5
+    sd = np.sqrt(6.5 + 1e-6)
+    assert np.array_equal(out, np.array([[3 / sd, -4 / sd, 0, 1 / sd]], np.float32))
+    # residual: x + y enters, and a constant offset is removed
+    y2 = np.array([[1.0, 0.0, 0.0, 2.0]]) + 10.0
+    v = np.array([4.0, -4.0, 0.0, 3.0]) + 10.0
+    w = v - v.mean()
+    assert np.allclose(O.stack_glue(x, y2, "f32")[0], w / np.sqrt(np.mean(w * w) + 1e-6), rtol=1e-6)
     assert O.stack_glue(x, y2, "f16").dtype == np.float16
+    # the output is centred with unit variance (up to eps and rounding)
+    rng = np.random.default_rng(2)
+    o = O.stack_glue(rng.normal(size=(3, 256)), rng.normal(size=(3, 256)) + 5.0, "f32").astype(np.float64)
+    assert np.allclose(o.mean(axis=1), 0, atol=1e-6) and np.allclose(o.var(axis=1), 1, atol=1e-5)
 
 
 def test_hot_order_and_prefix():
