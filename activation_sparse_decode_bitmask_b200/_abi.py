@@ -169,10 +169,10 @@ class Workspace:
         _check(_lib.pi_diag_phase_clocks_enable(self.handle, int(on)), "pi_diag_phase_clocks_enable")
 
     def read_phase_clocks(self, L_max: int):
-        """[grid, L_max, 16] int64 SM cycle stamps of the last stack call."""
+        """[grid, L_max, 20] int64 SM cycle stamps of the last stack call."""
         import numpy as np
         g = self.grid()
-        out = np.zeros((g, L_max, 16), dtype=np.int64)
+        out = np.zeros((g, L_max, 20), dtype=np.int64)
         _check(_lib.pi_diag_phase_clocks_read(self.handle, out.ctypes.data, out.size), "pi_diag_phase_clocks_read")
         return out
 

@@ -117,16 +117,8 @@ pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedPara
   p.barrier_timeout_ns = kDefaultWaitNs;
   p.wait_cycles = kDefaultWaitNs * 3;   // cycles at up to 3 GHz: at least the nominal budget
   p.barrier_extra = 0;
-  static const unsigned poll_ns = [] {
-    const char* e = std::getenv("PI_POLL_NS");   // tuning knob for the exchange back-off
-    return e ? (unsigned)std::strtoul(e, nullptr, 10) : 64u;
-  }();
-  p.poll_ns = poll_ns;
-  static const int gate = [] {
-    const char* e = std::getenv("PI_GATE_PRODUCER");
-    return e ? std::atoi(e) : 0;
-  }();
-  p.gate_producer = gate;
+  p.poll_ns = 64;          // back-off between exchange polling rounds
+  p.gate_producer = 0;
   return PI_OK;
 }
 
@@ -507,7 +499,7 @@ pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on) {
   }
   ws->phase_global = on == 2;
   if (ws->phase_clk) return PI_OK;
-  const size_t n = (size_t)ws->grid * ws->L_max * 16;
+  const size_t n = (size_t)ws->grid * ws->L_max * 20;
   if (dmalloc(&ws->phase_clk, n * sizeof(long long)) != cudaSuccess) return PI_ERR_OOM;
   PI_TRY(cudaMemset(ws->phase_clk, 0, n * sizeof(long long)));
   return PI_OK;
@@ -515,7 +507,7 @@ pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on) {
 
 pi_status pi_diag_phase_clocks_read(pi_workspace* ws, long long* host_out, size_t n) {
   if (!ws || !host_out || !ws->phase_clk) return PI_ERR_ARG;
-  const size_t total = (size_t)ws->grid * ws->L_max * 16;
+  const size_t total = (size_t)ws->grid * ws->L_max * 20;
   if (n > total) return PI_ERR_ARG;
   PI_TRY(cudaMemcpy(host_out, ws->phase_clk, n * sizeof(long long), cudaMemcpyDeviceToHost));
   return PI_OK;

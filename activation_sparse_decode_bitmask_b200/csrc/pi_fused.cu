@@ -43,7 +43,7 @@ constexpr float kRmsEps = 1e-6f;
 constexpr int kRedBar = 1;          // named barrier id among consumers
 constexpr int kMaxColGroups = 4;    // 32-column groups per reduce slice
 constexpr int kItems = 32;          // ring items in flight (mbarrier pairs)
-constexpr int kMaxBatch = 8;        // records per F batch
+constexpr int kMaxBatch = 16;       // records per F batch (one warp each)
 
 struct Smem {
   uint64_t full[kItems];
@@ -68,7 +68,7 @@ struct Smem {
 };
 
 // Diagnostics: SM cycle stamps at phase boundaries, [block][layer][kPhases].
-constexpr int kPhases = 16;
+constexpr int kPhases = 20;
 __device__ __forceinline__ long long stamp_now(const FusedParams& p) {
   return p.phase_global ? (long long)globaltimer_ns() : clock64();
 }
@@ -532,6 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           if (base + t + k * kConsumerThreads < B * G * W) bm[base + t + k * kConsumerThreads] = (uint32_t)w[k];
       }
       named_bar_sync(kRedBar, kConsumerThreads);
+      stamp(p, l, 14);
       // active count per owner block (union over tokens), prefix over blocks
       if (t < G) {
         int n = 0;
@@ -558,6 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         if (lane == 0) { sm.cstart[0] = 0; sm.count = carry; }
       }
       named_bar_sync(kRedBar, kConsumerThreads);
+      stamp(p, l, 15);
       const int count = sm.count;
       // this block's even share of the active neurons, in (owner block, owner position) order
       const int a0 = (int)((long long)c * count / G), a1 = (int)((long long)(c + 1) * count / G);
@@ -693,12 +695,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         const uint8_t* rec = ring.base + pos;
         ring_wait_item(item0 + warp, sm, p);
         if (e0 == 0 && warp == 0) stamp(p, l, 5);
-        float ua[NB];
-        warp_dot_w<FAM, NB>(rec + p.up_off, xs, d, ua);
-        float ga[NB];
+        float ua[NB], ga[NB];
+        if constexpr (ACT == PI_REGLU) {
+          warp_dot_w2<FAM, NB>(rec + p.up_off, rec + p.gate_off, xs, d, ua, ga);
+        } else {
+          warp_dot_w<FAM, NB>(rec + p.up_off, xs, d, ua);
 #pragma unroll
-        for (int b = 0; b < NB; ++b) ga[b] = 0.f;
-        if constexpr (ACT == PI_REGLU) warp_dot_w<FAM, NB>(rec + p.gate_off, xs, d, ga);
+          for (int b = 0; b < NB; ++b) ga[b] = 0.f;
+        }
         if (lane == 0) {
           const int e = e0 + warp;
           const uint32_t bits = sm.list_bits[e];
@@ -861,7 +865,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           sm.gsd[warp] = sqrtf(var + kRmsEps);
         }
       }
-      named_bar_sync(kRedBar, kConsumerThreads);   // rms known; every warp is done reading xs
+      named_bar_sync(kRedBar, kConsumerThreads);
+      stamp(p, l, 16);   // rms known; every warp is done reading xs
       {
         const int npairs = B * d / 2;
         for (int base = 0; base < npairs; base += 8 * kConsumerThreads) {
@@ -898,6 +903,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           }
         }
       }
+      stamp(p, l, 17);
       // slice owners: the new input of their slice, the trace, and the output
       if (slice_owner && warp < NB && warp < B) {
         const int b = warp;
@@ -967,22 +973,22 @@ __global__ void __launch_bounds__(kThreads, 1) barrier_probe_kernel(const FusedP
 
 // Largest per-thread unit count of each (family, tokens) instantiation.
 template <int FAM, int NB> struct NUof;
-template <> struct NUof<FAM_F32, 1> { static constexpr int v = 4; };
-template <> struct NUof<FAM_F32, 2> { static constexpr int v = 4; };
-template <> struct NUof<FAM_F32, 4> { static constexpr int v = 4; };
-template <> struct NUof<FAM_F16, 1> { static constexpr int v = 6; };
-template <> struct NUof<FAM_F16, 2> { static constexpr int v = 4; };
-template <> struct NUof<FAM_F16, 4> { static constexpr int v = 2; };
-template <> struct NUof<FAM_Q4, 1> { static constexpr int v = 2; };
+template <> struct NUof<FAM_F32, 1> { static constexpr int v = 2; };
+template <> struct NUof<FAM_F32, 2> { static constexpr int v = 2; };
+template <> struct NUof<FAM_F32, 4> { static constexpr int v = 2; };
+template <> struct NUof<FAM_F16, 1> { static constexpr int v = 3; };
+template <> struct NUof<FAM_F16, 2> { static constexpr int v = 2; };
+template <> struct NUof<FAM_F16, 4> { static constexpr int v = 1; };
+template <> struct NUof<FAM_Q4, 1> { static constexpr int v = 1; };
 template <> struct NUof<FAM_Q4, 2> { static constexpr int v = 1; };
 
 constexpr int ue_of(int fam) { return fam == FAM_F32 ? 4 : fam == FAM_F16 ? 8 : 32; }
 
 int nu_max(int fam, int nb) {
   switch (fam) {
-    case FAM_F32: return 4;
-    case FAM_F16: return nb == 1 ? 6 : nb == 2 ? 4 : 2;
-    case FAM_Q4: return nb == 1 ? 2 : nb == 2 ? 1 : 0;
+    case FAM_F32: return 2;
+    case FAM_F16: return nb == 1 ? 3 : nb == 2 ? 2 : 1;
+    case FAM_Q4: return nb <= 2 ? 1 : 0;
   }
   return 0;
 }

@@ -21,8 +21,8 @@ enum DevErr : int {
 // dtype families (w, x, p)
 enum Family : int { FAM_F32 = 0, FAM_F16 = 1, FAM_Q4 = 2 };
 
-// Kernel launch geometry of the fused kernel: 8 consumer warps + 1 producer warp.
-constexpr int kConsumerWarps = 8;
+// Kernel launch geometry of the fused kernel: 16 consumer warps + 1 producer warp.
+constexpr int kConsumerWarps = 16;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;
 constexpr int kMaxOwn = 512;          // owned neurons per block (d_ff <= 512 * grid)

@@ -117,7 +117,54 @@ __device__ __forceinline__ void warp_dot_w(const uint8_t* row, const void* xs, i
   }
 }
 
-// y[b] += h[b] * row for the thread's units (consumer thread t owns units t + 256*j).
+// Warp dots of two weight rows (up and gate of one neuron) with x, reading x once.
+template <int FAM, int NB>
+__device__ __forceinline__ void warp_dot_w2(const uint8_t* row_a, const uint8_t* row_b, const void* xs, int d,
+                                            float (&acc_a)[NB], float (&acc_b)[NB]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) acc_a[b] = acc_b[b] = 0.f;
+  if constexpr (FAM == FAM_F32) {
+    const float4* wa = reinterpret_cast<const float4*>(row_a);
+    const float4* wb = reinterpret_cast<const float4*>(row_b);
+    const float* x = reinterpret_cast<const float*>(xs);
+#pragma unroll 4
+    for (int q = lane; q < d / 4; q += 32) {
+      const float4 a = wa[q], c = wb[q];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const float4 xv = reinterpret_cast<const float4*>(x + (size_t)b * d)[q];
+        acc_a[b] = fmaf(a.x, xv.x, fmaf(a.y, xv.y, fmaf(a.z, xv.z, fmaf(a.w, xv.w, acc_a[b]))));
+        acc_b[b] = fmaf(c.x, xv.x, fmaf(c.y, xv.y, fmaf(c.z, xv.z, fmaf(c.w, xv.w, acc_b[b]))));
+      }
+    }
+  } else if constexpr (FAM == FAM_F16) {
+    const uint4* wa = reinterpret_cast<const uint4*>(row_a);
+    const uint4* wb = reinterpret_cast<const uint4*>(row_b);
+    const __half* x = reinterpret_cast<const __half*>(xs);
+#pragma unroll 4
+    for (int q = lane; q < d / 8; q += 32) {
+      const uint4 a = wa[q], c = wb[q];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const uint4 xv = reinterpret_cast<const uint4*>(x + (size_t)b * d)[q];
+        acc_a[b] += dot8_h(a, xv);
+        acc_b[b] += dot8_h(c, xv);
+      }
+    }
+  } else {
+    warp_dot_w<FAM, NB>(row_a, xs, d, acc_a);
+    warp_dot_w<FAM, NB>(row_b, xs, d, acc_b);
+    return;
+  }
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    acc_a[b] = warp_sum(acc_a[b]);
+    acc_b[b] = warp_sum(acc_b[b]);
+  }
+}
+
+// y[b] += h[b] * row for the thread's units (consumer thread t owns units t + kConsumerThreads*j).
 template <int FAM, int NB, int NU>
 __device__ __forceinline__ void axpy_units(const uint8_t* row, int nunits, int d, const float (&h)[NB],
                                            float (&y)[NB][NU][Fam<FAM>::UE]) {

@@ -196,17 +196,18 @@ pi_status pi_workspace_layer_counts(pi_workspace* ws, int32_t* host_out, int L);
 pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaStream_t stream);
 
 /* Diagnostic: with `on`, every later pi_decode_stack on this workspace records each
- * block's SM cycle counter at 16 points of every layer. The consumer warps record 0-8:
+ * block's SM cycle counter at 20 points of every layer. The consumer warps record 0-8:
  * layer start, predictor rows done, after the first grid barrier, own active list ready,
  * FFN done, after the second barrier, slice reduce done, after the third barrier, and
  * glue done. The producer warp records 9-11: waiting for the active list, list
  * received, and all of the layer's weight rows issued; 12 and 13 mark the first
- * predictor item landing (P2, P1). With `on` = 2 the stamps come from
+ * predictor item landing (P2, P1); 14-17 split the bitmap and glue exchanges (bitmaps
+ * read, prefix formed, moments read, v read). With `on` = 2 the stamps come from
  * the GPU's global nanosecond timer instead, so blocks can be compared with one another.
  * With `on` = 0 recording stops and the buffer is freed. */
 pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on);
 
-/* Copy the first n stamps ([grid][L_max][16], int64) to host memory (synchronous). */
+/* Copy the first n stamps ([grid][L_max][20], int64) to host memory (synchronous). */
 pi_status pi_diag_phase_clocks_read(pi_workspace* ws, long long* host_out, size_t n);
 
 /* Blocks per launch of the fused kernel on this workspace's device (its SM count). */
