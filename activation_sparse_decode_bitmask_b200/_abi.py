@@ -18,6 +18,7 @@ from . import _build
 PI_F32, PI_F16, PI_Q4_0 = 0, 1, 2
 PI_RELU, PI_REGLU = 0, 1
 PI_MAX_BATCH = 32
+PI_NOALLOC_SCRATCH_BYTES = 256 * 1024
 
 STATUS = {0: "PI_OK", 1: "PI_ERR_ARG", 2: "PI_ERR_UNSUPPORTED", 3: "PI_ERR_OOM", 4: "PI_ERR_CUDA",
           5: "PI_ERR_TIMEOUT", 6: "PI_ERR_DEVICE"}
@@ -26,7 +27,7 @@ STATUS = {0: "PI_OK", 1: "PI_ERR_ARG", 2: "PI_ERR_UNSUPPORTED", 3: "PI_ERR_OOM",
 EXPORTS = ["pi_load_layer", "pi_reorder_hot_prefix", "pi_get_perm", "pi_layer_get_desc", "pi_free_layer",
            "pi_workspace_create", "pi_workspace_free", "pi_stream_status", "pi_workspace_active_total",
            "pi_workspace_layer_counts", "pi_diag_phase_clocks_enable", "pi_diag_phase_clocks_read",
-           "pi_device_grid", "pi_diag_barrier_timeout", "pi_predict", "pi_compact_active",
+           "pi_device_grid", "pi_diag_barrier_timeout", "pi_predict", "pi_predict_noalloc", "pi_compact_active",
            "pi_sparse_ffn", "pi_decode_stack", "pi_decode_stack_host", "pi_status_str", "pi_abi_version"]
 
 
@@ -71,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "pi_diag_phase_clocks_read": (i, [vp, vp, ctypes.c_size_t]),
         "pi_device_grid": (i, [vp]),
         "pi_predict": (i, [vp, vp, i, vp, vp, vp, vp]),
+        "pi_predict_noalloc": (i, [vp, vp, i, vp, vp, vp, vp]),
         "pi_compact_active": (i, [vp, i, i, vp, vp, vp]),
         "pi_sparse_ffn": (i, [vp, vp, i, vp, vp, vp, vp, vp, vp]),
         "pi_decode_stack": (i, [vp, i, vp, i, POINTER(Trace), vp, vp]),
@@ -212,6 +214,13 @@ def predict(layer: Layer, x: torch.Tensor, B: int, mask: torch.Tensor, logits: O
             ws: Workspace, stream=None) -> None:
     _check(_lib.pi_predict(layer.handle, _ptr(x), B, _ptr(mask), _ptr(logits), ws.handle,
                            c_void_p(_stream(stream))), "pi_predict")
+
+
+def predict_noalloc(layer: Layer, x: torch.Tensor, B: int, mask: torch.Tensor, logits: Optional[torch.Tensor],
+                    status: torch.Tensor, stream=None) -> None:
+    """pi_predict without a workspace; `status` is a device int32 tensor of one element."""
+    _check(_lib.pi_predict_noalloc(layer.handle, _ptr(x), B, _ptr(mask), _ptr(logits), _ptr(status),
+                                   c_void_p(_stream(stream))), "pi_predict_noalloc")
 
 
 def compact_active(mask: torch.Tensor, B: int, d_ff: int, idx: torch.Tensor, count: torch.Tensor,

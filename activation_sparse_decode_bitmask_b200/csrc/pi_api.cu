@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "pi_internal.h"
@@ -526,6 +527,112 @@ pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaSt
   p.wait_cycles = timeout_ns * 2;   // SM cycles, about 2 per ns
   p.barrier_extra = 1;   // one arrival more than the grid has: no wait can complete
   PI_TRY(launch_barrier_probe(p, 2, stream));
+  return PI_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ predictor without a workspace
+// pi_predict_noalloc runs the predictor launch of pi_predict with its cross-block
+// scratch in one static device array instead of a workspace. It exists for callers that
+// cannot allocate device memory when they call it: a serving loop that has already
+// handed all free HBM to its weights and KV cache, and a plug-in that sees only a stream
+// and plain pointers and so has nowhere to keep a workspace between calls.
+// Layout of the array: [0, 64) launch words (probe count, exit count, epoch),
+// [64, 128) error word, [128, 256) active-list total, then the tagged u words
+// (B * rank * 8 bytes) and the tagged bitmap words (B * G * W * 8 bytes), each section
+// starting on a 256-byte boundary.
+namespace {
+
+constexpr size_t kNoallocCtlBytes = 256;
+constexpr int kNoallocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PI_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+unsigned char* g_noalloc_base[kNoallocMaxDevices];   // per device, set once
+
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Launch words start as {0, 0, 1}: counts at zero, epoch 1, so that no zeroed tagged
+// word matches a live tag.
+__global__ void noalloc_init_kernel(uint32_t* ctl) { ctl[2] = 1u; }
+
+// After the predictor launch: report its error word and, if it aborted, leave the
+// scratch as a fresh workspace would be (counts at zero, a new epoch, error cleared).
+__global__ void noalloc_status_kernel(uint32_t* ctl, int* err, int32_t* status) {
+  const int e = *err;
+  *status = e == 0 ? PI_OK
+                   : (e == DEV_ERR_GRID_TIMEOUT || e == DEV_ERR_RING_TIMEOUT) ? PI_ERR_TIMEOUT : PI_ERR_DEVICE;
+  if (e != 0) {
+    ctl[0] = 0u;
+    ctl[1] = 0u;
+    ctl[2] += 1u;
+    *err = 0;
+  }
+}
+
+// The scratch of the current device: on its first use the symbol's address is taken,
+// the array cleared and the epoch set, and `stream` synchronised so that any stream
+// may make the next call.
+pi_status noalloc_scratch(int dev, cudaStream_t stream, unsigned char** out) {
+  if (dev < 0 || dev >= kNoallocMaxDevices) return PI_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_base[dev]) {
+    void* ptr = nullptr;
+    PI_TRY(cudaGetSymbolAddress(&ptr, g_noalloc_scratch));
+    PI_TRY(cudaMemsetAsync(ptr, 0, PI_NOALLOC_SCRATCH_BYTES, stream));
+    noalloc_init_kernel<<<1, 1, 0, stream>>>(static_cast<uint32_t*>(ptr));
+    PI_TRY(cudaGetLastError());
+    PI_TRY(cudaStreamSynchronize(stream));
+    g_noalloc_base[dev] = static_cast<unsigned char*>(ptr);
+  }
+  *out = g_noalloc_base[dev];
+  return PI_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pi_status pi_predict_noalloc(const pi_layer* L, const void* x, int B, uint32_t* mask, float* logits,
+                             int32_t* status, cudaStream_t stream) {
+  if (!L || !x || !mask || !status || B < 1 || B > PI_MAX_BATCH) return PI_ERR_ARG;
+  int dev = -1;
+  PI_TRY(cudaGetDevice(&dev));
+  const int G = sm_count(dev);
+  if (G <= 0) return PI_ERR_CUDA;
+  if (L->G != G) return PI_ERR_ARG;   // layer laid out for another device
+  const size_t W = (size_t)(L->nown_max + 31) / 32;
+  const size_t u_bytes = round256((size_t)B * L->desc.rank * 8);
+  const size_t b_bytes = round256((size_t)B * G * W * 8);
+  if (kNoallocCtlBytes + u_bytes + b_bytes > PI_NOALLOC_SCRATCH_BYTES) return PI_ERR_UNSUPPORTED;
+  unsigned char* s = nullptr;
+  pi_status st = noalloc_scratch(dev, stream, &s);
+  if (st != PI_OK) return st;
+  pi_workspace w;   // a view of the static scratch; nothing is allocated
+  std::memset(&w, 0, sizeof(w));
+  w.d_max = L->desc.d_model; w.f_max = L->desc.d_ff; w.r_max = L->desc.rank; w.B_max = B; w.L_max = 1;
+  w.grid = G;
+  w.device = dev;
+  w.bar = reinterpret_cast<uint32_t*>(s);
+  w.err = reinterpret_cast<int*>(s + 64);
+  w.active_total = reinterpret_cast<unsigned long long*>(s + 128);
+  w.ux = reinterpret_cast<uint64_t*>(s + kNoallocCtlBytes);
+  w.bx = reinterpret_cast<uint64_t*>(s + kNoallocCtlBytes + u_bytes);
+  FusedParams p;
+  size_t smem = 0;
+  st = plan_fused(L, B, &w, p, smem);
+  if (st != PI_OK) return st;
+  p.mode = MODE_PREDICT;
+  p.L = 1;
+  p.layers[0] = dev_view(L);
+  p.x_in = x;
+  p.mask_out = mask;
+  p.logits_out = logits;
+  PI_TRY(launch_fused(L->family, L->desc.act, B, p, smem, stream));
+  noalloc_status_kernel<<<1, 1, 0, stream>>>(w.bar, w.err, status);
+  PI_TRY(cudaGetLastError());
   return PI_OK;
 }
 

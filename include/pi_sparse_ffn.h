@@ -221,6 +221,33 @@ int pi_device_grid(pi_workspace* ws);
 pi_status pi_predict(const pi_layer* layer, const void* x, int B, uint32_t* mask,
                      float* logits, pi_workspace* ws, cudaStream_t stream);
 
+/* Bytes of the static device scratch behind pi_predict_noalloc (256 KiB). */
+#define PI_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+
+/* pi_predict without a workspace: the same predictor launch, with the same outputs and
+ * the same bits as pi_predict. It allocates no memory: its cross-block scratch is
+ * one static device array of PI_NOALLOC_SCRATCH_BYTES per device. The pages have no
+ * counterpart; this entry point is this library's own. It is for callers that cannot
+ * allocate device memory when they call it, such as a serving loop that has already
+ * handed all free HBM to its weights and KV cache, or a plug-in that sees only a
+ * stream and plain pointers and has nowhere to keep a workspace between calls.
+ *
+ * status: device i32, owned by the caller (required). After the launch it receives
+ *   PI_OK, PI_ERR_TIMEOUT (a bounded device-side wait gave up) or PI_ERR_DEVICE (a
+ *   device-side check failed). After an error the scratch is reset on the device for
+ *   the next call.
+ * Scratch needed: 256 + round256(B * rank * 8) + round256(B * G * W * 8) bytes, where
+ *   G is the SM count and W = ceil(ceil(d_ff / G) / 32). A shape that needs more than
+ *   PI_NOALLOC_SCRATCH_BYTES returns PI_ERR_UNSUPPORTED and enqueues nothing.
+ * Set-up: the first call on each device takes the array's address, clears it and
+ *   synchronises `stream` before it returns. Make that first call before any stream
+ *   capture begins.
+ * Calls share the one array per device. Two calls that may run at the same time (on
+ *   different streams, or from different threads without ordering) race on it and
+ *   give undefined results. Order them on one stream or with events. */
+pi_status pi_predict_noalloc(const pi_layer* layer, const void* x, int B, uint32_t* mask,
+                             float* logits, int32_t* status, cudaStream_t stream);
+
 /* Compaction. idx (device i32 [d_ff]) receives the ascending ids of the neurons whose
  * bit is set for any of the B tokens (the OR of mask[0..B-1]). *count (device i32)
  * receives their number. Only the first *count entries of idx are written. */
