@@ -74,8 +74,10 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def profiled_traffic(workload, batch):
-    """DRAM bytes per launch from a committed ncu capture of this exact kernel source."""
+def profiled_traffic(workload, n_layers, batch):
+    """DRAM bytes per launch (read + write) from a committed ncu capture of this exact
+    kernel source.  Captures run a shorter stack of the same layers; the record holds
+    bytes per layer, scaled here by the stack depth of the timed launch."""
     if not os.path.exists(PROFILE_TRAFFIC):
         return None
     with open(PROFILE_TRAFFIC) as fh:
@@ -83,7 +85,7 @@ def profiled_traffic(workload, batch):
     rec = d.get(f"{workload}/B{batch}")
     if not rec or rec.get("source_hash") != source_hash():
         return None
-    return rec.get("dram_bytes_per_launch")
+    return int(rec["dram_bytes_per_layer"] * n_layers)
 
 
 class ClockSampler:
@@ -263,7 +265,7 @@ def run_ours(args, world, rank, local):
     algo_bytes = wl.n_layers * predictor_bytes(wl) + active_per_step * bytes_per_neuron(wl)
     achieved = algo_bytes / (ms_local / K / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
-    traffic = profiled_traffic(wl.name, B)
+    traffic = profiled_traffic(wl.name, wl.n_layers, B)
 
     # end to end through the host-buffer entry point: H2D x, the stack, D2H x, sync
     Ke = min(K, args.e2e_steps)
