@@ -19,6 +19,7 @@ PI_F32, PI_F16, PI_Q4_0 = 0, 1, 2
 PI_RELU, PI_REGLU = 0, 1
 PI_MAX_BATCH = 32
 PI_NOALLOC_SCRATCH_BYTES = 256 * 1024
+DIAG_SLOTS = 64   # diagnostic stamps per block and layer
 
 STATUS = {0: "PI_OK", 1: "PI_ERR_ARG", 2: "PI_ERR_UNSUPPORTED", 3: "PI_ERR_OOM", 4: "PI_ERR_CUDA",
           5: "PI_ERR_TIMEOUT", 6: "PI_ERR_DEVICE"}
@@ -174,7 +175,7 @@ class Workspace:
         """[grid, L_max, 20] int64 SM cycle stamps of the last stack call."""
         import numpy as np
         g = self.grid()
-        out = np.zeros((g, L_max, 20), dtype=np.int64)
+        out = np.zeros((g, L_max, DIAG_SLOTS), dtype=np.int64)
         _check(_lib.pi_diag_phase_clocks_read(self.handle, out.ctypes.data, out.size), "pi_diag_phase_clocks_read")
         return out
 

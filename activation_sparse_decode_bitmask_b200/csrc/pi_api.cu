@@ -95,24 +95,27 @@ pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedPara
   if (L->G != ws->grid) return PI_ERR_ARG;   // layer laid out for another device
   if (L->nown_max > kMaxOwn) return PI_ERR_UNSUPPORTED;
   if (!fused_supported(L->family, B, d.d_model)) return PI_ERR_UNSUPPORTED;
-  // ring items: whole neuron records, and predictor rows grouped into ~32 KB copies
-  const int cap = std::max(L->rec_stride, 32 * 1024);
-  p.p1_rows_per_item = std::max(1, cap / L->p1_row);
-  p.p2_rows_per_item = std::max(1, cap / L->p2_stride);
-  const long long max_item = std::max({(long long)L->rec_stride, (long long)p.p1_rows_per_item * L->p1_row,
-                                       (long long)p.p2_rows_per_item * L->p2_stride});
   const size_t budget = (size_t)smem_optin(ws->device);
   const size_t fixed = fused_fixed_smem(B, d.d_model, d.rank, ws->grid, L->nown_max, L->family);
   if (budget <= fixed) return PI_ERR_UNSUPPORTED;
   p.ring_bytes = (int)((budget - fixed) / 128 * 128);
+  // ring items: whole neuron records; P1^T rows grouped into ~32 KB copies; the block's
+  // own P2 rows in as few copies as fit twice in the ring (up to 96 KB each), so that
+  // every consumer warp has rows to work on in the logits pass
+  const int cap = std::max(L->rec_stride, 32 * 1024);
+  const int cap_p2 = std::max(cap, std::min(96 * 1024, p.ring_bytes / 2 - 128));
+  p.p1_rows_per_item = std::max(1, cap / L->p1_row);
+  p.p2_rows_per_item = std::max(1, std::min(L->nown_max, cap_p2 / L->p2_stride));
+  const long long max_item = std::max({(long long)L->rec_stride, (long long)p.p1_rows_per_item * L->p1_row,
+                                       (long long)p.p2_rows_per_item * L->p2_stride});
   if (p.ring_bytes < 2 * max_item || max_item >= (1 << 20)) return PI_ERR_UNSUPPORTED;
-  // records per F batch: the whole batch must sit in the ring at once (one record of
-  // slack for the placement that never wraps an item)
-  p.batch = std::min(fused_max_batch(), p.ring_bytes / L->rec_stride - 1);
-  if (p.batch < 1) return PI_ERR_UNSUPPORTED;
+  // records outstanding at once: floor(ring / stride) - 1 (an item never wraps); a
+  // window plus the record after it must fit
+  p.rec_window = p.ring_bytes / L->rec_stride - 2;
+  if (p.rec_window < 1) return PI_ERR_UNSUPPORTED;
   smem = fixed + (size_t)p.ring_bytes;
   // ws fields
-  p.ux = ws->ux; p.px = ws->px; p.vx = ws->vx; p.sx = ws->sx; p.bx = ws->bx;
+  p.ux = ws->ux; p.px = ws->px; p.vx = ws->vx; p.sx = ws->sx;
   p.bar = ws->bar; p.err = ws->err; p.active_total = ws->active_total;
   p.layer_count = nullptr;
   p.barrier_timeout_ns = kDefaultWaitNs;
@@ -335,12 +338,10 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
   if (ws->grid <= 0) { delete ws; return PI_ERR_CUDA; }
   if (ws->grid > kMaxGrid) { delete ws; return PI_ERR_UNSUPPORTED; }
   const size_t G = ws->grid, Bm = B_max;
-  const size_t Wm = ((f_max + G - 1) / G + 31) / 32;   // bitmap words per block and token
   bool ok = dmalloc(&ws->ux, Bm * r_max * 8) == cudaSuccess &&
             dmalloc(&ws->px, G * Bm * d_max * 8) == cudaSuccess &&
             dmalloc(&ws->vx, Bm * d_max * 8) == cudaSuccess &&
             dmalloc(&ws->sx, Bm * G * 16) == cudaSuccess &&
-            dmalloc(&ws->bx, Bm * G * Wm * 8) == cudaSuccess &&
             dmalloc(&ws->bar, 64) == cudaSuccess &&
             dmalloc(&ws->err, 16) == cudaSuccess &&
             dmalloc(&ws->active_total, 16) == cudaSuccess &&
@@ -351,7 +352,6 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
     const uint32_t bar0[4] = {0u, 0u, 1u, 0u};
     ok = cudaMemset(ws->ux, 0, Bm * r_max * 8) == cudaSuccess && cudaMemset(ws->px, 0, G * Bm * d_max * 8) == cudaSuccess &&
          cudaMemset(ws->vx, 0, Bm * d_max * 8) == cudaSuccess && cudaMemset(ws->sx, 0, Bm * G * 16) == cudaSuccess &&
-         cudaMemset(ws->bx, 0, Bm * G * Wm * 8) == cudaSuccess &&
          cudaMemset(ws->bar, 0, 64) == cudaSuccess &&
          cudaMemcpy(ws->bar, bar0, sizeof(bar0), cudaMemcpyHostToDevice) == cudaSuccess &&
          cudaMemset(ws->err, 0, 16) == cudaSuccess && cudaMemset(ws->active_total, 0, 16) == cudaSuccess &&
@@ -368,7 +368,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
 
 void pi_workspace_free(pi_workspace* ws) {
   if (!ws) return;
-  cudaFree(ws->ux); cudaFree(ws->px); cudaFree(ws->vx); cudaFree(ws->sx); cudaFree(ws->bx);
+  cudaFree(ws->ux); cudaFree(ws->px); cudaFree(ws->vx); cudaFree(ws->sx);
   cudaFree(ws->bar); cudaFree(ws->err); cudaFree(ws->active_total);
   cudaFree(ws->layer_count); cudaFree(ws->x_dev); cudaFree(ws->phase_clk);
   delete ws;
@@ -419,6 +419,7 @@ pi_status pi_predict(const pi_layer* L, const void* x, int B, uint32_t* mask, fl
   p.x_in = x;
   p.mask_out = mask;
   p.logits_out = logits;
+  PI_TRY(cudaMemsetAsync(mask, 0, (size_t)B * (L->desc.d_ff / 32) * 4, stream));   // bits are OR-ed in
   PI_TRY(launch_fused(L->family, L->desc.act, B, p, smem, stream));
   return PI_OK;
 }
@@ -470,12 +471,24 @@ pi_status pi_decode_stack(pi_layer* const* layers, int Lc, void* x_inout, int B,
   for (int l = 0; l < Lc; ++l) p.layers[l] = dev_view(layers[l], B);
   p.x_in = x_inout;
   p.x_out = x_inout;
-  if (trace) p.trace = *trace;
+  const int words = L0->desc.d_ff / 32;
+  if (trace) {
+    // idx and count are the compaction of the layer's mask, so they come with it
+    if ((trace->idx || trace->count) && !(trace->idx && trace->count && trace->mask)) return PI_ERR_ARG;
+    p.trace = *trace;
+    p.trace.idx = nullptr;
+    p.trace.count = nullptr;
+  }
   p.layer_count = ws->layer_count;
   p.phase_clk = ws->phase_clk;
   p.phase_global = ws->phase_global;
   PI_TRY(cudaMemsetAsync(ws->layer_count, 0, (size_t)Lc * 4, stream));
+  if (trace && trace->mask) PI_TRY(cudaMemsetAsync(trace->mask, 0, (size_t)Lc * B * words * 4, stream));
   PI_TRY(launch_fused(L0->family, L0->desc.act, B, p, smem, stream));
+  if (trace && trace->idx)
+    for (int l = 0; l < Lc; ++l)
+      PI_TRY(launch_compact(trace->mask + (size_t)l * B * words, B, L0->desc.d_ff, trace->idx + (size_t)l * L0->desc.d_ff,
+                            trace->count + l, stream));
   return PI_OK;
 }
 
@@ -500,7 +513,7 @@ pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on) {
   }
   ws->phase_global = on == 2;
   if (ws->phase_clk) return PI_OK;
-  const size_t n = (size_t)ws->grid * ws->L_max * 20;
+  const size_t n = (size_t)ws->grid * ws->L_max * kDiagSlots;
   if (dmalloc(&ws->phase_clk, n * sizeof(long long)) != cudaSuccess) return PI_ERR_OOM;
   PI_TRY(cudaMemset(ws->phase_clk, 0, n * sizeof(long long)));
   return PI_OK;
@@ -508,7 +521,7 @@ pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on) {
 
 pi_status pi_diag_phase_clocks_read(pi_workspace* ws, long long* host_out, size_t n) {
   if (!ws || !host_out || !ws->phase_clk) return PI_ERR_ARG;
-  const size_t total = (size_t)ws->grid * ws->L_max * 20;
+  const size_t total = (size_t)ws->grid * ws->L_max * kDiagSlots;
   if (n > total) return PI_ERR_ARG;
   PI_TRY(cudaMemcpy(host_out, ws->phase_clk, n * sizeof(long long), cudaMemcpyDeviceToHost));
   return PI_OK;
@@ -540,8 +553,7 @@ pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaSt
 // and plain pointers and so has nowhere to keep a workspace between calls.
 // Layout of the array: [0, 64) launch words (probe count, exit count, epoch),
 // [64, 128) error word, [128, 256) active-list total, then the tagged u words
-// (B * rank * 8 bytes) and the tagged bitmap words (B * G * W * 8 bytes), each section
-// starting on a 256-byte boundary.
+// (B * rank * 8 bytes).
 namespace {
 
 constexpr size_t kNoallocCtlBytes = 256;
@@ -603,10 +615,8 @@ pi_status pi_predict_noalloc(const pi_layer* L, const void* x, int B, uint32_t* 
   const int G = sm_count(dev);
   if (G <= 0) return PI_ERR_CUDA;
   if (L->G != G) return PI_ERR_ARG;   // layer laid out for another device
-  const size_t W = (size_t)(L->nown_max + 31) / 32;
   const size_t u_bytes = round256((size_t)B * L->desc.rank * 8);
-  const size_t b_bytes = round256((size_t)B * G * W * 8);
-  if (kNoallocCtlBytes + u_bytes + b_bytes > PI_NOALLOC_SCRATCH_BYTES) return PI_ERR_UNSUPPORTED;
+  if (kNoallocCtlBytes + u_bytes > PI_NOALLOC_SCRATCH_BYTES) return PI_ERR_UNSUPPORTED;
   unsigned char* s = nullptr;
   pi_status st = noalloc_scratch(dev, stream, &s);
   if (st != PI_OK) return st;
@@ -619,7 +629,6 @@ pi_status pi_predict_noalloc(const pi_layer* L, const void* x, int B, uint32_t* 
   w.err = reinterpret_cast<int*>(s + 64);
   w.active_total = reinterpret_cast<unsigned long long*>(s + 128);
   w.ux = reinterpret_cast<uint64_t*>(s + kNoallocCtlBytes);
-  w.bx = reinterpret_cast<uint64_t*>(s + kNoallocCtlBytes + u_bytes);
   FusedParams p;
   size_t smem = 0;
   st = plan_fused(L, B, &w, p, smem);
@@ -630,6 +639,7 @@ pi_status pi_predict_noalloc(const pi_layer* L, const void* x, int B, uint32_t* 
   p.x_in = x;
   p.mask_out = mask;
   p.logits_out = logits;
+  PI_TRY(cudaMemsetAsync(mask, 0, (size_t)B * (L->desc.d_ff / 32) * 4, stream));   // bits are OR-ed in
   PI_TRY(launch_fused(L->family, L->desc.act, B, p, smem, stream));
   noalloc_status_kernel<<<1, 1, 0, stream>>>(w.bar, w.err, status);
   PI_TRY(cudaGetLastError());

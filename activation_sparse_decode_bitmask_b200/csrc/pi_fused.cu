@@ -10,10 +10,9 @@
 // Per layer, for block c of G (stack mode):
 //   P-a  u_k = P1^T[k] . x for the block's rank rows k (one warp per row) -> u exchange
 //   P-b  logit_i = P2^T[i] . u - t_i for the block's own neurons i = c, c+G, c+2G, ...
-//        (one warp per row, four rows at a time); bit = logit > 0 -> bitmap exchange
-//   list every block reads every block's bitmap, so all know the active set; the
-//        active neurons are split evenly: block c takes a contiguous share of them in
-//        (owner block, owner position) order
+//        (8 rows per warp pass); bit = logit > 0
+//   list the block's own active neurons, ascending: nothing is exchanged, so the
+//        producer starts on the records as soon as the block's own bits are known
 //   F    for each of its records: one warp forms the gate/up dot products with x
 //          ReLU : h = max(0, w_up_i . x + b_i)    ReGLU: max(0, w_gate_i . x + b_i) * (w_up_i . x)
 //          h[b] = 0 where token b's bit is 0
@@ -23,6 +22,7 @@
 //        and the slice's sum and sum of squares -> v / moments exchange
 //   glue x' = (v - mean(v)) / sqrt(var(v) + 1e-6) from the slices' sums and sums of
 //        squares, rounded to the activation dtype
+// Mask words (predict output, trace) are OR-ed in by the owner blocks of their bits.
 // Cross-block exchanges use 64-bit words {tag, value}: a reader polls the words
 // themselves until every tag matches, so data and completion arrive together and no grid
 // barrier is needed.  Tags are unique per launch (a device epoch advanced by the last
@@ -43,7 +43,6 @@ constexpr float kRmsEps = 1e-6f;
 constexpr int kRedBar = 1;          // named barrier id among consumers
 constexpr int kMaxColGroups = 4;    // 32-column groups per reduce slice
 constexpr int kItems = 32;          // ring items in flight (mbarrier pairs)
-constexpr int kMaxBatch = 16;       // records per F batch (one warp each)
 
 struct Smem {
   uint64_t full[kItems];
@@ -58,17 +57,16 @@ struct Smem {
   uint32_t item_size[kItems];
   float gmean[4];   // glue: mean and standard deviation of v per token
   float gsd[4];
-  float hbuf[kMaxList][4];      // h of the layer's records, by list position
-  int hflag[kMaxList];          // = layer + 1 once hbuf[e] is written
+  float red[2][kConsumerWarps][16];   // block reductions: warp partials (double-buffered)
+  float hbuf[2][16][4];         // h of the records of an F window (double-buffered)
+  int win[2];                   // records in an F window; 0: not chosen yet
   int32_t list[kMaxList];
   uint8_t list_bits[kMaxList];
   uint8_t own_bits[kMaxOwn];
-  int32_t cstart[kMaxGrid + 1];   // prefix of active counts over owner blocks
-  int scan[kConsumerWarps + 1];
 };
 
 // Diagnostics: SM cycle stamps at phase boundaries, [block][layer][kPhases].
-constexpr int kPhases = 20;
+constexpr int kPhases = kDiagSlots;
 __device__ __forceinline__ long long stamp_now(const FusedParams& p) {
   return p.phase_global ? (long long)globaltimer_ns() : clock64();
 }
@@ -76,6 +74,10 @@ __device__ __forceinline__ void stamp(const FusedParams& p, int l, int ph) {
   if (p.phase_clk && threadIdx.x == 0)
     p.phase_clk[((size_t)blockIdx.x * p.L + l) * kPhases + ph] = stamp_now(p);
 }
+__device__ __forceinline__ void stamp_val(const FusedParams& p, int l, int ph, long long v) {
+  if (p.phase_clk && threadIdx.x == 0) p.phase_clk[((size_t)blockIdx.x * p.L + l) * kPhases + ph] = v;
+}
+__device__ __forceinline__ long long diag_clock(const FusedParams& p) { return p.phase_clk ? clock64() : 0; }
 __device__ __forceinline__ void pstamp(const FusedParams& p, int l, int ph) {
   if (p.phase_clk) p.phase_clk[((size_t)blockIdx.x * p.L + l) * kPhases + ph] = stamp_now(p);
 }
@@ -97,9 +99,6 @@ __device__ __forceinline__ uint64_t tagged(uint32_t bits, uint32_t tag) { return
 __device__ __forceinline__ void st_tag(uint64_t* p, float v, uint32_t tag) {
   asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(tagged(__float_as_uint(v), tag)) : "memory");
 }
-__device__ __forceinline__ void st_tag_u(uint64_t* p, uint32_t v, uint32_t tag) {
-  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(tagged(v, tag)) : "memory");
-}
 __device__ __forceinline__ void st_tag2(uint64_t* p, float v0, float v1, uint32_t tag) {
   asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(p), "l"(tagged(__float_as_uint(v0), tag)),
                "l"(tagged(__float_as_uint(v1), tag))
@@ -115,6 +114,34 @@ __device__ __forceinline__ void ld_tag2(const uint64_t* p, uint64_t& a, uint64_t
 }
 __device__ __forceinline__ bool tag_ok(uint64_t w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
 __device__ __forceinline__ float tag_val(uint64_t w) { return __uint_as_float((uint32_t)w); }
+
+// Butterfly reduce-scatter of 8 per-lane partial sums (per token) across the warp: on
+// return, out[b] in every lane is the full sum of row (lane >> 2) & 7.  The order of
+// the additions is fixed, so the sums are reproducible.
+template <int NB>
+__device__ __forceinline__ void reduce_scatter8(const float (&a)[8][NB], int lane, float (&out)[NB]) {
+  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    float s4[4], s2[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float send = h16 ? a[i][b] : a[i + 4][b];
+      const float keep = h16 ? a[i + 4][b] : a[i][b];
+      s4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float send = h8 ? s4[i] : s4[i + 2];
+      const float keep = h8 ? s4[i + 2] : s4[i];
+      s2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float s1 = (h4 ? s2[1] : s2[0]) + __shfl_xor_sync(0xffffffffu, h4 ? s2[0] : s2[1], 4);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+    out[b] = s1;
+  }
+}
 
 // Poll the tagged words base[first + k*stride] (k < MAXK, index < n) until every one
 // carries `tag`: each round issues all outstanding loads together, so a round costs one
@@ -178,6 +205,11 @@ __device__ __forceinline__ void ring_wait_item(uint32_t item, Smem& sm, const Fu
     }
   }
 }
+// Has ring item `item` landed?  (Non-blocking; valid for items fewer than kItems ahead
+// of the oldest item not yet released.)
+__device__ __forceinline__ bool ring_item_ready(uint32_t item, Smem& sm) {
+  return mbar_test_wait(&sm.full[item % kItems], (item / kItems) & 1u);
+}
 __device__ __forceinline__ void ring_release_item(uint32_t item, Smem& sm) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.empty[item % kItems]);
@@ -219,7 +251,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
   XT* xs = reinterpret_cast<XT*>(ring_base + p.ring_bytes);            // [NB][d] current input
   float* u_s = reinterpret_cast<float*>(xs + (size_t)NB * p.d);        // [NB][r]
   float* red2 = u_s + (size_t)NB * p.r;                                // [8][NB][4][32]
-  uint32_t* bm = reinterpret_cast<uint32_t*>(red2 + kConsumerWarps * NB * kMaxColGroups * 32);   // [B][G][W]
 
   const int c = blockIdx.x, G = gridDim.x;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -227,11 +258,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
   const int d = p.d, f = p.f, r = p.r, B = p.B;
   const int k0 = (int)((long long)c * r / G), k1 = (int)((long long)(c + 1) * r / G);
   const int nown = (c < f) ? (f - c + G - 1) / G : 0;
-  const int W = (p.nown_max + 31) / 32;   // bitmap words per block and token
   const int nunits = d / UE;
   const int words = f / 32;
   const uint32_t epoch = *reinterpret_cast<volatile const uint32_t*>(p.bar + 2);
-  const bool trace_idx = do_glue && (p.trace.idx || p.trace.count);
 
   if (t == 0) {
     for (int s = 0; s < kItems; ++s) {
@@ -240,7 +269,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     }
     mbar_init(&sm.list_ready, 1);
     mbar_init(&sm.layer_start, 1);
-    for (int e = 0; e < kMaxList; ++e) sm.hflag[e] = 0;
     sm.abort_flag = 0;
     sm.nlist = 0;
     mbar_fence_init();
@@ -329,23 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           // memory); the ring copies below then find them in L2 as space frees up.
           for (int e = 0; e < n && ok; ++e)
             prefetch_l2_bulk(Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride);
-          // Warm L2 with the next layer's predictor rows of this block while this layer's
-          // records stream: that bulk traffic then lands in the F phase instead of slowing
-          // the cross-block exchanges that follow it, and the ring copies of those rows
-          // later come from L2.  The prefetches are issued after the first records.
-          const bool warm = do_pred && l + 1 < p.L;
-          const int first_recs = min(n, 2);
-          for (int e = 0; e < first_recs && ok; ++e) {
-            if (!(ok = begin_item((uint32_t)p.rec_stride, dst, fb))) break;
-            bulk_g2s(dst, Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride, fb);
-          }
-          if (warm && ok) {
-            const LayerDev Ln = p.layers[l + 1];
-            if (k1 > k0) prefetch_l2_bulk(Ln.p1t + (size_t)k0 * p.p1_row, (uint32_t)(k1 - k0) * p.p1_row);
-            if (nown > 0)
-              prefetch_l2_bulk(Ln.p2o + (size_t)c * p.nown_max * p.p2_stride, (uint32_t)nown * p.p2_stride);
-          }
-          for (int e = first_recs; e < n && ok; ++e) {
+          for (int e = 0; e < n && ok; ++e) {
             if (!(ok = begin_item((uint32_t)p.rec_stride, dst, fb))) break;
             bulk_g2s(dst, Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride, fb);
           }
@@ -395,28 +407,68 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
   }
   named_bar_sync(kRedBar, kConsumerThreads);
 
+  int redbuf = 0;   // which half of sm.red the next block reduction uses
   for (int l = 0; l < p.L; ++l) {
-    const uint32_t tag_u = tag_of(epoch, l, 0), tag_p = tag_of(epoch, l, 1), tag_v = tag_of(epoch, l, 2),
-                   tag_b = tag_of(epoch, l, 3);
+    const uint32_t tag_u = tag_of(epoch, l, 0), tag_p = tag_of(epoch, l, 1), tag_v = tag_of(epoch, l, 2);
     int nlist = 0;
     stamp(p, l, 0);
+    // this layer's x units, fp32, in registers for P-a and F
+    float xr[NU][NB][UE];
+#pragma unroll
+    for (int j = 0; j < NU; ++j) {
+      const int q = t + kConsumerThreads * j;
+      if (q < nunits) {
+        load_x_unit<FAM, NB>(xs, d, q, xr[j]);
+      } else {
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int e = 0; e < UE; ++e) xr[j][b][e] = 0.f;
+      }
+    }
     if (t == 0) mbar_arrive(&sm.layer_start);
 
     if (do_pred) {
-      // ---------------------------------------------------------- P-a: u rows, a warp per row
+      // ---------------------------------------------------------- P-a: u rows of this block
+      // Every thread dots its x units with each row; a warp reduce-scatter and a 16-warp
+      // sum in shared memory finish 16 / NB rows per pass.
+      constexpr int RP = 16 / NB;
       for (int k = k0; k < k1; k += p.p1_rows_per_item) {
         const int n = min(p.p1_rows_per_item, k1 - k);
         const uint8_t* item = ring_next(ring, (uint32_t)n * p.p1_row);
         ring_wait_item(ring.item, sm, p);
         if (k == k0) stamp(p, l, 13);
-        for (int kk = warp; kk < n; kk += kConsumerWarps) {
-          float acc[NB];
-          warp_dot_p<FAM, NB>(item + (size_t)kk * p.p1_row, xs, d, acc);
-          if (lane < B) {
-            float v = acc[0];
+        for (int i0 = 0; i0 < n; i0 += RP) {
+          float v[16];
 #pragma unroll
-            for (int b = 1; b < NB; ++b) if (lane == b) v = acc[b];
-            st_tag(p.ux + (size_t)lane * r + k + kk, v, tag_u);
+          for (int s2 = 0; s2 < 16; ++s2) v[s2] = 0.f;
+#pragma unroll
+          for (int i = 0; i < RP; ++i) {
+            if (i0 + i < n) {
+              const uint8_t* row = item + (size_t)(i0 + i) * p.p1_row;
+              float acc[NB];
+#pragma unroll
+              for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+#pragma unroll
+              for (int j = 0; j < NU; ++j)
+                if (t + kConsumerThreads * j < nunits) unit_dot_p<FAM, NB>(row, t + kConsumerThreads * j, xr[j], acc);
+#pragma unroll
+              for (int b = 0; b < NB; ++b) v[i * NB + b] = acc[b];
+            }
+          }
+          const float sw = reduce_scatter16(v, lane);
+          float* red = &sm.red[redbuf][0][0];
+          redbuf ^= 1;
+          if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = sw;
+          named_bar_sync(kRedBar, kConsumerThreads);
+          if (t < RP * NB) {
+            const int i = t / NB, b = t % NB;
+            if (i0 + i < n && b < B) {
+              float u = 0.f;
+#pragma unroll
+              for (int w = 0; w < kConsumerWarps; ++w) u += red[w * 16 + t];
+              st_tag(p.ux + (size_t)b * r + k + i0 + i, u, tag_u);
+            }
           }
         }
         ring_release_item(ring.item++, sm);
@@ -434,17 +486,27 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       named_bar_sync(kRedBar, kConsumerThreads);
       stamp(p, l, 2);
 
-      // ---------------------------------------------------------- P-b: own logits, 4 rows per warp
+      // ---------------------------------------------------------- P-b: own logits
+      // A warp takes 8 rows at a time: lane q accumulates the 16-byte chunks q, q+32, ...
+      // of all 8 rows, then a butterfly reduce-scatter leaves the whole dot of row
+      // (lane >> 2) & 7 in lanes 4j..4j+3 (9 shuffles for 8 rows).
+      uint32_t* mask_dst = do_glue ? (p.trace.mask ? p.trace.mask + (size_t)l * B * words : nullptr) : p.mask_out;
       const int rchunks = r * PB / 16;
+      long long pb_wait = 0;   // diagnostics: cycles spent waiting for P2 items
       for (int m0 = 0; m0 < nown; m0 += p.p2_rows_per_item) {
         const int n = min(p.p2_rows_per_item, nown - m0);
         const uint8_t* item = ring_next(ring, (uint32_t)n * p.p2_stride);
+        const long long wt0 = diag_clock(p);
         ring_wait_item(ring.item, sm, p);
+        pb_wait += diag_clock(p) - wt0;
         if (m0 == 0) stamp(p, l, 12);
-        for (int mb = warp * 4; mb < n; mb += kConsumerWarps * 4) {
-          float acc[4][NB];
+        for (int mb = warp * 8; mb < n; mb += kConsumerWarps * 8) {
+          const uint8_t* rows[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
+          for (int i = 0; i < 8; ++i) rows[i] = item + (size_t)min(mb + i, n - 1) * p.p2_stride;   // past n: repeats, unused
+          float acc[8][NB];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
 #pragma unroll
             for (int b = 0; b < NB; ++b) acc[i][b] = 0.f;
           for (int q = lane; q < rchunks; q += 32) {
@@ -453,13 +515,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
 #pragma unroll
               for (int b = 0; b < NB; ++b) uu[b] = *reinterpret_cast<const float4*>(u_s + b * r + 4 * q);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                if (mb + i < n) {
-                  const float4 w = *reinterpret_cast<const float4*>(item + (size_t)(mb + i) * p.p2_stride + 16 * q);
+              for (int i = 0; i < 8; ++i) {
+                const float4 w = *reinterpret_cast<const float4*>(rows[i] + 16 * q);
 #pragma unroll
-                  for (int b = 0; b < NB; ++b)
-                    acc[i][b] = fmaf(w.x, uu[b].x, fmaf(w.y, uu[b].y, fmaf(w.z, uu[b].z, fmaf(w.w, uu[b].w, acc[i][b]))));
-                }
+                for (int b = 0; b < NB; ++b)
+                  acc[i][b] = fmaf(w.w, uu[b].w, fmaf(w.z, uu[b].z, fmaf(w.y, uu[b].y, fmaf(w.x, uu[b].x, acc[i][b]))));
               }
             } else {
               float4 u0[NB], u1[NB];
@@ -469,40 +529,35 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
                 u1[b] = *reinterpret_cast<const float4*>(u_s + b * r + 8 * q + 4);
               }
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                if (mb + i < n) {
-                  const uint4 w = *reinterpret_cast<const uint4*>(item + (size_t)(mb + i) * p.p2_stride + 16 * q);
-                  const float2 a = h2f2(w.x), bb = h2f2(w.y), cc = h2f2(w.z), e = h2f2(w.w);
+              for (int i = 0; i < 8; ++i) {
+                const uint4 w = *reinterpret_cast<const uint4*>(rows[i] + 16 * q);
+                const float2 a = h2f2(w.x), bb = h2f2(w.y), cc = h2f2(w.z), e = h2f2(w.w);
 #pragma unroll
-                  for (int b = 0; b < NB; ++b) {
-                    float s = acc[i][b];
-                    s = fmaf(a.x, u0[b].x, s); s = fmaf(a.y, u0[b].y, s); s = fmaf(bb.x, u0[b].z, s);
-                    s = fmaf(bb.y, u0[b].w, s); s = fmaf(cc.x, u1[b].x, s); s = fmaf(cc.y, u1[b].y, s);
-                    s = fmaf(e.x, u1[b].z, s); s = fmaf(e.y, u1[b].w, s);
-                    acc[i][b] = s;
-                  }
+                for (int b = 0; b < NB; ++b) {
+                  float s = acc[i][b];
+                  s = fmaf(a.x, u0[b].x, s); s = fmaf(a.y, u0[b].y, s); s = fmaf(bb.x, u0[b].z, s);
+                  s = fmaf(bb.y, u0[b].w, s); s = fmaf(cc.x, u1[b].x, s); s = fmaf(cc.y, u1[b].y, s);
+                  s = fmaf(e.x, u1[b].z, s); s = fmaf(e.y, u1[b].w, s);
+                  acc[i][b] = s;
                 }
               }
             }
           }
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int b = 0; b < NB; ++b) acc[i][b] = warp_sum(acc[i][b]);
-          if (lane < 4 && mb + lane < n) {
-            const int m = mb + lane;
-            const uint8_t* prow = item + (size_t)m * p.p2_stride;
-            const float ti = *reinterpret_cast<const float*>(prow + (size_t)r * PB);
+          float dot[NB];
+          reduce_scatter8<NB>(acc, lane, dot);
+          const int m = mb + ((lane >> 2) & 7);
+          if ((lane & 3) == 0 && m < n) {
+            const float ti = *reinterpret_cast<const float*>(rows[(lane >> 2) & 7] + (size_t)r * PB);
             const int i = c + (m0 + m) * G;
             uint32_t bits = 0;
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
-              float lgv = acc[0][b];
-#pragma unroll
-              for (int ii = 1; ii < 4; ++ii) if (lane == ii) lgv = acc[ii][b];
               if (b < B) {
-                const float lg = lgv - ti;
-                if (lg > 0.f) bits |= 1u << b;
+                const float lg = dot[b] - ti;
+                if (lg > 0.f) {
+                  bits |= 1u << b;
+                  if (mask_dst) atomicOr(mask_dst + (size_t)b * words + (i >> 5), 1u << (i & 31));
+                }
                 if (p.logits_out) p.logits_out[(size_t)b * f + i] = lg;
                 if (p.trace.logits) p.trace.logits[((size_t)l * B + b) * f + i] = lg;
               }
@@ -514,129 +569,34 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       }
       named_bar_sync(kRedBar, kConsumerThreads);
       stamp(p, l, 7);
+      stamp_val(p, l, 18, pb_wait);
 
-      // ---------------------------------------------------------- bitmap exchange
-      // publish this block's per-token bitmap words (bit m of word m/32 = own neuron m)
-      for (int qb = warp; qb < W * B; qb += kConsumerWarps) {
-        const int q = qb % W, b = qb / W;
-        const int m = 32 * q + lane;
-        const uint32_t bit = (m < nown) ? ((sm.own_bits[m] >> b) & 1u) : 0u;
-        const uint32_t word = __ballot_sync(0xffffffffu, bit != 0);
-        if (lane == 0) st_tag_u(p.bx + ((size_t)b * G + c) * W + q, word, tag_b);
-      }
-      for (int base = 0; base < B * G * W; base += 8 * kConsumerThreads) {
-        uint64_t w[8];
-        poll_words<8>(p.bx + base, t, kConsumerThreads, B * G * W - base, tag_b, w, sm, p);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          if (base + t + k * kConsumerThreads < B * G * W) bm[base + t + k * kConsumerThreads] = (uint32_t)w[k];
-      }
-      named_bar_sync(kRedBar, kConsumerThreads);
-      stamp(p, l, 14);
-      // active count per owner block (union over tokens), prefix over blocks
-      if (t < G) {
-        int n = 0;
-        for (int q = 0; q < W; ++q) {
-          uint32_t un = 0;
-          for (int b = 0; b < B; ++b) un |= bm[((size_t)b * G + t) * W + q];
-          n += __popc(un);
-        }
-        sm.cstart[t + 1] = n;
-      }
-      named_bar_sync(kRedBar, kConsumerThreads);
-      if (warp == 0) {   // inclusive scan over the G (<= kMaxGrid) block counts
-        int carry = 0;
-        for (int c0 = 0; c0 < G; c0 += 32) {
-          int v = (c0 + lane < G) ? sm.cstart[c0 + lane + 1] : 0;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int u = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += u;
-          }
-          if (c0 + lane < G) sm.cstart[c0 + lane + 1] = v + carry;
-          carry += __shfl_sync(0xffffffffu, v, 31);
-        }
-        if (lane == 0) { sm.cstart[0] = 0; sm.count = carry; }
-      }
-      named_bar_sync(kRedBar, kConsumerThreads);
-      stamp(p, l, 15);
-      const int count = sm.count;
-      // this block's even share of the active neurons, in (owner block, owner position) order
-      const int a0 = (int)((long long)c * count / G), a1 = (int)((long long)(c + 1) * count / G);
-      nlist = min(a1 - a0, kMaxList);
-      if (t < G && sm.cstart[t] < a1 && sm.cstart[t + 1] > a0) {
-        int pos = sm.cstart[t];
-        for (int q = 0; q < W && pos < a1; ++q) {
-          uint32_t un = 0;
-          for (int b = 0; b < B; ++b) un |= bm[((size_t)b * G + t) * W + q];
-          while (un && pos < a1) {
-            const int bit = __ffs(un) - 1;
-            un &= un - 1;
-            if (pos >= a0 && pos - a0 < kMaxList) {
-              const int m = 32 * q + bit;
-              const int e = pos - a0;
-              uint32_t tb = 0;
-              for (int b = 0; b < B; ++b) tb |= ((bm[((size_t)b * G + t) * W + q] >> bit) & 1u) << b;
-              sm.list[e] = t + m * G;
-              sm.list_bits[e] = (uint8_t)tb;
-            }
-            ++pos;
-          }
-        }
-      }
-      if (t == 0 && c == 0 && do_ffn) {
-        atomicAdd(p.active_total, (unsigned long long)count);
-        if (p.layer_count) p.layer_count[l] = count;
-      }
-      if (t == 0 && a1 - a0 > kMaxList) atomicExch(p.err, DEV_ERR_LIST);
-      // mask words (predict output or trace): block c assembles words w = c, c+G, ...
-      uint32_t* mask_dst = do_glue ? (p.trace.mask ? p.trace.mask + (size_t)l * B * words : nullptr) : p.mask_out;
-      if (mask_dst) {
-        for (int wb = c + G * warp; wb < words * B; wb += G * kConsumerWarps) {
-          const int b = wb / words, w = wb % words;
-          const int i = 32 * w + lane;
-          const int oc = i % G, om = i / G;
-          const uint32_t bit = (bm[((size_t)b * G + oc) * W + (om >> 5)] >> (om & 31)) & 1u;
-          const uint32_t word = __ballot_sync(0xffffffffu, bit != 0);
-          if (lane == 0) mask_dst[(size_t)b * words + w] = word;
-        }
-      }
-      // trace: ascending index list and count of the layer (the union over tokens)
-      if (trace_idx && c == 0) {
+      // ---------------------------------------------------------- own active list
+      // Block c processes the active neurons it owns, i = c + m*G in ascending m: the
+      // list needs nothing from other blocks.
+      if (warp == 0) {
         int base = 0;
-        for (int w0 = 0; w0 < words; w0 += kConsumerThreads) {
-          const int w = w0 + t;
-          uint32_t un = 0;
-          if (w < words)
-            for (int j = 0; j < 32; ++j) {
-              const int i = 32 * w + j, oc = i % G, om = i / G;
-              uint32_t bit = 0;
-              for (int b = 0; b < B; ++b) bit |= (bm[((size_t)b * G + oc) * W + (om >> 5)] >> (om & 31)) & 1u;
-              un |= bit << j;
-            }
-          const int cnt = __popc(un);
-          int incl = cnt;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
+        for (int mm = 0; mm < nown; mm += 32) {
+          const int m = mm + lane;
+          const uint32_t tb = (m < nown) ? sm.own_bits[m] : 0u;
+          const uint32_t bal = __ballot_sync(0xffffffffu, tb != 0u);
+          if (tb) {
+            const int e = base + __popc(bal & ((1u << lane) - 1u));
+            sm.list[e] = c + m * G;
+            sm.list_bits[e] = (uint8_t)tb;
           }
-          if (lane == 31) sm.scan[warp] = incl;
-          named_bar_sync(kRedBar, kConsumerThreads);
-          int wb = 0, tot = 0;
-          for (int q = 0; q < kConsumerWarps; ++q) { if (q < warp) wb += sm.scan[q]; tot += sm.scan[q]; }
-          int pos = base + wb + incl - cnt;
-          if (p.trace.idx)
-            while (un) {
-              const int bit = __ffs(un) - 1;
-              un &= un - 1;
-              p.trace.idx[(size_t)l * f + pos++] = w * 32 + bit;
-            }
-          base += tot;
-          named_bar_sync(kRedBar, kConsumerThreads);
+          base += __popc(bal);
         }
-        if (t == 0 && p.trace.count) p.trace.count[l] = base;
+        if (lane == 0) sm.count = base;
       }
+      named_bar_sync(kRedBar, kConsumerThreads);
+      nlist = sm.count;
+      if (t == 0 && do_ffn && nlist > 0) {
+        atomicAdd(p.active_total, (unsigned long long)nlist);
+        if (p.layer_count) atomicAdd(p.layer_count + l, nlist);
+      }
+      stamp(p, l, 15);
+      stamp_val(p, l, 14, nlist);
     } else if (do_ffn) {
       // ---------------------------------------------------------- list from the caller
       int cnt = __ldg(p.count_in);
@@ -669,78 +629,146 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     }
     stamp(p, l, 3);
 
-    // ------------------------------------------------------------ F: gather + scatter in batches
-    float y[NB][NU][UE];
+    // ------------------------------------------------------------ F: windows of landed records
+    // A window is the next record and the ones after it that have already landed (up
+    // to KW).  Every thread dots its units of the window's gate/up rows with its x units
+    // and a block reduction gives the window's dot products.  Windows are pipelined with
+    // one barrier each: after window w's barrier, 16 threads form h of window w while
+    // every thread adds h * (its units of each down row) of window w-1 into its y units.
+    // Thread 0 chooses window w+1 before that barrier.  A record's sums do not depend on
+    // how the records fall into windows.
+    float y[NU][NB][UE];
 #pragma unroll
-    for (int b = 0; b < NB; ++b)
+    for (int j = 0; j < NU; ++j)
 #pragma unroll
-      for (int j = 0; j < NU; ++j)
+      for (int b = 0; b < NB; ++b)
 #pragma unroll
-        for (int e = 0; e < UE; ++e) y[b][j][e] = 0.f;
-    // Records stream through the ring in windows of p.batch; warp k of a window forms the
-    // dot products of its record and flags h, and every warp adds each record's down row
-    // as soon as that record's h is flagged (no block-wide barrier in between).
-    const int hval = l + 1;
-    for (int e0 = 0; e0 < nlist; e0 += p.batch) {
-      const int nb = min(p.batch, nlist - e0);
-      uint32_t rpos[kMaxBatch];
-      const uint32_t item0 = ring.item;
+        for (int e = 0; e < UE; ++e) y[j][b][e] = 0.f;
+    constexpr int NV = (ACT == PI_REGLU) ? 2 : 1;
+    constexpr int KW = (16 / (NB * NV) < 8) ? 16 / (NB * NV) : 8;   // 16 reduced values, 8 records
+    // window cap: one window and one more record always fit in the ring together, so
+    // waiting for a record while a window is held can never block the producer
+    const int kw = min(KW, p.rec_window);
+    long long f_wait = 0;   // diagnostics: cycles thread 0 waits for records
+    // thread 0: the window that starts at list position e (ring item `item`): the records
+    // from there that have landed, 0 if none has
+    auto choose = [&](int e, uint32_t item) {
+      int nb = 0;
+      while (nb < kw && e + nb < nlist && ring_item_ready(item + nb, sm)) ++nb;
+      return nb;
+    };
+    uint32_t item_e = ring.item;
+    bool first = true;   // the first window is always chosen with a wait
+    int nwin = 0;        // diagnostics: windows so far
+    int wb = 0;          // buffer of the current window
+    int nb_prev = 0;     // records of the previous window, whose down rows are still to add
+    uint32_t pos_prev[KW];
 #pragma unroll
-      for (int k = 0; k < kMaxBatch; ++k)
-        rpos[k] = (k < nb) ? (uint32_t)(ring_next(ring, (uint32_t)p.rec_stride) - ring.base) : 0u;
-      if (warp < nb) {
-        uint32_t pos = rpos[0];
-#pragma unroll
-        for (int k = 1; k < kMaxBatch; ++k) if (warp == k) pos = rpos[k];
-        const uint8_t* rec = ring.base + pos;
-        ring_wait_item(item0 + warp, sm, p);
-        if (e0 == 0 && warp == 0) stamp(p, l, 5);
-        float ua[NB], ga[NB];
-        if constexpr (ACT == PI_REGLU) {
-          warp_dot_w2<FAM, NB>(rec + p.up_off, rec + p.gate_off, xs, d, ua, ga);
-        } else {
-          warp_dot_w<FAM, NB>(rec + p.up_off, xs, d, ua);
-#pragma unroll
-          for (int b = 0; b < NB; ++b) ga[b] = 0.f;
+    for (int kk = 0; kk < KW; ++kk) pos_prev[kk] = 0;
+    for (int e = 0; e < nlist || nb_prev > 0;) {
+      if (e < nlist && (first || *(volatile int*)&sm.win[wb] == 0)) {
+        // not chosen before the last barrier: wait for its first record (only the previous
+        // window is held, so the producer can place it), then choose
+        named_bar_sync(kRedBar, kConsumerThreads);   // everyone has read sm.win[wb]
+        if (t == 0) {
+          const long long wt0 = diag_clock(p);
+          ring_wait_item(item_e, sm, p);
+          f_wait += diag_clock(p) - wt0;
+          if (e == 0) stamp(p, l, 5);
+          sm.win[wb] = max(1, choose(e, item_e));
         }
-        if (lane == 0) {
-          const int e = e0 + warp;
-          const uint32_t bits = sm.list_bits[e];
-          const float bi = *reinterpret_cast<const float*>(rec + p.bias_off);
+        named_bar_sync(kRedBar, kConsumerThreads);
+      }
+      first = false;
+      const int nb = (e < nlist) ? *(volatile int*)&sm.win[wb] : 0;
+      if (p.phase_clk && nwin < 16 && nb > 0) {
+        stamp(p, l, 32 + 2 * nwin);
+        stamp_val(p, l, 33 + 2 * nwin, nb);
+      }
+      nwin += (nb > 0);
+      uint32_t pos[KW];
+      float v[16];
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2) v[s2] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < KW; ++kk) {
+        pos[kk] = 0;
+        if (kk < nb) {
+          pos[kk] = ring_place(ring.head, (uint32_t)p.rec_stride, ring.cap);
+          ring_wait_item(item_e + kk, sm, p);   // landed already: makes the data visible here
+          const uint8_t* rec = ring.base + pos[kk];
+          float au[NB], ag[NB];
+#pragma unroll
+          for (int b = 0; b < NB; ++b) au[b] = ag[b] = 0.f;
+#pragma unroll
+          for (int j = 0; j < NU; ++j) {
+            const int q = t + kConsumerThreads * j;
+            if (q < nunits) {
+              unit_dot<FAM, NB>(rec + p.up_off, d, q, xr[j], au);
+              if constexpr (ACT == PI_REGLU) unit_dot<FAM, NB>(rec + p.gate_off, d, q, xr[j], ag);
+            }
+          }
 #pragma unroll
           for (int b = 0; b < NB; ++b) {
-            float a;
-            if constexpr (ACT == PI_REGLU) a = fmaxf(ga[b] + bi, 0.f) * ua[b];
-            else a = fmaxf(ua[b] + bi, 0.f);
-            sm.hbuf[e][b] = ((bits >> b) & 1u) ? a : 0.f;
-          }
-          __threadfence_block();
-          *(volatile int*)&sm.hflag[e] = hval;
-        }
-        __syncwarp();
-      }
-      for (int k = 0; k < nb; ++k) {
-        uint32_t pos = rpos[0];
-#pragma unroll
-        for (int kk = 1; kk < kMaxBatch; ++kk) if (k == kk) pos = rpos[kk];
-        const int e = e0 + k;
-        if (*(volatile int*)&sm.hflag[e] != hval) {
-          const uint64_t t0 = wait_start();
-          while (*(volatile int*)&sm.hflag[e] != hval) {
-            if (aborted(sm)) break;
-            if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); break; }
+            v[(kk * NB + b) * NV] = au[b];
+            if constexpr (ACT == PI_REGLU) v[(kk * NB + b) * NV + 1] = ag[b];
           }
         }
-        __threadfence_block();
-        ring_wait_item(item0 + k, sm, p);   // completed already: makes the data visible here
-        float h[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) h[b] = sm.hbuf[e][b];
-        axpy_units<FAM, NB, NU>(ring.base + pos + p.down_off, nunits, d, h, y);
-        ring_release_item(item0 + k, sm);
       }
-      ring.item = item0 + nb;
+      float* red = &sm.red[redbuf][0][0];
+      if (nb > 0) {
+        const float sw = reduce_scatter16(v, lane);
+        redbuf ^= 1;
+        if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = sw;
+      }
+      const int dw = (nwin == 2 || nwin == 3) ? 22 + 3 * (nwin - 2) : -1;   // diagnostics: windows 1, 2
+      if (dw >= 0) stamp(p, l, dw);
+      // the next window, if its records have landed already (never blocks)
+      if (t == 0) sm.win[wb ^ 1] = (e + nb < nlist) ? choose(e + nb, item_e + nb) : 0;
+      named_bar_sync(kRedBar, kConsumerThreads);
+      if (dw >= 0) stamp(p, l, dw + 1);
+      if (t < nb * NB) {
+        const int kk = t / NB, b = t % NB;
+        float su = 0.f, sg = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          su += red[w * 16 + (kk * NB + b) * NV];
+          if constexpr (ACT == PI_REGLU) sg += red[w * 16 + (kk * NB + b) * NV + 1];
+        }
+        uint32_t mypos = pos[0];
+#pragma unroll
+        for (int k2 = 1; k2 < KW; ++k2) if (k2 == kk) mypos = pos[k2];
+        const float bi = *reinterpret_cast<const float*>(ring.base + mypos + p.bias_off);
+        float a;
+        if constexpr (ACT == PI_REGLU) a = fmaxf(sg + bi, 0.f) * su;
+        else a = fmaxf(su + bi, 0.f);
+        sm.hbuf[wb][kk][b] = (b < B && ((sm.list_bits[e + kk] >> b) & 1u)) ? a : 0.f;
+      }
+      // down rows of the previous window (its h was formed before this barrier)
+#pragma unroll
+      for (int kk = 0; kk < KW; ++kk) {
+        if (kk < nb_prev) {
+          float h[NB];
+#pragma unroll
+          for (int b = 0; b < NB; ++b) h[b] = sm.hbuf[wb ^ 1][kk][b];
+          const uint8_t* drow = ring.base + pos_prev[kk] + p.down_off;
+#pragma unroll
+          for (int j = 0; j < NU; ++j)
+            if (t + kConsumerThreads * j < nunits) unit_axpy<FAM, NB>(drow, d, t + kConsumerThreads * j, h, y[j]);
+          ring_release_item(item_e - nb_prev + kk, sm);
+        }
+      }
+      if (dw >= 0) stamp(p, l, dw + 2);
+#pragma unroll
+      for (int kk = 0; kk < KW; ++kk) pos_prev[kk] = pos[kk];
+      nb_prev = nb;
+      item_e += nb;
+      e += nb;
+      wb ^= 1;
     }
+    ring.item = item_e;
+    stamp(p, l, 20);
+    stamp_val(p, l, 21, nwin);
     // publish the partial y of this block as tagged words
     {
       uint64_t* part = p.px + (size_t)c * B * d;
@@ -752,11 +780,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           if (b < B && q < nunits) {
             uint64_t* dst = part + (size_t)b * d + (size_t)q * UE;
 #pragma unroll
-            for (int e = 0; e < UE; e += 2) st_tag2(dst + e, y[b][j][e], y[b][j][e + 1], tag_p);
+            for (int e = 0; e < UE; e += 2) st_tag2(dst + e, y[j][b][e], y[j][b][e + 1], tag_p);
           }
         }
     }
     stamp(p, l, 4);
+    stamp_val(p, l, 19, f_wait);
 
     // ------------------------------------------------------------ R: slice reduce
     if (slice_owner) {
@@ -971,33 +1000,19 @@ __global__ void __launch_bounds__(kThreads, 1) barrier_probe_kernel(const FusedP
   }
 }
 
-// Largest per-thread unit count of each (family, tokens) instantiation.
-template <int FAM, int NB> struct NUof;
-template <> struct NUof<FAM_F32, 1> { static constexpr int v = 2; };
-template <> struct NUof<FAM_F32, 2> { static constexpr int v = 2; };
-template <> struct NUof<FAM_F32, 4> { static constexpr int v = 2; };
-template <> struct NUof<FAM_F16, 1> { static constexpr int v = 3; };
-template <> struct NUof<FAM_F16, 2> { static constexpr int v = 2; };
-template <> struct NUof<FAM_F16, 4> { static constexpr int v = 1; };
-template <> struct NUof<FAM_Q4, 1> { static constexpr int v = 1; };
-template <> struct NUof<FAM_Q4, 2> { static constexpr int v = 1; };
+constexpr int ue_of(int fam) { return fam == FAM_F32 ? 4 : fam == FAM_F16 ? 8 : 16; }
 
-constexpr int ue_of(int fam) { return fam == FAM_F32 ? 4 : fam == FAM_F16 ? 8 : 32; }
-
-int nu_max(int fam, int nb) {
-  switch (fam) {
-    case FAM_F32: return 2;
-    case FAM_F16: return nb == 1 ? 3 : nb == 2 ? 2 : 1;
-    case FAM_Q4: return nb <= 2 ? 1 : 0;
-  }
-  return 0;
+// Largest unit count per consumer thread that each (family, tokens) pair is built for;
+// a launch takes the smallest count that covers d, so x and y in registers stay small.
+constexpr int nu_max(int fam, int nb) {
+  return fam == FAM_F32 ? (nb == 4 ? 1 : 2) : fam == FAM_F16 ? (nb == 1 ? 3 : nb == 2 ? 2 : 1) : (nb <= 2 ? 1 : 0);
 }
 
 int nb_of(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 0; }
 
-template <int FAM, int ACT, int NB>
+template <int FAM, int ACT, int NB, int NU>
 cudaError_t launch_t(const FusedParams& p, size_t smem, cudaStream_t stream) {
-  auto kern = fused_kernel<FAM, ACT, NB, NUof<FAM, NB>::v>;
+  auto kern = fused_kernel<FAM, ACT, NB, NU>;
   static int configured = 0;   // the attribute is per function; raise it when a launch needs more
   if ((int)smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1008,13 +1023,24 @@ cudaError_t launch_t(const FusedParams& p, size_t smem, cudaStream_t stream) {
   return cudaLaunchCooperativeKernel((const void*)kern, dim3(p.grid), dim3(kThreads), args, smem, stream);
 }
 
+template <int FAM, int ACT, int NB>
+cudaError_t launch_nu(const FusedParams& p, size_t smem, cudaStream_t stream) {
+  constexpr int M = nu_max(FAM, NB);
+  const int nunits = p.d / ue_of(FAM);
+  const int nu = (nunits + kConsumerThreads - 1) / kConsumerThreads;
+  if constexpr (M >= 1) if (nu <= 1) return launch_t<FAM, ACT, NB, 1>(p, smem, stream);
+  if constexpr (M >= 2) if (nu == 2) return launch_t<FAM, ACT, NB, 2>(p, smem, stream);
+  if constexpr (M >= 3) if (nu == 3) return launch_t<FAM, ACT, NB, 3>(p, smem, stream);
+  return cudaErrorNotSupported;
+}
+
 template <int FAM, int ACT>
 cudaError_t launch_nb(int B, const FusedParams& p, size_t smem, cudaStream_t stream) {
   switch (nb_of(B)) {
-    case 1: return launch_t<FAM, ACT, 1>(p, smem, stream);
-    case 2: return launch_t<FAM, ACT, 2>(p, smem, stream);
+    case 1: return launch_nu<FAM, ACT, 1>(p, smem, stream);
+    case 2: return launch_nu<FAM, ACT, 2>(p, smem, stream);
     case 4:
-      if constexpr (FAM != FAM_Q4) return launch_t<FAM, ACT, 4>(p, smem, stream);
+      if constexpr (FAM != FAM_Q4) return launch_nu<FAM, ACT, 4>(p, smem, stream);
       else return cudaErrorNotSupported;
   }
   return cudaErrorNotSupported;
@@ -1033,12 +1059,10 @@ bool fused_supported(int family, int B, int d) {
 size_t fused_fixed_smem(int B, int d, int r, int grid, int nown_max, int family) {
   const int nb = nb_of(B) ? nb_of(B) : 4;
   const size_t xbytes = family == FAM_F32 ? 4 : 2;
-  const size_t W = (size_t)(nown_max + 31) / 32;
   return ((sizeof(Smem) + 127) / 128) * 128 + (size_t)nb * d * xbytes + (size_t)nb * r * sizeof(float) +
-         (size_t)kConsumerWarps * nb * kMaxColGroups * 32 * sizeof(float) + (size_t)nb * grid * W * 4 + 128;
+         (size_t)kConsumerWarps * nb * kMaxColGroups * 32 * sizeof(float) + 128;
 }
 
-int fused_max_batch() { return kMaxBatch; }
 
 cudaError_t launch_fused(int family, int act, int B, const FusedParams& p, size_t smem, cudaStream_t stream) {
   if (family == FAM_F32)

@@ -29,6 +29,7 @@ constexpr int kMaxOwn = 512;          // owned neurons per block (d_ff <= 512 * 
 constexpr int kMaxList = 512;         // active neurons a block may process in one layer
 constexpr int kMaxLayers = 100;       // layers of one pi_decode_stack call
 constexpr int kMaxGrid = 256;         // blocks of the fused kernel (SMs)
+constexpr int kDiagSlots = 64;        // diagnostic stamps per block and layer
 
 // Library-owned, re-laid-out layer.
 struct LayerDev {
@@ -72,7 +73,6 @@ struct pi_workspace {
   uint64_t* px;      // [grid][B_max][d_max]    tagged y partials
   uint64_t* vx;      // [B_max][d_max]          tagged x + y
   uint64_t* sx;      // [B_max][grid][2]        tagged slice sums and sums of squares
-  uint64_t* bx;      // [B_max][grid][W_max]    tagged own-neuron bitmaps
   uint32_t* bar;     // [0] probe barrier count, [1] exit count, [2] launch epoch (tags)
   int* err;          // device error word
   unsigned long long* active_total;  // running sum of active-list lengths (all calls)
@@ -91,7 +91,8 @@ struct FusedParams {
   int L, B, d, f, r;
   int grid;
   int row_bytes, rec_stride, gate_off, up_off, down_off, bias_off, p1_row, p2_stride;
-  int ring_bytes, p1_rows_per_item, p2_rows_per_item, nown_max, batch;
+  int ring_bytes, p1_rows_per_item, p2_rows_per_item, nown_max;
+  int rec_window;      // records per F window at most (one window and one record fit in the ring)
   int nslices;
   LayerDev layers[kMaxLayers];
   // inputs / outputs
@@ -109,7 +110,6 @@ struct FusedParams {
   uint64_t* px;
   uint64_t* vx;
   uint64_t* sx;
-  uint64_t* bx;              // [B][G][W] tagged bitmaps of the blocks' own neurons
   uint32_t* bar;
   int* err;
   unsigned long long* active_total;
@@ -128,7 +128,6 @@ enum : int { MODE_PREDICT = 1, MODE_FFN = 2, MODE_GLUE = 4 };
 cudaError_t launch_fused(int family, int act, int B, const FusedParams& p, size_t smem_bytes,
                          cudaStream_t stream);
 size_t fused_fixed_smem(int B, int d, int r, int grid, int nown_max, int family);
-int fused_max_batch();
 bool fused_supported(int family, int B, int d);
 cudaError_t launch_barrier_probe(const FusedParams& p, int rounds, cudaStream_t stream);
 

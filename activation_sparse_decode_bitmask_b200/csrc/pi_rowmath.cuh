@@ -1,12 +1,16 @@
 // Row arithmetic of the fused kernel.
-//   warp dots: one warp forms the dot product of a row held in shared memory with the
-//              tokens' x (also in shared memory); lanes stride over 16-byte chunks, the
-//              sum is reduced with shuffles and returned in every lane
-//   axpy:      the down projection y += h * row, one thread per 16-byte unit of y
-// Rows are fp32, fp16 or Q4_0 (32-weight blocks: 16 bytes of nibbles, element j in the
-// low four bits of byte j and element j + 16 in the high four bits, then the fp16 scales
-// of all blocks of the row); x is fp32 for the fp32 family and fp16 otherwise.  Products
-// and sums are formed in fp32.
+//
+// Consumer thread t owns the units q = t + kConsumerThreads * j (j < NU) of every d-long
+// row: 4 elements for fp32, 8 for fp16 and 16 (half a Q4_0 block) for Q4_0.  It keeps
+// its units of every token's x and y in registers as fp32 for a whole layer, so a row's
+// dot product is a per-thread partial sum over the thread's units (the caller reduces
+// the partials across the block) and the down projection y += h * row needs no
+// cross-thread step at all.
+//
+// Q4_0 rows: 32-weight blocks; the row holds the 16 nibble bytes of every block (byte j
+// has element j in its low four bits and element j + 16 in its high four bits), then the
+// fp16 scales of all its blocks.  Value = (code - 8) * scale.  A unit is the low or the
+// high nibbles of one block.  Products and sums are formed in fp32.
 #pragma once
 #include <cuda_fp16.h>
 #include <cstdint>
@@ -19,7 +23,7 @@ namespace pi {
 template <int FAM> struct Fam;
 template <> struct Fam<FAM_F32> { static constexpr int UE = 4;  static constexpr int PB = 4; using X = float; };
 template <> struct Fam<FAM_F16> { static constexpr int UE = 8;  static constexpr int PB = 2; using X = __half; };
-template <> struct Fam<FAM_Q4>  { static constexpr int UE = 32; static constexpr int PB = 2; using X = __half; };
+template <> struct Fam<FAM_Q4>  { static constexpr int UE = 16; static constexpr int PB = 2; using X = __half; };
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -32,187 +36,170 @@ __device__ __forceinline__ float q4_val(uint32_t nibbles_in_bytes, int k) {
   return __uint_as_float(__byte_perm(nibbles_in_bytes, 0x4B000000u, 0x7540 + k)) - 8388616.f;
 }
 
-// Sum over 8 fp16 weights (one 16-byte chunk) times 8 x values.
-__device__ __forceinline__ float dot8_h(const uint4 w, const uint4 xv) {
-  const float2 w0 = h2f2(w.x), w1 = h2f2(w.y), w2 = h2f2(w.z), w3 = h2f2(w.w);
-  const float2 x0 = h2f2(xv.x), x1 = h2f2(xv.y), x2 = h2f2(xv.z), x3 = h2f2(xv.w);
-  float s = w0.x * x0.x;
-  s = fmaf(w0.y, x0.y, s); s = fmaf(w1.x, x1.x, s); s = fmaf(w1.y, x1.y, s);
-  s = fmaf(w2.x, x2.x, s); s = fmaf(w2.y, x2.y, s); s = fmaf(w3.x, x3.x, s); s = fmaf(w3.y, x3.y, s);
-  return s;
+// 8 fp16 values of a 16-byte chunk, widened
+__device__ __forceinline__ void widen8(const uint4 v, float* o) {
+  const float2 a = h2f2(v.x), b = h2f2(v.y), c = h2f2(v.z), e = h2f2(v.w);
+  o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y; o[4] = c.x; o[5] = c.y; o[6] = e.x; o[7] = e.y;
 }
 
-// Warp dot of a row in the p dtype (fp32 for the fp32 family, else fp16) with x.
-// xs: [NB][d] in the family's x type.  acc[b] holds the full sum in every lane.
+// Unit q of every token's x (xs: [NB][d] in the family's x type), widened to fp32.
 template <int FAM, int NB>
-__device__ __forceinline__ void warp_dot_p(const uint8_t* row, const void* xs, int d, float (&acc)[NB]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int b = 0; b < NB; ++b) acc[b] = 0.f;
-  if constexpr (FAM == FAM_F32) {
-    const float4* w4 = reinterpret_cast<const float4*>(row);
-    const float* x = reinterpret_cast<const float*>(xs);
-#pragma unroll 4
-    for (int q = lane; q < d / 4; q += 32) {
-      const float4 w = w4[q];
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const float4 xv = reinterpret_cast<const float4*>(x + (size_t)b * d)[q];
-        acc[b] = fmaf(w.x, xv.x, fmaf(w.y, xv.y, fmaf(w.z, xv.z, fmaf(w.w, xv.w, acc[b]))));
-      }
-    }
-  } else {
-    const uint4* w4 = reinterpret_cast<const uint4*>(row);
-    const __half* x = reinterpret_cast<const __half*>(xs);
-#pragma unroll 4
-    for (int q = lane; q < d / 8; q += 32) {
-      const uint4 w = w4[q];
-#pragma unroll
-      for (int b = 0; b < NB; ++b) acc[b] += dot8_h(w, reinterpret_cast<const uint4*>(x + (size_t)b * d)[q]);
-    }
-  }
-#pragma unroll
-  for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
-}
-
-// Warp dot of a weight row (family format) with x.
-template <int FAM, int NB>
-__device__ __forceinline__ void warp_dot_w(const uint8_t* row, const void* xs, int d, float (&acc)[NB]) {
-  if constexpr (FAM != FAM_Q4) {
-    warp_dot_p<FAM, NB>(row, xs, d, acc);
-  } else {
-    const int lane = threadIdx.x & 31;
-    const uint4* nib = reinterpret_cast<const uint4*>(row);
-    const __half* scl = reinterpret_cast<const __half*>(row + (d >> 1));
-    const __half* x = reinterpret_cast<const __half*>(xs);
-#pragma unroll
-    for (int b = 0; b < NB; ++b) acc[b] = 0.f;
-#pragma unroll 2
-    for (int q = lane; q < d / 32; q += 32) {
-      const uint4 nb = nib[q];
-      const float s = __half2float(scl[q]);
-      const uint32_t wv[4] = {nb.x, nb.y, nb.z, nb.w};
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const uint4* xq = reinterpret_cast<const uint4*>(x + (size_t)b * d + 32 * q);
-        const uint4 xa = xq[0], xb = xq[1], xc = xq[2], xd = xq[3];   // elements 0-7, 8-15, 16-23, 24-31
-        const uint32_t xl[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-        const uint32_t xh[8] = {xc.x, xc.y, xc.z, xc.w, xd.x, xd.y, xd.z, xd.w};
-        float part = 0.f;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint32_t lo = wv[m] & 0x0F0F0F0Fu, hi = (wv[m] >> 4) & 0x0F0F0F0Fu;
-          const float2 l0 = h2f2(xl[2 * m]), l1 = h2f2(xl[2 * m + 1]);   // x[4m .. 4m+3]
-          const float2 h0 = h2f2(xh[2 * m]), h1 = h2f2(xh[2 * m + 1]);   // x[16+4m .. 16+4m+3]
-          part = fmaf(q4_val(lo, 0), l0.x, part); part = fmaf(q4_val(lo, 1), l0.y, part);
-          part = fmaf(q4_val(lo, 2), l1.x, part); part = fmaf(q4_val(lo, 3), l1.y, part);
-          part = fmaf(q4_val(hi, 0), h0.x, part); part = fmaf(q4_val(hi, 1), h0.y, part);
-          part = fmaf(q4_val(hi, 2), h1.x, part); part = fmaf(q4_val(hi, 3), h1.y, part);
-        }
-        acc[b] = fmaf(s, part, acc[b]);
-      }
-    }
-#pragma unroll
-    for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
-  }
-}
-
-// Warp dots of two weight rows (up and gate of one neuron) with x, reading x once.
-template <int FAM, int NB>
-__device__ __forceinline__ void warp_dot_w2(const uint8_t* row_a, const uint8_t* row_b, const void* xs, int d,
-                                            float (&acc_a)[NB], float (&acc_b)[NB]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int b = 0; b < NB; ++b) acc_a[b] = acc_b[b] = 0.f;
-  if constexpr (FAM == FAM_F32) {
-    const float4* wa = reinterpret_cast<const float4*>(row_a);
-    const float4* wb = reinterpret_cast<const float4*>(row_b);
-    const float* x = reinterpret_cast<const float*>(xs);
-#pragma unroll 4
-    for (int q = lane; q < d / 4; q += 32) {
-      const float4 a = wa[q], c = wb[q];
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const float4 xv = reinterpret_cast<const float4*>(x + (size_t)b * d)[q];
-        acc_a[b] = fmaf(a.x, xv.x, fmaf(a.y, xv.y, fmaf(a.z, xv.z, fmaf(a.w, xv.w, acc_a[b]))));
-        acc_b[b] = fmaf(c.x, xv.x, fmaf(c.y, xv.y, fmaf(c.z, xv.z, fmaf(c.w, xv.w, acc_b[b]))));
-      }
-    }
-  } else if constexpr (FAM == FAM_F16) {
-    const uint4* wa = reinterpret_cast<const uint4*>(row_a);
-    const uint4* wb = reinterpret_cast<const uint4*>(row_b);
-    const __half* x = reinterpret_cast<const __half*>(xs);
-#pragma unroll 4
-    for (int q = lane; q < d / 8; q += 32) {
-      const uint4 a = wa[q], c = wb[q];
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const uint4 xv = reinterpret_cast<const uint4*>(x + (size_t)b * d)[q];
-        acc_a[b] += dot8_h(a, xv);
-        acc_b[b] += dot8_h(c, xv);
-      }
-    }
-  } else {
-    warp_dot_w<FAM, NB>(row_a, xs, d, acc_a);
-    warp_dot_w<FAM, NB>(row_b, xs, d, acc_b);
-    return;
-  }
+__device__ __forceinline__ void load_x_unit(const void* xs, int d, int q, float (&xu)[NB][Fam<FAM>::UE]) {
+  constexpr int UE = Fam<FAM>::UE;
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
-    acc_a[b] = warp_sum(acc_a[b]);
-    acc_b[b] = warp_sum(acc_b[b]);
+    if constexpr (FAM == FAM_F32) {
+      const float4 v = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(xs) + (size_t)b * d)[q];
+      xu[b][0] = v.x; xu[b][1] = v.y; xu[b][2] = v.z; xu[b][3] = v.w;
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(xs) + (size_t)b * d + UE * q);
+#pragma unroll
+      for (int c = 0; c < UE / 8; ++c) widen8(src[c], &xu[b][8 * c]);
+    }
   }
 }
 
-// y[b] += h[b] * row for the thread's units (consumer thread t owns units t + kConsumerThreads*j).
-template <int FAM, int NB, int NU>
-__device__ __forceinline__ void axpy_units(const uint8_t* row, int nunits, int d, const float (&h)[NB],
-                                           float (&y)[NB][NU][Fam<FAM>::UE]) {
-  const int t = threadIdx.x;
+// acc[b] += (unit q of a weight row) . xu[b]
+template <int FAM, int NB>
+__device__ __forceinline__ void unit_dot(const uint8_t* row, int d, int q, const float (&xu)[NB][Fam<FAM>::UE],
+                                         float (&acc)[NB]) {
+  if constexpr (FAM == FAM_F32) {
+    const float4 w = reinterpret_cast<const float4*>(row)[q];
 #pragma unroll
-  for (int j = 0; j < NU; ++j) {
-    const int q = t + kConsumerThreads * j;
-    if (q < nunits) {
-      if constexpr (FAM == FAM_F32) {
-        const float4 w = reinterpret_cast<const float4*>(row)[q];
+    for (int b = 0; b < NB; ++b)
+      acc[b] = fmaf(w.w, xu[b][3], fmaf(w.z, xu[b][2], fmaf(w.y, xu[b][1], fmaf(w.x, xu[b][0], acc[b]))));
+  } else if constexpr (FAM == FAM_F16) {
+    float w[8];
+    widen8(reinterpret_cast<const uint4*>(row)[q], w);
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          y[b][j][0] = fmaf(h[b], w.x, y[b][j][0]); y[b][j][1] = fmaf(h[b], w.y, y[b][j][1]);
-          y[b][j][2] = fmaf(h[b], w.z, y[b][j][2]); y[b][j][3] = fmaf(h[b], w.w, y[b][j][3]);
-        }
-      } else if constexpr (FAM == FAM_F16) {
-        const uint4 w = reinterpret_cast<const uint4*>(row)[q];
-        const float2 a = h2f2(w.x), bb = h2f2(w.y), c = h2f2(w.z), e = h2f2(w.w);
+    for (int b = 0; b < NB; ++b) {
+      float s = acc[b], s2 = w[4] * xu[b][4];
+      s = fmaf(w[0], xu[b][0], s); s2 = fmaf(w[5], xu[b][5], s2);
+      s = fmaf(w[1], xu[b][1], s); s2 = fmaf(w[6], xu[b][6], s2);
+      s = fmaf(w[2], xu[b][2], s); s2 = fmaf(w[7], xu[b][7], s2);
+      s = fmaf(w[3], xu[b][3], s);
+      acc[b] = s + s2;
+    }
+  } else {
+    const int blk = q >> 1;
+    const uint4 nb = reinterpret_cast<const uint4*>(row)[blk];
+    const float sc = __half2float(reinterpret_cast<const __half*>(row + (d >> 1))[blk]);
+    const int sh = (q & 1) * 4;
+    const uint32_t wv[4] = {(nb.x >> sh) & 0x0F0F0F0Fu, (nb.y >> sh) & 0x0F0F0F0Fu, (nb.z >> sh) & 0x0F0F0F0Fu,
+                            (nb.w >> sh) & 0x0F0F0F0Fu};
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          y[b][j][0] = fmaf(h[b], a.x, y[b][j][0]);  y[b][j][1] = fmaf(h[b], a.y, y[b][j][1]);
-          y[b][j][2] = fmaf(h[b], bb.x, y[b][j][2]); y[b][j][3] = fmaf(h[b], bb.y, y[b][j][3]);
-          y[b][j][4] = fmaf(h[b], c.x, y[b][j][4]);  y[b][j][5] = fmaf(h[b], c.y, y[b][j][5]);
-          y[b][j][6] = fmaf(h[b], e.x, y[b][j][6]);  y[b][j][7] = fmaf(h[b], e.y, y[b][j][7]);
-        }
-      } else {
-        const uint4 nb = reinterpret_cast<const uint4*>(row)[q];
-        const float s = __half2float(reinterpret_cast<const __half*>(row + (d >> 1))[q]);
-        const uint32_t wv[4] = {nb.x, nb.y, nb.z, nb.w};
-        float hs[NB];
+    for (int b = 0; b < NB; ++b) {
+      float s = 0.f, s2 = 0.f;
 #pragma unroll
-        for (int b = 0; b < NB; ++b) hs[b] = h[b] * s;
+      for (int m = 0; m < 4; ++m) {
+        s = fmaf(q4_val(wv[m], 0), xu[b][4 * m], s);
+        s2 = fmaf(q4_val(wv[m], 1), xu[b][4 * m + 1], s2);
+        s = fmaf(q4_val(wv[m], 2), xu[b][4 * m + 2], s);
+        s2 = fmaf(q4_val(wv[m], 3), xu[b][4 * m + 3], s2);
+      }
+      acc[b] = fmaf(sc, s + s2, acc[b]);
+    }
+  }
+}
+
+// acc[b] += (unit q of a predictor row in the p dtype: fp32 for the fp32 family, else
+// fp16) . xu[b]
+template <int FAM, int NB>
+__device__ __forceinline__ void unit_dot_p(const uint8_t* row, int q, const float (&xu)[NB][Fam<FAM>::UE],
+                                           float (&acc)[NB]) {
+  constexpr int UE = Fam<FAM>::UE;
+  if constexpr (FAM == FAM_F32) {
+    unit_dot<FAM_F32, NB>(row, 0, q, xu, acc);
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(row + (size_t)q * UE * 2);
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint32_t lo = wv[m] & 0x0F0F0F0Fu, hi = (wv[m] >> 4) & 0x0F0F0F0Fu;
+    for (int c = 0; c < UE / 8; ++c) {
+      float w[8];
+      widen8(src[c], w);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float cl = q4_val(lo, k), ch = q4_val(hi, k);
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-              y[b][j][4 * m + k] = fmaf(hs[b], cl, y[b][j][4 * m + k]);
-              y[b][j][4 * m + k + 16] = fmaf(hs[b], ch, y[b][j][4 * m + k + 16]);
-            }
-          }
-        }
+      for (int b = 0; b < NB; ++b) {
+        float s = acc[b], s2 = w[4] * xu[b][8 * c + 4];
+        s = fmaf(w[0], xu[b][8 * c + 0], s); s2 = fmaf(w[5], xu[b][8 * c + 5], s2);
+        s = fmaf(w[1], xu[b][8 * c + 1], s); s2 = fmaf(w[6], xu[b][8 * c + 6], s2);
+        s = fmaf(w[2], xu[b][8 * c + 2], s); s2 = fmaf(w[7], xu[b][8 * c + 7], s2);
+        s = fmaf(w[3], xu[b][8 * c + 3], s);
+        acc[b] = s + s2;
       }
     }
   }
+}
+
+// yu[b] += h[b] * (unit q of a weight row)
+template <int FAM, int NB>
+__device__ __forceinline__ void unit_axpy(const uint8_t* row, int d, int q, const float (&h)[NB],
+                                          float (&yu)[NB][Fam<FAM>::UE]) {
+  if constexpr (FAM == FAM_F32) {
+    const float4 w = reinterpret_cast<const float4*>(row)[q];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      yu[b][0] = fmaf(h[b], w.x, yu[b][0]); yu[b][1] = fmaf(h[b], w.y, yu[b][1]);
+      yu[b][2] = fmaf(h[b], w.z, yu[b][2]); yu[b][3] = fmaf(h[b], w.w, yu[b][3]);
+    }
+  } else if constexpr (FAM == FAM_F16) {
+    float w[8];
+    widen8(reinterpret_cast<const uint4*>(row)[q], w);
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) yu[b][e] = fmaf(h[b], w[e], yu[b][e]);
+  } else {
+    const int blk = q >> 1;
+    const uint4 nb = reinterpret_cast<const uint4*>(row)[blk];
+    const float sc = __half2float(reinterpret_cast<const __half*>(row + (d >> 1))[blk]);
+    const int sh = (q & 1) * 4;
+    const uint32_t wv[4] = {(nb.x >> sh) & 0x0F0F0F0Fu, (nb.y >> sh) & 0x0F0F0F0Fu, (nb.z >> sh) & 0x0F0F0F0Fu,
+                            (nb.w >> sh) & 0x0F0F0F0Fu};
+    float hs[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) hs[b] = h[b] * sc;
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float cv = q4_val(wv[m], k);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) yu[b][4 * m + k] = fmaf(hs[b], cv, yu[b][4 * m + k]);
+      }
+  }
+}
+
+// Butterfly reduce-scatter of 16 per-lane values across the warp: on return every lane
+// holds the warp's sum of value (lane >> 1).  The pairing of the additions is the same
+// for every value, so a value's sum does not depend on its slot.
+__device__ __forceinline__ float reduce_scatter16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool up = lane & 16;
+    const float send = up ? v[i] : v[i + 8];
+    const float keep = up ? v[i + 8] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool up = lane & 8;
+    const float send = up ? v[i] : v[i + 4];
+    const float keep = up ? v[i + 4] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool up = lane & 4;
+    const float send = up ? v[i] : v[i + 2];
+    const float keep = up ? v[i + 2] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  {
+    const bool up = lane & 2;
+    const float send = up ? v[0] : v[1];
+    const float keep = up ? v[1] : v[0];
+    v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
 }  // namespace pi

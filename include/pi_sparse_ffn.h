@@ -123,6 +123,8 @@ typedef struct pi_workspace pi_workspace;
  *   mask   [L][B][f/32] u32
  *   idx    [L][f] i32; only the first count[l] entries of layer l are written
  *   count  [L] i32
+ *   idx and count are the compaction of the layer's mask, so they are filled only
+ *   together and only with mask (PI_ERR_ARG otherwise).
  *   y      [L][B][d] f32, the FFN output before the residual and the normalisation */
 typedef struct {
   void* x;
@@ -196,18 +198,19 @@ pi_status pi_workspace_layer_counts(pi_workspace* ws, int32_t* host_out, int L);
 pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaStream_t stream);
 
 /* Diagnostic: with `on`, every later pi_decode_stack on this workspace records each
- * block's SM cycle counter at 20 points of every layer. The consumer warps record 0-8:
- * layer start, predictor rows done, after the first grid barrier, own active list ready,
- * FFN done, after the second barrier, slice reduce done, after the third barrier, and
- * glue done. The producer warp records 9-11: waiting for the active list, list
- * received, and all of the layer's weight rows issued; 12 and 13 mark the first
- * predictor item landing (P2, P1); 14-17 split the bitmap and glue exchanges (bitmaps
- * read, prefix formed, moments read, v read). With `on` = 2 the stamps come from
- * the GPU's global nanosecond timer instead, so blocks can be compared with one another.
- * With `on` = 0 recording stops and the buffer is freed. */
+ * block's SM cycle counter at up to 64 points of every layer. Consumer warps: 0 layer
+ * start, 1 u rows published, 2 u received, 7 logits done, 15 own active list formed,
+ * 3 list handed to the producer, 5 first record landed, 4 FFN partials published,
+ * 6 slice reduce done, 16 moments read, 17 v read, 8 glue done. Producer warp: 9 waits
+ * for the list, 10 list received, 11 all records issued; 12 and 13 mark the first
+ * predictor item landing (P2, P1). Slot 14 holds the block's record count, 18 the
+ * cycles spent waiting for P2 rows, 19 those spent waiting for records, and 32-63 the
+ * start and size of up to 16 F windows. With `on` = 2
+ * the stamps come from the GPU's global nanosecond timer instead, so blocks can be
+ * compared with one another. With `on` = 0 recording stops and the buffer is freed. */
 pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on);
 
-/* Copy the first n stamps ([grid][L_max][20], int64) to host memory (synchronous). */
+/* Copy the first n stamps ([grid][L_max][64], int64) to host memory (synchronous). */
 pi_status pi_diag_phase_clocks_read(pi_workspace* ws, long long* host_out, size_t n);
 
 /* Blocks per launch of the fused kernel on this workspace's device (its SM count). */
@@ -236,8 +239,7 @@ pi_status pi_predict(const pi_layer* layer, const void* x, int B, uint32_t* mask
  *   PI_OK, PI_ERR_TIMEOUT (a bounded device-side wait gave up) or PI_ERR_DEVICE (a
  *   device-side check failed). After an error the scratch is reset on the device for
  *   the next call.
- * Scratch needed: 256 + round256(B * rank * 8) + round256(B * G * W * 8) bytes, where
- *   G is the SM count and W = ceil(ceil(d_ff / G) / 32). A shape that needs more than
+ * Scratch needed: 256 + round256(B * rank * 8) bytes. A shape that needs more than
  *   PI_NOALLOC_SCRATCH_BYTES returns PI_ERR_UNSUPPORTED and enqueues nothing.
  * Set-up: the first call on each device takes the array's address, clears it and
  *   synchronises `stream` before it returns. Make that first call before any stream

@@ -109,13 +109,8 @@ def test_noalloc_rejects_oversized_scratch():
     is enqueued; a valid call afterwards still works."""
     wl = W_WIDE_RANK   # 32 tokens x rank 1024 of tagged u words alone fill the array
     gl, _ = H.build_layers(pi, wl, 1, keep_host=False)
-    G = torch.cuda.get_device_properties(0).multi_processor_count
     B = pi.PI_MAX_BATCH
-    W = -(-(-(-wl.d_ff // G)) // 32)
-
-    def r256(v):
-        return -(-v // 256) * 256
-    need = 256 + r256(B * wl.rank * 8) + r256(B * G * W * 8)
+    need = 256 + -(-(B * wl.rank * 8) // 256) * 256
     assert need > pi.PI_NOALLOC_SCRATCH_BYTES
     x = S.make_inputs(wl, B, "cuda", stream_id=70)
     mask = torch.full((B, wl.d_ff // 32), 7, dtype=torch.int32, device="cuda")
