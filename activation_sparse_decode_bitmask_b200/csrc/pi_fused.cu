@@ -205,6 +205,13 @@ __device__ __forceinline__ void ring_wait_item(uint32_t item, Smem& sm, const Fu
     }
   }
 }
+// Warp-collective wait for ring item `item`: lane 0 waits on the barrier (acquire) and
+// __syncwarp passes the visibility of the landed bytes on to the other lanes, so the
+// mbarrier sees one waiter per warp instead of 32.
+__device__ __forceinline__ void ring_wait_item_warp(uint32_t item, Smem& sm, const FusedParams& p) {
+  if ((threadIdx.x & 31) == 0) ring_wait_item(item, sm, p);
+  __syncwarp();
+}
 // Has ring item `item` landed?  (Non-blocking; valid for items fewer than kItems ahead
 // of the oldest item not yet released.)
 __device__ __forceinline__ bool ring_item_ready(uint32_t item, Smem& sm) {
@@ -239,10 +246,50 @@ __device__ __forceinline__ uint32_t tag_of(uint32_t epoch, int l, int e) {
   return epoch * 1024u + (uint32_t)l * 8u + (uint32_t)e;
 }
 
+// The gate/up dot products of an F window of N records (ring positions pos) over this
+// thread's units, reduced across the warp: returns this lane's share of the reduce-scatter
+// of the window's N * NB * NV values and sets lg = log2 of their padded count.
+__host__ __device__ constexpr int pow2_ceil(int v) { return v <= 1 ? 1 : 2 * pow2_ceil((v + 1) / 2); }
+__host__ __device__ constexpr int log2_exact(int v) { return v <= 1 ? 0 : 1 + log2_exact(v / 2); }
+
+template <int FAM, int ACT, int NB, int NU, int N, int KW>
+__device__ __forceinline__ float window_dots(uint32_t base, const uint32_t (&pos)[KW], const FusedParams& p,
+                                             int t, int nunits, const uint32_t (&xr)[NU][NB][Fam<FAM>::XW], int lane,
+                                             int& lg) {
+  constexpr int NV = (ACT == PI_REGLU) ? 2 : 1;
+  constexpr int V = pow2_ceil(N * NB * NV);
+  float v[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) v[i] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < N; ++kk) {
+    const uint32_t rec = base + pos[kk];
+    float au[NB], ag[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) au[b] = ag[b] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NU; ++j) {
+      const int q = t + kConsumerThreads * j;
+      if (q < nunits) {
+        unit_dot<FAM, NB>(rec + (uint32_t)p.up_off, p.d, q, xr[j], au);
+        if constexpr (ACT == PI_REGLU) unit_dot<FAM, NB>(rec + (uint32_t)p.gate_off, p.d, q, xr[j], ag);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      v[(kk * NB + b) * NV] = au[b];
+      if constexpr (ACT == PI_REGLU) v[(kk * NB + b) * NV + 1] = ag[b];
+    }
+  }
+  lg = log2_exact(V);
+  return reduce_scatter<V>(v, lane);
+}
+
 // ------------------------------------------------------------------ the kernel
 template <int FAM, int ACT, int NB, int NU>
 __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p) {
   constexpr int UE = Fam<FAM>::UE;
+  constexpr int XW = Fam<FAM>::XW;
   constexpr int PB = Fam<FAM>::PB;
   using XT = typename Fam<FAM>::X;
   extern __shared__ __align__(128) uint8_t dsmem[];
@@ -413,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     int nlist = 0;
     stamp(p, l, 0);
     // this layer's x units, fp32, in registers for P-a and F
-    float xr[NU][NB][UE];
+    uint32_t xr[NU][NB][XW];
 #pragma unroll
     for (int j = 0; j < NU; ++j) {
       const int q = t + kConsumerThreads * j;
@@ -423,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
 #pragma unroll
         for (int b = 0; b < NB; ++b)
 #pragma unroll
-          for (int e = 0; e < UE; ++e) xr[j][b][e] = 0.f;
+          for (int e = 0; e < XW; ++e) xr[j][b][e] = 0u;
       }
     }
     if (t == 0) mbar_arrive(&sm.layer_start);
@@ -436,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       for (int k = k0; k < k1; k += p.p1_rows_per_item) {
         const int n = min(p.p1_rows_per_item, k1 - k);
         const uint8_t* item = ring_next(ring, (uint32_t)n * p.p1_row);
-        ring_wait_item(ring.item, sm, p);
+        ring_wait_item_warp(ring.item, sm, p);
         if (k == k0) stamp(p, l, 13);
         for (int i0 = 0; i0 < n; i0 += RP) {
           float v[16];
@@ -445,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
 #pragma unroll
           for (int i = 0; i < RP; ++i) {
             if (i0 + i < n) {
-              const uint8_t* row = item + (size_t)(i0 + i) * p.p1_row;
+              const uint32_t row = smem_u32(item) + (uint32_t)((i0 + i) * p.p1_row);
               float acc[NB];
 #pragma unroll
               for (int b = 0; b < NB; ++b) acc[b] = 0.f;
@@ -456,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
               for (int b = 0; b < NB; ++b) v[i * NB + b] = acc[b];
             }
           }
-          const float sw = reduce_scatter16(v, lane);
+          const float sw = reduce_scatter<16>(v, lane);
           float* red = &sm.red[redbuf][0][0];
           redbuf ^= 1;
           if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = sw;
@@ -497,13 +544,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         const int n = min(p.p2_rows_per_item, nown - m0);
         const uint8_t* item = ring_next(ring, (uint32_t)n * p.p2_stride);
         const long long wt0 = diag_clock(p);
-        ring_wait_item(ring.item, sm, p);
+        ring_wait_item_warp(ring.item, sm, p);
         pb_wait += diag_clock(p) - wt0;
         if (m0 == 0) stamp(p, l, 12);
         for (int mb = warp * 8; mb < n; mb += kConsumerWarps * 8) {
-          const uint8_t* rows[8];
+          uint32_t rows[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) rows[i] = item + (size_t)min(mb + i, n - 1) * p.p2_stride;   // past n: repeats, unused
+          for (int i = 0; i < 8; ++i) rows[i] = smem_u32(item) + (uint32_t)(min(mb + i, n - 1) * p.p2_stride);   // past n: repeats, unused
           float acc[8][NB];
 #pragma unroll
           for (int i = 0; i < 8; ++i)
@@ -516,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
               for (int b = 0; b < NB; ++b) uu[b] = *reinterpret_cast<const float4*>(u_s + b * r + 4 * q);
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const float4 w = *reinterpret_cast<const float4*>(rows[i] + 16 * q);
+                const float4 w = u4f(lds128(rows[i] + 16u * q));
 #pragma unroll
                 for (int b = 0; b < NB; ++b)
                   acc[i][b] = fmaf(w.w, uu[b].w, fmaf(w.z, uu[b].z, fmaf(w.y, uu[b].y, fmaf(w.x, uu[b].x, acc[i][b]))));
@@ -530,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
               }
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const uint4 w = *reinterpret_cast<const uint4*>(rows[i] + 16 * q);
+                const uint4 w = lds128(rows[i] + 16u * q);
                 const float2 a = h2f2(w.x), bb = h2f2(w.y), cc = h2f2(w.z), e = h2f2(w.w);
 #pragma unroll
                 for (int b = 0; b < NB; ++b) {
@@ -547,7 +594,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           reduce_scatter8<NB>(acc, lane, dot);
           const int m = mb + ((lane >> 2) & 7);
           if ((lane & 3) == 0 && m < n) {
-            const float ti = *reinterpret_cast<const float*>(rows[(lane >> 2) & 7] + (size_t)r * PB);
+            uint32_t trow = rows[0];
+#pragma unroll
+            for (int i = 1; i < 8; ++i) if (i == ((lane >> 2) & 7)) trow = rows[i];
+            const float ti = lds_f32(trow + (uint32_t)(r * PB));
             const int i = c + (m0 + m) * G;
             uint32_t bits = 0;
 #pragma unroll
@@ -687,39 +737,23 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       }
       nwin += (nb > 0);
       uint32_t pos[KW];
-      float v[16];
-#pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2) v[s2] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < KW; ++kk) {
         pos[kk] = 0;
-        if (kk < nb) {
-          pos[kk] = ring_place(ring.head, (uint32_t)p.rec_stride, ring.cap);
-          ring_wait_item(item_e + kk, sm, p);   // landed already: makes the data visible here
-          const uint8_t* rec = ring.base + pos[kk];
-          float au[NB], ag[NB];
-#pragma unroll
-          for (int b = 0; b < NB; ++b) au[b] = ag[b] = 0.f;
-#pragma unroll
-          for (int j = 0; j < NU; ++j) {
-            const int q = t + kConsumerThreads * j;
-            if (q < nunits) {
-              unit_dot<FAM, NB>(rec + p.up_off, d, q, xr[j], au);
-              if constexpr (ACT == PI_REGLU) unit_dot<FAM, NB>(rec + p.gate_off, d, q, xr[j], ag);
-            }
-          }
-#pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            v[(kk * NB + b) * NV] = au[b];
-            if constexpr (ACT == PI_REGLU) v[(kk * NB + b) * NV + 1] = ag[b];
-          }
-        }
+        // thread 0 saw these records land (acquire) before the barrier that precedes this
+        if (kk < nb) pos[kk] = ring_place(ring.head, (uint32_t)p.rec_stride, ring.cap);
       }
       float* red = &sm.red[redbuf][0][0];
       if (nb > 0) {
-        const float sw = reduce_scatter16(v, lane);
+        float sw = 0.f;
+        int lg = 0;   // log2 of the number of reduced values
+        switch (nb) {
+#define PI_WIN(N) case N: if constexpr (N <= KW) sw = window_dots<FAM, ACT, NB, NU, N>(smem_u32(ring.base), pos, p, t, nunits, xr, lane, lg); break;
+          PI_WIN(1) PI_WIN(2) PI_WIN(3) PI_WIN(4) PI_WIN(5) PI_WIN(6) PI_WIN(7) PI_WIN(8)
+#undef PI_WIN
+        }
         redbuf ^= 1;
-        if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = sw;
+        if ((lane & ((32 >> lg) - 1)) == 0) red[warp * 16 + (lane >> (5 - lg))] = sw;
       }
       const int dw = (nwin == 2 || nwin == 3) ? 22 + 3 * (nwin - 2) : -1;   // diagnostics: windows 1, 2
       if (dw >= 0) stamp(p, l, dw);
@@ -738,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         uint32_t mypos = pos[0];
 #pragma unroll
         for (int k2 = 1; k2 < KW; ++k2) if (k2 == kk) mypos = pos[k2];
-        const float bi = *reinterpret_cast<const float*>(ring.base + mypos + p.bias_off);
+        const float bi = lds_f32(smem_u32(ring.base) + mypos + (uint32_t)p.bias_off);
         float a;
         if constexpr (ACT == PI_REGLU) a = fmaxf(sg + bi, 0.f) * su;
         else a = fmaxf(su + bi, 0.f);
@@ -751,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           float h[NB];
 #pragma unroll
           for (int b = 0; b < NB; ++b) h[b] = sm.hbuf[wb ^ 1][kk][b];
-          const uint8_t* drow = ring.base + pos_prev[kk] + p.down_off;
+          const uint32_t drow = smem_u32(ring.base) + pos_prev[kk] + (uint32_t)p.down_off;
 #pragma unroll
           for (int j = 0; j < NU; ++j)
             if (t + kConsumerThreads * j < nunits) unit_axpy<FAM, NB>(drow, d, t + kConsumerThreads * j, h, y[j]);
@@ -1002,10 +1036,15 @@ __global__ void __launch_bounds__(kThreads, 1) barrier_probe_kernel(const FusedP
 
 constexpr int ue_of(int fam) { return fam == FAM_F32 ? 4 : fam == FAM_F16 ? 8 : 16; }
 
-// Largest unit count per consumer thread that each (family, tokens) pair is built for;
-// a launch takes the smallest count that covers d, so x and y in registers stay small.
+// Largest d_model each (family, tokens) pair serves, and the unit count per consumer
+// thread that covers it; a launch takes the smallest count that covers its d, so x and y
+// in registers stay small.
+constexpr int d_max_of(int fam, int nb) {
+  return fam == FAM_F32 ? (nb == 4 ? 2048 : 4096)
+                        : fam == FAM_F16 ? (nb == 1 ? 12288 : nb == 2 ? 8192 : 4096) : (nb <= 2 ? 8192 : 0);
+}
 constexpr int nu_max(int fam, int nb) {
-  return fam == FAM_F32 ? (nb == 4 ? 1 : 2) : fam == FAM_F16 ? (nb == 1 ? 3 : nb == 2 ? 2 : 1) : (nb <= 2 ? 1 : 0);
+  return (d_max_of(fam, nb) / ue_of(fam) + kConsumerThreads - 1) / kConsumerThreads;
 }
 
 int nb_of(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 0; }
@@ -1031,6 +1070,10 @@ cudaError_t launch_nu(const FusedParams& p, size_t smem, cudaStream_t stream) {
   if constexpr (M >= 1) if (nu <= 1) return launch_t<FAM, ACT, NB, 1>(p, smem, stream);
   if constexpr (M >= 2) if (nu == 2) return launch_t<FAM, ACT, NB, 2>(p, smem, stream);
   if constexpr (M >= 3) if (nu == 3) return launch_t<FAM, ACT, NB, 3>(p, smem, stream);
+  if constexpr (M >= 4) if (nu == 4) return launch_t<FAM, ACT, NB, 4>(p, smem, stream);
+  if constexpr (M >= 5) if (nu == 5) return launch_t<FAM, ACT, NB, 5>(p, smem, stream);
+  if constexpr (M >= 6) if (nu == 6) return launch_t<FAM, ACT, NB, 6>(p, smem, stream);
+  static_assert(M <= 6, "unit counts above 6 are not instantiated");
   return cudaErrorNotSupported;
 }
 
@@ -1051,9 +1094,7 @@ cudaError_t launch_nb(int B, const FusedParams& p, size_t smem, cudaStream_t str
 bool fused_supported(int family, int B, int d) {
   const int nb = nb_of(B);
   if (nb == 0) return false;
-  const int nu = nu_max(family, nb);
-  if (nu == 0) return false;
-  return d <= nu * ue_of(family) * kConsumerThreads;
+  return d <= d_max_of(family, nb);
 }
 
 size_t fused_fixed_smem(int B, int d, int r, int grid, int nown_max, int family) {

@@ -21,9 +21,12 @@
 namespace pi {
 
 template <int FAM> struct Fam;
-template <> struct Fam<FAM_F32> { static constexpr int UE = 4;  static constexpr int PB = 4; using X = float; };
-template <> struct Fam<FAM_F16> { static constexpr int UE = 8;  static constexpr int PB = 2; using X = __half; };
-template <> struct Fam<FAM_Q4>  { static constexpr int UE = 16; static constexpr int PB = 2; using X = __half; };
+// UE: elements per unit; PB: bytes per predictor element; XW: 32-bit registers that hold
+// one token's unit of x (fp32 values, or fp16 pairs for the fp16 family, whose dots use
+// fp16 x fp16 products accumulated in fp32)
+template <> struct Fam<FAM_F32> { static constexpr int UE = 4;  static constexpr int PB = 4; static constexpr int XW = 4;  using X = float; };
+template <> struct Fam<FAM_F16> { static constexpr int UE = 8;  static constexpr int PB = 2; static constexpr int XW = 4;  using X = __half; };
+template <> struct Fam<FAM_Q4>  { static constexpr int UE = 16; static constexpr int PB = 2; static constexpr int XW = 16; using X = __half; };
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -42,48 +45,86 @@ __device__ __forceinline__ void widen8(const uint4 v, float* o) {
   o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y; o[4] = c.x; o[5] = c.y; o[6] = e.x; o[7] = e.y;
 }
 
-// Unit q of every token's x (xs: [NB][d] in the family's x type), widened to fp32.
+// Loads from shared memory by 32-bit shared-window address (the ring holds every row)
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds_h2f(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return __half2float(__ushort_as_half(v));
+}
+__device__ __forceinline__ float4 u4f(uint4 v) {
+  return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
+}
+
+// acc + lo(w) * lo(x) and acc2 + hi(w) * hi(x): fp16 x fp16 products (exact in fp32)
+// added in fp32 with one rounding each
+__device__ __forceinline__ void fma2_h(uint32_t w2, uint32_t x2, float& acc, float& acc2) {
+  asm("{\n .reg .f16 wl, wh, xl, xh;\n mov.b32 {wl, wh}, %2;\n mov.b32 {xl, xh}, %3;\n"
+      " fma.rn.f32.f16 %0, wl, xl, %0;\n fma.rn.f32.f16 %1, wh, xh, %1;\n}"
+      : "+f"(acc), "+f"(acc2)
+      : "r"(w2), "r"(x2));
+}
+
+// Unit q of every token's x (xs: [NB][d] in the family's x type) in registers.
 template <int FAM, int NB>
-__device__ __forceinline__ void load_x_unit(const void* xs, int d, int q, float (&xu)[NB][Fam<FAM>::UE]) {
+__device__ __forceinline__ void load_x_unit(const void* xs, int d, int q, uint32_t (&xu)[NB][Fam<FAM>::XW]) {
   constexpr int UE = Fam<FAM>::UE;
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
     if constexpr (FAM == FAM_F32) {
-      const float4 v = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(xs) + (size_t)b * d)[q];
+      const uint4 v = reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(xs) + (size_t)b * d)[q];
+      xu[b][0] = v.x; xu[b][1] = v.y; xu[b][2] = v.z; xu[b][3] = v.w;
+    } else if constexpr (FAM == FAM_F16) {
+      const uint4 v = reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(xs) + (size_t)b * d)[q];
       xu[b][0] = v.x; xu[b][1] = v.y; xu[b][2] = v.z; xu[b][3] = v.w;
     } else {
       const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(xs) + (size_t)b * d + UE * q);
 #pragma unroll
-      for (int c = 0; c < UE / 8; ++c) widen8(src[c], &xu[b][8 * c]);
+      for (int c = 0; c < UE / 8; ++c) {
+        float w[8];
+        widen8(src[c], w);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xu[b][8 * c + e] = __float_as_uint(w[e]);
+      }
     }
   }
 }
 
 // acc[b] += (unit q of a weight row) . xu[b]
 template <int FAM, int NB>
-__device__ __forceinline__ void unit_dot(const uint8_t* row, int d, int q, const float (&xu)[NB][Fam<FAM>::UE],
+__device__ __forceinline__ void unit_dot(uint32_t row, int d, int q, const uint32_t (&xu)[NB][Fam<FAM>::XW],
                                          float (&acc)[NB]) {
   if constexpr (FAM == FAM_F32) {
-    const float4 w = reinterpret_cast<const float4*>(row)[q];
+    const float4 w = u4f(lds128(row + 16u * q));
 #pragma unroll
     for (int b = 0; b < NB; ++b)
-      acc[b] = fmaf(w.w, xu[b][3], fmaf(w.z, xu[b][2], fmaf(w.y, xu[b][1], fmaf(w.x, xu[b][0], acc[b]))));
+      acc[b] = fmaf(w.w, __uint_as_float(xu[b][3]),
+                    fmaf(w.z, __uint_as_float(xu[b][2]),
+                         fmaf(w.y, __uint_as_float(xu[b][1]), fmaf(w.x, __uint_as_float(xu[b][0]), acc[b]))));
   } else if constexpr (FAM == FAM_F16) {
-    float w[8];
-    widen8(reinterpret_cast<const uint4*>(row)[q], w);
+    const uint4 w = lds128(row + 16u * q);
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      float s = acc[b], s2 = w[4] * xu[b][4];
-      s = fmaf(w[0], xu[b][0], s); s2 = fmaf(w[5], xu[b][5], s2);
-      s = fmaf(w[1], xu[b][1], s); s2 = fmaf(w[6], xu[b][6], s2);
-      s = fmaf(w[2], xu[b][2], s); s2 = fmaf(w[7], xu[b][7], s2);
-      s = fmaf(w[3], xu[b][3], s);
+      float s = acc[b], s2 = 0.f;
+      fma2_h(w.x, xu[b][0], s, s2);
+      fma2_h(w.y, xu[b][1], s, s2);
+      fma2_h(w.z, xu[b][2], s, s2);
+      fma2_h(w.w, xu[b][3], s, s2);
       acc[b] = s + s2;
     }
   } else {
     const int blk = q >> 1;
-    const uint4 nb = reinterpret_cast<const uint4*>(row)[blk];
-    const float sc = __half2float(reinterpret_cast<const __half*>(row + (d >> 1))[blk]);
+    const uint4 nb = lds128(row + 16u * blk);
+    const float sc = lds_h2f(row + (uint32_t)(d >> 1) + 2u * blk);
     const int sh = (q & 1) * 4;
     const uint32_t wv[4] = {(nb.x >> sh) & 0x0F0F0F0Fu, (nb.y >> sh) & 0x0F0F0F0Fu, (nb.z >> sh) & 0x0F0F0F0Fu,
                             (nb.w >> sh) & 0x0F0F0F0Fu};
@@ -92,10 +133,10 @@ __device__ __forceinline__ void unit_dot(const uint8_t* row, int d, int q, const
       float s = 0.f, s2 = 0.f;
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        s = fmaf(q4_val(wv[m], 0), xu[b][4 * m], s);
-        s2 = fmaf(q4_val(wv[m], 1), xu[b][4 * m + 1], s2);
-        s = fmaf(q4_val(wv[m], 2), xu[b][4 * m + 2], s);
-        s2 = fmaf(q4_val(wv[m], 3), xu[b][4 * m + 3], s2);
+        s = fmaf(q4_val(wv[m], 0), __uint_as_float(xu[b][4 * m]), s);
+        s2 = fmaf(q4_val(wv[m], 1), __uint_as_float(xu[b][4 * m + 1]), s2);
+        s = fmaf(q4_val(wv[m], 2), __uint_as_float(xu[b][4 * m + 2]), s);
+        s2 = fmaf(q4_val(wv[m], 3), __uint_as_float(xu[b][4 * m + 3]), s2);
       }
       acc[b] = fmaf(sc, s + s2, acc[b]);
     }
@@ -105,24 +146,24 @@ __device__ __forceinline__ void unit_dot(const uint8_t* row, int d, int q, const
 // acc[b] += (unit q of a predictor row in the p dtype: fp32 for the fp32 family, else
 // fp16) . xu[b]
 template <int FAM, int NB>
-__device__ __forceinline__ void unit_dot_p(const uint8_t* row, int q, const float (&xu)[NB][Fam<FAM>::UE],
+__device__ __forceinline__ void unit_dot_p(uint32_t row, int q, const uint32_t (&xu)[NB][Fam<FAM>::XW],
                                            float (&acc)[NB]) {
   constexpr int UE = Fam<FAM>::UE;
-  if constexpr (FAM == FAM_F32) {
-    unit_dot<FAM_F32, NB>(row, 0, q, xu, acc);
+  if constexpr (FAM == FAM_F32 || FAM == FAM_F16) {
+    unit_dot<FAM, NB>(row, 0, q, xu, acc);
   } else {
-    const uint4* src = reinterpret_cast<const uint4*>(row + (size_t)q * UE * 2);
+    const uint32_t src = row + (uint32_t)q * UE * 2;
 #pragma unroll
     for (int c = 0; c < UE / 8; ++c) {
       float w[8];
-      widen8(src[c], w);
+      widen8(lds128(src + 16u * c), w);
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
-        float s = acc[b], s2 = w[4] * xu[b][8 * c + 4];
-        s = fmaf(w[0], xu[b][8 * c + 0], s); s2 = fmaf(w[5], xu[b][8 * c + 5], s2);
-        s = fmaf(w[1], xu[b][8 * c + 1], s); s2 = fmaf(w[6], xu[b][8 * c + 6], s2);
-        s = fmaf(w[2], xu[b][8 * c + 2], s); s2 = fmaf(w[7], xu[b][8 * c + 7], s2);
-        s = fmaf(w[3], xu[b][8 * c + 3], s);
+        float s = acc[b], s2 = w[4] * __uint_as_float(xu[b][8 * c + 4]);
+        s = fmaf(w[0], __uint_as_float(xu[b][8 * c + 0]), s); s2 = fmaf(w[5], __uint_as_float(xu[b][8 * c + 5]), s2);
+        s = fmaf(w[1], __uint_as_float(xu[b][8 * c + 1]), s); s2 = fmaf(w[6], __uint_as_float(xu[b][8 * c + 6]), s2);
+        s = fmaf(w[2], __uint_as_float(xu[b][8 * c + 2]), s); s2 = fmaf(w[7], __uint_as_float(xu[b][8 * c + 7]), s2);
+        s = fmaf(w[3], __uint_as_float(xu[b][8 * c + 3]), s);
         acc[b] = s + s2;
       }
     }
@@ -131,10 +172,10 @@ __device__ __forceinline__ void unit_dot_p(const uint8_t* row, int q, const floa
 
 // yu[b] += h[b] * (unit q of a weight row)
 template <int FAM, int NB>
-__device__ __forceinline__ void unit_axpy(const uint8_t* row, int d, int q, const float (&h)[NB],
+__device__ __forceinline__ void unit_axpy(uint32_t row, int d, int q, const float (&h)[NB],
                                           float (&yu)[NB][Fam<FAM>::UE]) {
   if constexpr (FAM == FAM_F32) {
-    const float4 w = reinterpret_cast<const float4*>(row)[q];
+    const float4 w = u4f(lds128(row + 16u * q));
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       yu[b][0] = fmaf(h[b], w.x, yu[b][0]); yu[b][1] = fmaf(h[b], w.y, yu[b][1]);
@@ -142,15 +183,15 @@ __device__ __forceinline__ void unit_axpy(const uint8_t* row, int d, int q, cons
     }
   } else if constexpr (FAM == FAM_F16) {
     float w[8];
-    widen8(reinterpret_cast<const uint4*>(row)[q], w);
+    widen8(lds128(row + 16u * q), w);
 #pragma unroll
     for (int b = 0; b < NB; ++b)
 #pragma unroll
       for (int e = 0; e < 8; ++e) yu[b][e] = fmaf(h[b], w[e], yu[b][e]);
   } else {
     const int blk = q >> 1;
-    const uint4 nb = reinterpret_cast<const uint4*>(row)[blk];
-    const float sc = __half2float(reinterpret_cast<const __half*>(row + (d >> 1))[blk]);
+    const uint4 nb = lds128(row + 16u * blk);
+    const float sc = lds_h2f(row + (uint32_t)(d >> 1) + 2u * blk);
     const int sh = (q & 1) * 4;
     const uint32_t wv[4] = {(nb.x >> sh) & 0x0F0F0F0Fu, (nb.y >> sh) & 0x0F0F0F0Fu, (nb.z >> sh) & 0x0F0F0F0Fu,
                             (nb.w >> sh) & 0x0F0F0F0Fu};
@@ -168,38 +209,27 @@ __device__ __forceinline__ void unit_axpy(const uint8_t* row, int d, int q, cons
   }
 }
 
-// Butterfly reduce-scatter of 16 per-lane values across the warp: on return every lane
-// holds the warp's sum of value (lane >> 1).  The pairing of the additions is the same
-// for every value, so a value's sum does not depend on its slot.
-__device__ __forceinline__ float reduce_scatter16(float (&v)[16], int lane) {
+// Butterfly reduce-scatter of V (a power of two, <= 16) per-lane values across the
+// warp: on return every lane holds the warp's sum of value lane >> (5 - log2 V).  The
+// lanes are paired at offsets 16, 8, 4, 2, 1 in that order for every V and every value,
+// so a value's sum does not depend on V or on its slot.
+template <int V>
+__device__ __forceinline__ float reduce_scatter(float (&v)[V], int lane) {
+  static_assert(V >= 1 && V <= 16 && (V & (V - 1)) == 0, "V must be a power of two <= 16");
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const bool up = lane & 16;
-    const float send = up ? v[i] : v[i + 8];
-    const float keep = up ? v[i + 8] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-  }
+  for (int o = 16, n = V / 2; n >= 1; o >>= 1, n >>= 1) {
+    const bool up = lane & o;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const bool up = lane & 8;
-    const float send = up ? v[i] : v[i + 4];
-    const float keep = up ? v[i + 4] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    for (int i = 0; i < n; ++i) {
+      const float send = up ? v[i] : v[i + n];
+      const float keep = up ? v[i + n] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
   }
+  float s = v[0];
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const bool up = lane & 4;
-    const float send = up ? v[i] : v[i + 2];
-    const float keep = up ? v[i + 2] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-  }
-  {
-    const bool up = lane & 2;
-    const float send = up ? v[0] : v[1];
-    const float keep = up ? v[1] : v[0];
-    v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-  }
-  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+  for (int o = 16 / V; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
 }
 
 }  // namespace pi
