@@ -163,6 +163,12 @@ def dist_max(v: float, world: int) -> float:
     return float(t.item())
 
 
+def whole_job_rate(world: int, steps: int, batch: int, ms_max: float) -> float:
+    """Tokens per second of the whole job: every rank decodes `steps` steps of `batch`
+    tokens on its own replica; the time is the slowest rank's."""
+    return world * steps * batch / (ms_max / 1e3)
+
+
 def dist_barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -260,7 +266,7 @@ def run_ours(args, world, rank, local):
     ms_local = e0.elapsed_time(e1)
     ms = dist_max(ms_local, world)
     ms_step = ms / K
-    value = world * K * B / (ms / 1e3)
+    value = whole_job_rate(world, K, B, ms)
     active_per_step = (act1 - act0) / K                     # summed over layers
     algo_bytes = wl.n_layers * predictor_bytes(wl) + active_per_step * bytes_per_neuron(wl)
     achieved = algo_bytes / (ms_local / K / 1e3) / 1e9
