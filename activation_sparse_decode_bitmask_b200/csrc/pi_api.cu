@@ -144,6 +144,52 @@ int hot_len(const pi_layer* L, int B) {
   return n;
 }
 
+BatchedLayer bview(const pi_layer* L) {
+  BatchedLayer b;
+  b.d = L->desc.d_model; b.f = L->desc.d_ff; b.r = L->desc.rank; b.G = L->G; b.nown_max = L->nown_max;
+  b.rec = L->rec; b.rec_stride = L->rec_stride; b.up_off = L->up_off; b.gate_off = L->gate_off; b.down_off = L->down_off;
+  b.p1t = L->p1t; b.p1_row = L->p1_row; b.p2o = L->p2o; b.p2_stride = L->p2_stride;
+  b.thresh = L->thresh; b.bias = L->bias;
+  return b;
+}
+// Calls the fused kernel does not serve take the batched path: more than 4 tokens, or
+// 2 to 4 tokens with a d_model beyond the fused kernel's registers for that many tokens.
+bool use_batched(const pi_layer* L, int B) {
+  if (B > 4) return true;
+  return !fused_supported(L->family, B, L->desc.d_model) &&
+         batched_supported(L->family, B, L->desc.d_model, L->desc.rank);
+}
+
+// pi_decode_stack for more than 4 tokens: per layer, the predictor (mask words), the
+// compaction of the union, the gate/up rows and the down columns of the active neurons,
+// and the stack glue, as consecutive launches on the stream.
+pi_status decode_stack_batched(pi_layer* const* layers, int Lc, void* x_inout, int B, const pi_trace* trace,
+                               pi_workspace* ws, cudaStream_t stream) {
+  const pi_layer* L0 = layers[0];
+  const int d = L0->desc.d_model, f = L0->desc.d_ff, words = f / 32;
+  if (!batched_supported(L0->family, B, d, L0->desc.rank) || !ws->u_hi) return PI_ERR_UNSUPPORTED;
+  if (trace && (trace->idx || trace->count) && !(trace->idx && trace->count && trace->mask)) return PI_ERR_ARG;
+  PI_TRY(cudaMemsetAsync(ws->layer_count, 0, (size_t)Lc * 4, stream));
+  if (trace && trace->x)
+    PI_TRY(cudaMemcpyAsync(trace->x, x_inout, (size_t)B * d * 2, cudaMemcpyDeviceToDevice, stream));
+  for (int l = 0; l < Lc; ++l) {
+    const BatchedLayer bl = bview(layers[l]);
+    uint32_t* mask = (trace && trace->mask) ? trace->mask + (size_t)l * B * words : ws->bmask;
+    int32_t* idx = (trace && trace->idx) ? trace->idx + (size_t)l * f : ws->bidx;
+    int32_t* count = (trace && trace->count) ? trace->count + l : ws->bcount;
+    float* logits = (trace && trace->logits) ? trace->logits + (size_t)l * B * f : nullptr;
+    float* y = (trace && trace->y) ? trace->y + (size_t)l * B * d : ws->by;
+    void* tx = (trace && trace->x) ? static_cast<uint8_t*>(trace->x) + (size_t)(l + 1) * B * d * 2 : nullptr;
+    PI_TRY(cudaMemsetAsync(mask, 0, (size_t)B * words * 4, stream));
+    PI_TRY(batched_predict(bl, x_inout, B, mask, logits, ws->u_hi, ws->u_lo, stream));
+    PI_TRY(launch_compact(mask, B, f, idx, count, stream));
+    PI_TRY(batched_count(count, ws->active_total, ws->layer_count + l, stream));
+    PI_TRY(batched_ffn(bl, x_inout, B, mask, idx, count, ws->bh, y, ws->err, stream));
+    PI_TRY(batched_glue(x_inout, y, B, d, x_inout, tx, stream));
+  }
+  return PI_OK;
+}
+
 LayerDev dev_view(const pi_layer* L, int B = 0) { return LayerDev{L->rec, L->p1t, L->p2o, B > 0 ? hot_len(L, B) : 0, 0}; }
 
 bool same_desc(const pi_layer_desc& a, const pi_layer_desc& b) {
@@ -347,6 +393,12 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
             dmalloc(&ws->active_total, 16) == cudaSuccess &&
             dmalloc(&ws->layer_count, (size_t)L_max * 4) == cudaSuccess &&
             dmalloc(&ws->x_dev, Bm * d_max * 4) == cudaSuccess;
+  if (ok && B_max > 1) {   // batched path buffers (more than one token)
+    ok = dmalloc(&ws->u_hi, (size_t)32 * r_max * 2) == cudaSuccess && dmalloc(&ws->u_lo, (size_t)32 * r_max * 2) == cudaSuccess &&
+         dmalloc(&ws->bmask, (size_t)32 * (f_max / 32) * 4) == cudaSuccess && dmalloc(&ws->bidx, (size_t)f_max * 4) == cudaSuccess &&
+         dmalloc(&ws->bcount, 16) == cudaSuccess && dmalloc(&ws->bh, (size_t)f_max * 32 * 4) == cudaSuccess &&
+         dmalloc(&ws->by, (size_t)32 * d_max * 4) == cudaSuccess;
+  }
   if (ok) {
     // tagged words start with tag 0; launch epochs start at 1, so no stale word matches
     const uint32_t bar0[4] = {0u, 0u, 1u, 0u};
@@ -371,6 +423,8 @@ void pi_workspace_free(pi_workspace* ws) {
   cudaFree(ws->ux); cudaFree(ws->px); cudaFree(ws->vx); cudaFree(ws->sx);
   cudaFree(ws->bar); cudaFree(ws->err); cudaFree(ws->active_total);
   cudaFree(ws->layer_count); cudaFree(ws->x_dev); cudaFree(ws->phase_clk);
+  cudaFree(ws->u_hi); cudaFree(ws->u_lo); cudaFree(ws->bmask); cudaFree(ws->bidx); cudaFree(ws->bcount);
+  cudaFree(ws->bh); cudaFree(ws->by);
   delete ws;
 }
 
@@ -409,6 +463,12 @@ pi_status pi_predict(const pi_layer* L, const void* x, int B, uint32_t* mask, fl
   if (!L || !x || !mask || B < 1 || B > PI_MAX_BATCH) return PI_ERR_ARG;
   pi_status st = check_ws(ws, L->desc, B, 1);
   if (st != PI_OK) return st;
+  if (use_batched(L, B)) {
+    if (!batched_supported(L->family, B, L->desc.d_model, L->desc.rank) || !ws->u_hi) return PI_ERR_UNSUPPORTED;
+    PI_TRY(cudaMemsetAsync(mask, 0, (size_t)B * (L->desc.d_ff / 32) * 4, stream));
+    PI_TRY(batched_predict(bview(L), x, B, mask, logits, ws->u_hi, ws->u_lo, stream));
+    return PI_OK;
+  }
   FusedParams p;
   size_t smem = 0;
   st = plan_fused(L, B, ws, p, smem);
@@ -435,6 +495,11 @@ pi_status pi_sparse_ffn(const pi_layer* L, const void* x, int B, const uint32_t*
   if (!L || !x || !mask || !idx || !count || !y || B < 1 || B > PI_MAX_BATCH) return PI_ERR_ARG;
   pi_status st = check_ws(ws, L->desc, B, 1);
   if (st != PI_OK) return st;
+  if (use_batched(L, B)) {
+    if (!batched_supported(L->family, B, L->desc.d_model, L->desc.rank) || !ws->u_hi) return PI_ERR_UNSUPPORTED;
+    PI_TRY(batched_ffn(bview(L), x, B, mask, idx, count, ws->bh, y, ws->err, stream));
+    return PI_OK;
+  }
   FusedParams p;
   size_t smem = 0;
   st = plan_fused(L, B, ws, p, smem);
@@ -462,6 +527,7 @@ pi_status pi_decode_stack(pi_layer* const* layers, int Lc, void* x_inout, int B,
   const pi_layer* L0 = layers[0];
   pi_status st = check_ws(ws, L0->desc, B, Lc);
   if (st != PI_OK) return st;
+  if (use_batched(L0, B)) return decode_stack_batched(layers, Lc, x_inout, B, trace, ws, stream);
   FusedParams p;
   size_t smem = 0;
   st = plan_fused(L0, B, ws, p, smem);

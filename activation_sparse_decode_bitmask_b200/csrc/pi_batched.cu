@@ -1,0 +1,481 @@
+// The batched path: 5 to 32 tokens per call, fp16 family.
+//
+// At these batch sizes every step of a layer is a dense contraction over the rows it
+// touches, so each runs on the tensor cores: tiles of 16 rows x 8 tokens, K in steps of
+// 16 (mma.sync m16n8k16, fp16 operands, fp32 accumulation), operands staged through
+// shared memory with cp.async and read with ldmatrix.
+//   u       = P1^T x           rows: P1^T rows (contiguous)         tokens: x (fp16)
+//   logit   = P2^T u - t       rows: P2 columns (owner-major rows)  tokens: u as fp16 hi + lo
+//   h       = act(W x + b)     rows: gate/up rows of the active neurons (gathered by idx)
+//   y       = sum_i h_i Wd_i   columns of the down rows of the active neurons; h as fp16 hi + lo
+// fp16 x fp16 products are exact in fp32; u and h are fp32 values carried as the sum of
+// two fp16 numbers (hi = fp16(v), lo = fp16(v - hi)), about 22 significant bits, so no
+// step rounds an intermediate to fp16.  The active neurons are processed in the order of
+// idx; the neurons at the front of the stored order are the hot prefix, so the first
+// row tiles of every layer are its dense hot block and the rest are gathered cold rows.
+// Every sum runs in a fixed order: results are bitwise reproducible.
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "pi_internal.h"
+#include "pi_ptx.cuh"
+
+namespace pi {
+
+namespace {
+
+constexpr int kBW = 4;                    // warps per block
+constexpr int kRows = 16 * kBW;           // rows (or columns) per block
+constexpr int kKC = 64;                   // K elements staged per chunk
+constexpr int kPad = kKC * 2 + 16;        // bytes per staged row: the 16-byte pad keeps ldmatrix conflict-free
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t a, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t a, uint32_t (&r)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(a));
+}
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+__device__ __forceinline__ void split_h(float v, __half& hi, __half& lo) {
+  hi = __float2half_rn(v);
+  lo = __float2half_rn(v - __half2float(hi));
+}
+
+// ------------------------------------------------------------------ rows x tokens
+// out[row][token] = sum_k Rows[row][k] * Tok[token][k] for a block of 64 rows and all
+// tokens; Rows are fp16 rows found through the mode's addressing, Tok is [B][K] fp16 (and
+// a second [B][K] fp16 low part when SPLIT).
+enum RowMode { ROWS_P1 = 0, ROWS_P2 = 1, ROWS_FFN = 2 };
+
+struct RowTokArgs {
+  int mode, nrows_static, K, B;
+  const int32_t* count;        // ROWS_FFN: number of active rows (device)
+  const uint8_t* base;         // row storage
+  int stride;                  // bytes between consecutive rows (P1) or per record / P2 row
+  int G, nown_max;             // ROWS_P2: owner-major placement of neuron rows
+  const int32_t* idx;          // ROWS_FFN: stored ids of the active neurons
+  int up_off, gate_off;        // ROWS_FFN: byte offsets of the rows in a record (gate < 0: ReLU)
+  const __half* tok;           // [B][K]
+  const __half* tok_lo;        // [B][K] or null
+  // ROWS_P1 output: u as fp16 hi / lo, [B][r]
+  __half* u_hi;
+  __half* u_lo;
+  // ROWS_P2 output
+  const float* thresh;         // [f]
+  float* logits;               // [B][f] or null
+  uint32_t* mask;              // [B][f/32], zeroed by the caller; bits are OR-ed in
+  int f;
+  // ROWS_FFN output
+  const float* bias;           // [f]
+  const uint32_t* mask_in;     // [B][f/32]
+  float* h;                    // [count][32]
+  int* err;                    // device error word (index or count out of range)
+};
+
+template <int NT, int NMAT, bool SPLIT>
+__global__ void __launch_bounds__(32 * kBW) rowtok_kernel(const RowTokArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int NS = SPLIT ? 2 : 1;
+  constexpr int BP = NT * 8;                       // padded tokens
+  uint8_t* rows_s = smem;                          // [NMAT][kRows][kPad]
+  uint8_t* tok_s = smem + NMAT * kRows * kPad;     // [NS][BP][kPad]
+  int nrows = a.nrows_static;
+  if (a.mode == ROWS_FFN) {
+    const int cnt = *a.count;
+    if (cnt < 0 || cnt > a.nrows_static) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) atomicExch(a.err, DEV_ERR_INDEX);
+      return;
+    }
+    nrows = cnt;
+  }
+  const int row0 = blockIdx.x * kRows;
+  if (row0 >= nrows) return;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  // stored id of active row j, checked against d_ff (a bad id reads neuron 0 and is reported)
+  auto active_id = [&](int j) -> int {
+    int i = __ldg(a.idx + j);
+    if (i < 0 || i >= a.f) {
+      atomicExch(a.err, DEV_ERR_INDEX);
+      i = 0;
+    }
+    return i;
+  };
+
+  // byte address of row j (clamped into range: rows past the end repeat the last one
+  // and their results are never stored), matrix m
+  auto row_ptr = [&](int j, int m) -> const uint8_t* {
+    j = min(j, nrows - 1);
+    if (a.mode == ROWS_P1) return a.base + (size_t)j * a.stride;
+    if (a.mode == ROWS_P2) return a.base + ((size_t)(j % a.G) * a.nown_max + j / a.G) * a.stride;
+    return a.base + (size_t)active_id(j) * a.stride + (m == 0 ? a.up_off : a.gate_off);
+  };
+
+  float c[NMAT][NT][4];
+#pragma unroll
+  for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) c[m][n][e] = 0.f;
+
+  const uint32_t rows_u = smem_u32(rows_s), tok_u = smem_u32(tok_s);
+  for (int k0 = 0; k0 < a.K; k0 += kKC) {
+    // stage the chunk: rows (NMAT x 64 rows x 8 pieces of 16 bytes) and tokens
+    for (int e = t; e < NMAT * kRows * 8; e += 32 * kBW) {
+      const int m = e / (kRows * 8), rr = (e / 8) % kRows, pc = e % 8;
+      cp_async16(rows_u + (uint32_t)((m * kRows + rr) * kPad + pc * 16), row_ptr(row0 + rr, m) + (size_t)k0 * 2 + pc * 16);
+    }
+    for (int e = t; e < NS * BP * 8; e += 32 * kBW) {
+      const int s = e / (BP * 8), b = (e / 8) % BP, pc = e % 8;
+      const __half* src = (s == 0 ? a.tok : a.tok_lo) + (size_t)min(b, a.B - 1) * a.K + k0 + pc * 8;
+      cp_async16(tok_u + (uint32_t)((s * BP + b) * kPad + pc * 16), src);
+    }
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncthreads();
+#pragma unroll
+    for (int ks = 0; ks < kKC / 16; ++ks) {
+      uint32_t af[NMAT][4];
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) {
+        const int r = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int kk = ks * 16 + 8 * (lane >> 4);
+        ldsm_x4(rows_u + (uint32_t)((m * kRows + r) * kPad + kk * 2), af[m]);
+      }
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+#pragma unroll
+        for (int s = 0; s < NS; ++s) {
+          uint32_t bf[2];
+          const int b = n * 8 + (lane & 7);
+          const int kk = ks * 16 + 8 * ((lane >> 3) & 1);
+          ldsm_x2(tok_u + (uint32_t)((s * BP + b) * kPad + kk * 2), bf);
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m) mma16816(c[m][n], af[m], bf);
+        }
+      }
+    }
+    __syncthreads();   // the stage is refilled next chunk
+  }
+
+  // epilogue: thread holds rows g and g + 8 of the warp's tile, tokens 2t and 2t + 1 of
+  // every 8-token tile
+  const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int j = row0 + warp * 16 + g + 8 * half;
+    if (j >= nrows) continue;
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int b = n * 8 + 2 * tq + q;
+        const float v0 = c[0][n][2 * half + q];
+        if (a.mode == ROWS_P1) {
+          if (b < a.B) {
+            __half hi, lo;
+            split_h(v0, hi, lo);
+            a.u_hi[(size_t)b * a.nrows_static + j] = hi;
+            a.u_lo[(size_t)b * a.nrows_static + j] = lo;
+          }
+        } else if (a.mode == ROWS_P2) {
+          if (b < a.B) {
+            const float lg = v0 - __ldg(a.thresh + j);
+            if (a.logits) a.logits[(size_t)b * a.f + j] = lg;
+            if (lg > 0.f) atomicOr(a.mask + (size_t)b * (a.f / 32) + (j >> 5), 1u << (j & 31));
+          }
+        } else {
+          float hv = 0.f;
+          if (b < a.B) {
+            const int i = active_id(j);
+            const uint32_t bit = (__ldg(a.mask_in + (size_t)b * (a.f / 32) + (i >> 5)) >> (i & 31)) & 1u;
+            const float bi = __ldg(a.bias + i);
+            float act;
+            if constexpr (NMAT == 2) act = fmaxf(c[1][n][2 * half + q] + bi, 0.f) * v0;   // gate is matrix 1
+            else act = fmaxf(v0 + bi, 0.f);
+            hv = bit ? act : 0.f;
+          }
+          a.h[(size_t)j * 32 + b] = hv;
+        }
+      }
+  }
+}
+
+// ------------------------------------------------------------------ down projection
+// y[b][c] = sum_j h[j][b] * Wd[idx[j]][c] for a block of 64 columns and all tokens: the
+// columns' slices of the active down rows are staged [neuron][column] and read transposed.
+struct DownArgs {
+  const int32_t* count;
+  int fmax, d, B;
+  const uint8_t* rec;
+  int rec_stride, down_off;
+  const int32_t* idx;
+  const float* h;   // [count][32]
+  float* y;         // [B][d]
+  int* err;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(32 * kBW) down_kernel(const DownArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int BP = NT * 8;
+  uint8_t* w_s = smem;                          // [64 neurons][kPad]: 64 columns of each row
+  uint8_t* h_s = smem + kRows * kPad;           // [2][BP][kPad]: h hi / lo per token, 64 neurons
+  int count = *a.count;
+  if (count < 0 || count > a.fmax) count = 0;   // reported by the gate/up kernel; y becomes 0
+  const int c0 = blockIdx.x * kRows;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  float c[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c[n][e] = 0.f;
+  const uint32_t w_u = smem_u32(w_s), h_u = smem_u32(h_s);
+  for (int j0 = 0; j0 < count; j0 += kRows) {
+    for (int e = t; e < kRows * 8; e += 32 * kBW) {
+      const int jj = e / 8, pc = e % 8;
+      int i = __ldg(a.idx + min(j0 + jj, count - 1));
+      if (i < 0 || i >= a.fmax) i = 0;   // reported by the gate/up kernel
+      cp_async16(w_u + (uint32_t)(jj * kPad + pc * 16),
+                 a.rec + (size_t)i * a.rec_stride + a.down_off + (size_t)c0 * 2 + pc * 16);
+    }
+    cp_async_commit();
+    // h of the chunk, split into fp16 hi / lo; neurons past count contribute zero
+    for (int e = t; e < BP * kRows; e += 32 * kBW) {
+      const int b = e / kRows, jj = e % kRows;
+      const float v = (j0 + jj < count && b < a.B) ? a.h[(size_t)(j0 + jj) * 32 + b] : 0.f;
+      __half hi, lo;
+      split_h(v, hi, lo);
+      reinterpret_cast<__half*>(h_s + (size_t)b * kPad)[jj] = hi;
+      reinterpret_cast<__half*>(h_s + (size_t)(BP + b) * kPad)[jj] = lo;
+    }
+    cp_async_wait_all();
+    __syncthreads();
+#pragma unroll
+    for (int ks = 0; ks < kRows / 16; ++ks) {
+      uint32_t af[4];
+      {
+        const int jj = ks * 16 + (lane & 7) + 8 * (lane >> 4);   // neuron (K) of this lane's row address
+        const int cc = warp * 16 + 8 * ((lane >> 3) & 1);        // column (M) offset
+        ldsm_x4_t(w_u + (uint32_t)(jj * kPad + cc * 2), af);
+      }
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          uint32_t bf[2];
+          const int b = n * 8 + (lane & 7);
+          const int jj = ks * 16 + 8 * ((lane >> 3) & 1);
+          ldsm_x2(h_u + (uint32_t)((s * BP + b) * kPad + jj * 2), bf);
+          mma16816(c[n], af, bf);
+        }
+    }
+    __syncthreads();
+  }
+  const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int col = c0 + warp * 16 + g + 8 * (e >> 1);
+      const int b = n * 8 + 2 * tq + (e & 1);
+      if (b < a.B && col < a.d) a.y[(size_t)b * a.d + col] = c[n][e];
+    }
+}
+
+// ------------------------------------------------------------------ stack glue
+// x' = round_fp16((v - mean v) / sqrt(var v + 1e-6)), v = x + y, one block per token;
+// the sums run in a fixed order.
+__global__ void __launch_bounds__(256) glue_kernel(const __half* x, const float* y, int d, __half* x_out,
+                                                   __half* trace_x) {
+  __shared__ float red[2][8];
+  const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  float s = 0.f, s2 = 0.f;
+  for (int j = t; j < d; j += 256) {
+    const float v = __half2float(x[(size_t)b * d + j]) + y[(size_t)b * d + j];
+    s += v;
+    s2 += v * v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  }
+  if (lane == 0) { red[0][warp] = s; red[1][warp] = s2; }
+  __syncthreads();
+  float sum = 0.f, sumsq = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) { sum += red[0][w]; sumsq += red[1][w]; }
+  const float mean = sum / (float)d;
+  const float sd = sqrtf(fmaxf(sumsq / (float)d - mean * mean, 0.f) + 1e-6f);
+  __syncthreads();
+  for (int j = t; j < d; j += 256) {
+    const float v = __half2float(x[(size_t)b * d + j]) + y[(size_t)b * d + j];
+    const __half o = __float2half_rn((v - mean) / sd);
+    x_out[(size_t)b * d + j] = o;
+    if (trace_x) trace_x[(size_t)b * d + j] = o;
+  }
+}
+
+template <int NT>
+cudaError_t launch_rowtok_nt(const RowTokArgs& a, int nmat, int blocks, cudaStream_t s) {
+  const bool split = a.tok_lo != nullptr;
+  const int ns = split ? 2 : 1;
+  const size_t smem = (size_t)nmat * kRows * kPad + (size_t)ns * NT * 8 * kPad;
+  if (nmat == 2) {
+    if (split) return cudaErrorNotSupported;
+    auto k = rowtok_kernel<NT, 2, false>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<blocks, 32 * kBW, smem, s>>>(a);
+  } else if (split) {
+    auto k = rowtok_kernel<NT, 1, true>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<blocks, 32 * kBW, smem, s>>>(a);
+  } else {
+    auto k = rowtok_kernel<NT, 1, false>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<blocks, 32 * kBW, smem, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rowtok(const RowTokArgs& a, int nmat, int rows_max, cudaStream_t s) {
+  const int blocks = (rows_max + kRows - 1) / kRows;
+  if (blocks <= 0) return cudaSuccess;
+  switch ((a.B + 7) / 8) {
+    case 1: return launch_rowtok_nt<1>(a, nmat, blocks, s);
+    case 2: return launch_rowtok_nt<2>(a, nmat, blocks, s);
+    case 3: return launch_rowtok_nt<3>(a, nmat, blocks, s);
+    case 4: return launch_rowtok_nt<4>(a, nmat, blocks, s);
+  }
+  return cudaErrorNotSupported;
+}
+
+template <int NT>
+cudaError_t launch_down_nt(const DownArgs& a, cudaStream_t s) {
+  const size_t smem = (size_t)kRows * kPad + 2 * (size_t)NT * 8 * kPad;
+  auto k = down_kernel<NT>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  k<<<(a.d + kRows - 1) / kRows, 32 * kBW, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool batched_supported(int family, int B, int d, int r) {
+  return family == FAM_F16 && B >= 1 && B <= 32 && d % kKC == 0 && r % kKC == 0 && d % kRows == 0;
+}
+
+cudaError_t batched_predict(const BatchedLayer& L, const void* x, int B, uint32_t* mask, float* logits,
+                            __half* u_hi, __half* u_lo, cudaStream_t s) {
+  RowTokArgs a{};
+  a.mode = ROWS_P1;
+  a.nrows_static = L.r;
+  a.K = L.d;
+  a.B = B;
+  a.base = L.p1t;
+  a.stride = L.p1_row;
+  a.tok = reinterpret_cast<const __half*>(x);
+  a.u_hi = u_hi;
+  a.u_lo = u_lo;
+  cudaError_t e = launch_rowtok(a, 1, L.r, s);
+  if (e != cudaSuccess) return e;
+  RowTokArgs b{};
+  b.mode = ROWS_P2;
+  b.nrows_static = L.f;
+  b.K = L.r;
+  b.B = B;
+  b.base = L.p2o;
+  b.stride = L.p2_stride;
+  b.G = L.G;
+  b.nown_max = L.nown_max;
+  b.tok = u_hi;
+  b.tok_lo = u_lo;
+  b.thresh = L.thresh;
+  b.logits = logits;
+  b.mask = mask;
+  b.f = L.f;
+  return launch_rowtok(b, 1, L.f, s);
+}
+
+cudaError_t batched_ffn(const BatchedLayer& L, const void* x, int B, const uint32_t* mask, const int32_t* idx,
+                        const int32_t* count, float* h, float* y, int* err, cudaStream_t s) {
+  RowTokArgs a{};
+  a.mode = ROWS_FFN;
+  a.nrows_static = L.f;
+  a.count = count;
+  a.K = L.d;
+  a.B = B;
+  a.base = L.rec;
+  a.stride = L.rec_stride;
+  a.idx = idx;
+  a.up_off = L.up_off;
+  a.gate_off = L.gate_off;
+  a.tok = reinterpret_cast<const __half*>(x);
+  a.bias = L.bias;
+  a.mask_in = mask;
+  a.f = L.f;
+  a.h = h;
+  a.err = err;
+  cudaError_t e = launch_rowtok(a, L.gate_off >= 0 ? 2 : 1, L.f, s);
+  if (e != cudaSuccess) return e;
+  DownArgs dn{};
+  dn.count = count;
+  dn.fmax = L.f;
+  dn.d = L.d;
+  dn.B = B;
+  dn.rec = L.rec;
+  dn.rec_stride = L.rec_stride;
+  dn.down_off = L.down_off;
+  dn.idx = idx;
+  dn.h = h;
+  dn.y = y;
+  dn.err = err;
+  switch ((B + 7) / 8) {
+    case 1: return launch_down_nt<1>(dn, s);
+    case 2: return launch_down_nt<2>(dn, s);
+    case 3: return launch_down_nt<3>(dn, s);
+    case 4: return launch_down_nt<4>(dn, s);
+  }
+  return cudaErrorNotSupported;
+}
+
+namespace {
+__global__ void count_add_kernel(const int32_t* count, unsigned long long* total, int32_t* layer_count) {
+  const int c = *count;
+  atomicAdd(total, (unsigned long long)c);
+  if (layer_count) *layer_count = c;
+}
+}  // namespace
+
+cudaError_t batched_count(const int32_t* count, unsigned long long* total, int32_t* layer_count, cudaStream_t s) {
+  count_add_kernel<<<1, 1, 0, s>>>(count, total, layer_count);
+  return cudaGetLastError();
+}
+
+cudaError_t batched_glue(const void* x, const float* y, int B, int d, void* x_out, void* trace_x, cudaStream_t s) {
+  glue_kernel<<<B, 256, 0, s>>>(reinterpret_cast<const __half*>(x), y, d, reinterpret_cast<__half*>(x_out),
+                                reinterpret_cast<__half*>(trace_x));
+  return cudaGetLastError();
+}
+
+}  // namespace pi

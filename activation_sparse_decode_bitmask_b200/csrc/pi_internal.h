@@ -2,6 +2,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "../../include/pi_sparse_ffn.h"
@@ -78,6 +79,14 @@ struct pi_workspace {
   unsigned long long* active_total;  // running sum of active-list lengths (all calls)
   int32_t* layer_count;              // [L_max] per-layer union active count of the last stack
   void* x_dev;       // [B_max][d_max] staging for pi_decode_stack_host (fp32 size)
+  // batched path (B_max > 4 only)
+  __half* u_hi;      // [32][r_max] u as fp16 high part
+  __half* u_lo;      // [32][r_max] u low part
+  uint32_t* bmask;   // [32][f_max/32]
+  int32_t* bidx;     // [f_max]
+  int32_t* bcount;   // [1]
+  float* bh;         // [f_max][32] h of the active neurons
+  float* by;         // [32][d_max] FFN output
   long long* phase_clk;  // diagnostics: [grid][L_max][12] stamps, or null when off
   int phase_global;      // 1: stamps from the global ns timer
   void* x_host_pinned;
@@ -130,6 +139,26 @@ cudaError_t launch_fused(int family, int act, int B, const FusedParams& p, size_
 size_t fused_fixed_smem(int B, int d, int r, int grid, int nown_max, int family);
 bool fused_supported(int family, int B, int d);
 cudaError_t launch_barrier_probe(const FusedParams& p, int rounds, cudaStream_t stream);
+
+// Batched path (up to 32 tokens, fp16 family): tensor-core tiles for every contraction.
+struct BatchedLayer {
+  int d, f, r, G, nown_max;
+  const uint8_t* rec;
+  int rec_stride, up_off, gate_off, down_off;
+  const uint8_t* p1t;
+  int p1_row;
+  const uint8_t* p2o;
+  int p2_stride;
+  const float* thresh;
+  const float* bias;
+};
+bool batched_supported(int family, int B, int d, int r);
+cudaError_t batched_predict(const BatchedLayer& L, const void* x, int B, uint32_t* mask, float* logits,
+                            __half* u_hi, __half* u_lo, cudaStream_t s);
+cudaError_t batched_ffn(const BatchedLayer& L, const void* x, int B, const uint32_t* mask, const int32_t* idx,
+                        const int32_t* count, float* h, float* y, int* err, cudaStream_t s);
+cudaError_t batched_glue(const void* x, const float* y, int B, int d, void* x_out, void* trace_x, cudaStream_t s);
+cudaError_t batched_count(const int32_t* count, unsigned long long* total, int32_t* layer_count, cudaStream_t s);
 
 cudaError_t launch_compact(const uint32_t* mask, int B, int f, int32_t* idx, int32_t* count,
                            cudaStream_t stream);
