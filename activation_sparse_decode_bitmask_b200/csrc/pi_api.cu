@@ -181,10 +181,11 @@ pi_status decode_stack_batched(pi_layer* const* layers, int Lc, void* x_inout, i
     float* y = (trace && trace->y) ? trace->y + (size_t)l * B * d : ws->by;
     void* tx = (trace && trace->x) ? static_cast<uint8_t*>(trace->x) + (size_t)(l + 1) * B * d * 2 : nullptr;
     PI_TRY(cudaMemsetAsync(mask, 0, (size_t)B * words * 4, stream));
-    PI_TRY(batched_predict(bl, x_inout, B, mask, logits, ws->u_hi, ws->u_lo, stream));
+    PI_TRY(batched_predict(bl, x_inout, B, mask, logits, ws->u_hi, ws->u_lo, ws->bpart, ws->bpart_floats, stream));
     PI_TRY(launch_compact(mask, B, f, idx, count, stream));
     PI_TRY(batched_count(count, ws->active_total, ws->layer_count + l, stream));
-    PI_TRY(batched_ffn(bl, x_inout, B, mask, idx, count, ws->bh, y, ws->err, stream));
+    PI_TRY(batched_ffn(bl, x_inout, B, mask, idx, count, ws->bh, y, ws->bpart, ws->bpart_floats, ws->bypart, ws->err,
+                       stream));
     PI_TRY(batched_glue(x_inout, y, B, d, x_inout, tx, stream));
   }
   return PI_OK;
@@ -398,6 +399,9 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
          dmalloc(&ws->bmask, (size_t)32 * (f_max / 32) * 4) == cudaSuccess && dmalloc(&ws->bidx, (size_t)f_max * 4) == cudaSuccess &&
          dmalloc(&ws->bcount, 16) == cudaSuccess && dmalloc(&ws->bh, (size_t)f_max * 32 * 4) == cudaSuccess &&
          dmalloc(&ws->by, (size_t)32 * d_max * 4) == cudaSuccess;
+    ws->bpart_floats = batched_part_floats(d_max, f_max, r_max);
+    ok = ok && dmalloc(&ws->bpart, ws->bpart_floats * 4) == cudaSuccess &&
+         dmalloc(&ws->bypart, batched_ypart_floats(d_max) * 4) == cudaSuccess;
   }
   if (ok) {
     // tagged words start with tag 0; launch epochs start at 1, so no stale word matches
@@ -424,7 +428,7 @@ void pi_workspace_free(pi_workspace* ws) {
   cudaFree(ws->bar); cudaFree(ws->err); cudaFree(ws->active_total);
   cudaFree(ws->layer_count); cudaFree(ws->x_dev); cudaFree(ws->phase_clk);
   cudaFree(ws->u_hi); cudaFree(ws->u_lo); cudaFree(ws->bmask); cudaFree(ws->bidx); cudaFree(ws->bcount);
-  cudaFree(ws->bh); cudaFree(ws->by);
+  cudaFree(ws->bh); cudaFree(ws->by); cudaFree(ws->bpart); cudaFree(ws->bypart);
   delete ws;
 }
 
@@ -466,7 +470,7 @@ pi_status pi_predict(const pi_layer* L, const void* x, int B, uint32_t* mask, fl
   if (use_batched(L, B)) {
     if (!batched_supported(L->family, B, L->desc.d_model, L->desc.rank) || !ws->u_hi) return PI_ERR_UNSUPPORTED;
     PI_TRY(cudaMemsetAsync(mask, 0, (size_t)B * (L->desc.d_ff / 32) * 4, stream));
-    PI_TRY(batched_predict(bview(L), x, B, mask, logits, ws->u_hi, ws->u_lo, stream));
+    PI_TRY(batched_predict(bview(L), x, B, mask, logits, ws->u_hi, ws->u_lo, ws->bpart, ws->bpart_floats, stream));
     return PI_OK;
   }
   FusedParams p;
@@ -497,7 +501,8 @@ pi_status pi_sparse_ffn(const pi_layer* L, const void* x, int B, const uint32_t*
   if (st != PI_OK) return st;
   if (use_batched(L, B)) {
     if (!batched_supported(L->family, B, L->desc.d_model, L->desc.rank) || !ws->u_hi) return PI_ERR_UNSUPPORTED;
-    PI_TRY(batched_ffn(bview(L), x, B, mask, idx, count, ws->bh, y, ws->err, stream));
+    PI_TRY(batched_ffn(bview(L), x, B, mask, idx, count, ws->bh, y, ws->bpart, ws->bpart_floats, ws->bypart, ws->err,
+                       stream));
     return PI_OK;
   }
   FusedParams p;

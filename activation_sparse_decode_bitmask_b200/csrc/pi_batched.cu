@@ -15,6 +15,7 @@
 // row tiles of every layer are its dense hot block and the rest are gathered cold rows.
 // Every sum runs in a fixed order: results are bitwise reproducible.
 #include <cuda_fp16.h>
+#include <algorithm>
 #include <cstdint>
 
 #include "pi_internal.h"
@@ -28,12 +29,15 @@ constexpr int kBW = 4;                    // warps per block
 constexpr int kRows = 16 * kBW;           // rows (or columns) per block
 constexpr int kKC = 64;                   // K elements staged per chunk
 constexpr int kPad = kKC * 2 + 16;        // bytes per staged row: the 16-byte pad keeps ldmatrix conflict-free
+constexpr int kMaxKSplit = 32;            // K splits of a row kernel at most
+constexpr int kMaxDownSplit = 16;         // neuron splits of the down kernel at most
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -61,33 +65,26 @@ __device__ __forceinline__ void split_h(float v, __half& hi, __half& lo) {
 }
 
 // ------------------------------------------------------------------ rows x tokens
-// out[row][token] = sum_k Rows[row][k] * Tok[token][k] for a block of 64 rows and all
-// tokens; Rows are fp16 rows found through the mode's addressing, Tok is [B][K] fp16 (and
-// a second [B][K] fp16 low part when SPLIT).
+// part[split][row][token] = sum over the split's K range of Rows[row][k] * Tok[token][k]
+// for a block of 64 rows and all tokens.  Rows are fp16 rows found through the mode's
+// addressing; Tok is [B][K] fp16 (plus a [B][K] low part when SPLIT).  Chunks of 64 K
+// stream through a 3-stage cp.async pipeline.  An epilogue kernel then sums the splits in
+// order and finishes the mode's step.
 enum RowMode { ROWS_P1 = 0, ROWS_P2 = 1, ROWS_FFN = 2 };
+constexpr int kStages = 3;
 
 struct RowTokArgs {
-  int mode, nrows_static, K, B;
+  int mode, nrows_static, K, B, ksplit;
   const int32_t* count;        // ROWS_FFN: number of active rows (device)
   const uint8_t* base;         // row storage
   int stride;                  // bytes between consecutive rows (P1) or per record / P2 row
   int G, nown_max;             // ROWS_P2: owner-major placement of neuron rows
   const int32_t* idx;          // ROWS_FFN: stored ids of the active neurons
   int up_off, gate_off;        // ROWS_FFN: byte offsets of the rows in a record (gate < 0: ReLU)
+  int f;
   const __half* tok;           // [B][K]
   const __half* tok_lo;        // [B][K] or null
-  // ROWS_P1 output: u as fp16 hi / lo, [B][r]
-  __half* u_hi;
-  __half* u_lo;
-  // ROWS_P2 output
-  const float* thresh;         // [f]
-  float* logits;               // [B][f] or null
-  uint32_t* mask;              // [B][f/32], zeroed by the caller; bits are OR-ed in
-  int f;
-  // ROWS_FFN output
-  const float* bias;           // [f]
-  const uint32_t* mask_in;     // [B][f/32]
-  float* h;                    // [count][32]
+  float* part;                 // [ksplit][NMAT][nrows_static][32]
   int* err;                    // device error word (index or count out of range)
 };
 
@@ -95,14 +92,13 @@ template <int NT, int NMAT, bool SPLIT>
 __global__ void __launch_bounds__(32 * kBW) rowtok_kernel(const RowTokArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int NS = SPLIT ? 2 : 1;
-  constexpr int BP = NT * 8;                       // padded tokens
-  uint8_t* rows_s = smem;                          // [NMAT][kRows][kPad]
-  uint8_t* tok_s = smem + NMAT * kRows * kPad;     // [NS][BP][kPad]
+  constexpr int BP = NT * 8;                                   // padded tokens
+  constexpr int ROWS_B = NMAT * kRows * kPad, TOK_B = NS * BP * kPad, STAGE_B = ROWS_B + TOK_B;
   int nrows = a.nrows_static;
   if (a.mode == ROWS_FFN) {
     const int cnt = *a.count;
     if (cnt < 0 || cnt > a.nrows_static) {
-      if (blockIdx.x == 0 && threadIdx.x == 0) atomicExch(a.err, DEV_ERR_INDEX);
+      if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) atomicExch(a.err, DEV_ERR_INDEX);
       return;
     }
     nrows = cnt;
@@ -110,23 +106,36 @@ __global__ void __launch_bounds__(32 * kBW) rowtok_kernel(const RowTokArgs a) {
   const int row0 = blockIdx.x * kRows;
   if (row0 >= nrows) return;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  // stored id of active row j, checked against d_ff (a bad id reads neuron 0 and is reported)
-  auto active_id = [&](int j) -> int {
-    int i = __ldg(a.idx + j);
-    if (i < 0 || i >= a.f) {
-      atomicExch(a.err, DEV_ERR_INDEX);
-      i = 0;
-    }
-    return i;
-  };
+  const int nch = a.K / kKC;
+  const int c_begin = (int)((long long)blockIdx.y * nch / a.ksplit);
+  const int c_end = (int)((long long)(blockIdx.y + 1) * nch / a.ksplit);
 
-  // byte address of row j (clamped into range: rows past the end repeat the last one
-  // and their results are never stored), matrix m
+  // byte address of row j (clamped into range: rows past the end repeat the last one and
+  // their results are never used), matrix m
   auto row_ptr = [&](int j, int m) -> const uint8_t* {
     j = min(j, nrows - 1);
     if (a.mode == ROWS_P1) return a.base + (size_t)j * a.stride;
     if (a.mode == ROWS_P2) return a.base + ((size_t)(j % a.G) * a.nown_max + j / a.G) * a.stride;
-    return a.base + (size_t)active_id(j) * a.stride + (m == 0 ? a.up_off : a.gate_off);
+    int i = __ldg(a.idx + j);
+    if (i < 0 || i >= a.f) {   // a bad id reads neuron 0 and is reported
+      atomicExch(a.err, DEV_ERR_INDEX);
+      i = 0;
+    }
+    return a.base + (size_t)i * a.stride + (m == 0 ? a.up_off : a.gate_off);
+  };
+  const uint32_t base_u = smem_u32(smem);
+  auto stage_chunk = [&](int ch, int buf) {
+    const int k0 = ch * kKC;
+    const uint32_t rows_u = base_u + (uint32_t)(buf * STAGE_B), tok_u = rows_u + ROWS_B;
+    for (int e = t; e < NMAT * kRows * 8; e += 32 * kBW) {
+      const int m = e / (kRows * 8), rr = (e / 8) % kRows, pc = e % 8;
+      cp_async16(rows_u + (uint32_t)((m * kRows + rr) * kPad + pc * 16), row_ptr(row0 + rr, m) + (size_t)k0 * 2 + pc * 16);
+    }
+    for (int e = t; e < NS * BP * 8; e += 32 * kBW) {
+      const int s = e / (BP * 8), b = (e / 8) % BP, pc = e % 8;
+      const __half* src = (s == 0 ? a.tok : a.tok_lo) + (size_t)min(b, a.B - 1) * a.K + k0 + pc * 8;
+      cp_async16(tok_u + (uint32_t)((s * BP + b) * kPad + pc * 16), src);
+    }
   };
 
   float c[NMAT][NT][4];
@@ -137,21 +146,18 @@ __global__ void __launch_bounds__(32 * kBW) rowtok_kernel(const RowTokArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) c[m][n][e] = 0.f;
 
-  const uint32_t rows_u = smem_u32(rows_s), tok_u = smem_u32(tok_s);
-  for (int k0 = 0; k0 < a.K; k0 += kKC) {
-    // stage the chunk: rows (NMAT x 64 rows x 8 pieces of 16 bytes) and tokens
-    for (int e = t; e < NMAT * kRows * 8; e += 32 * kBW) {
-      const int m = e / (kRows * 8), rr = (e / 8) % kRows, pc = e % 8;
-      cp_async16(rows_u + (uint32_t)((m * kRows + rr) * kPad + pc * 16), row_ptr(row0 + rr, m) + (size_t)k0 * 2 + pc * 16);
-    }
-    for (int e = t; e < NS * BP * 8; e += 32 * kBW) {
-      const int s = e / (BP * 8), b = (e / 8) % BP, pc = e % 8;
-      const __half* src = (s == 0 ? a.tok : a.tok_lo) + (size_t)min(b, a.B - 1) * a.K + k0 + pc * 8;
-      cp_async16(tok_u + (uint32_t)((s * BP + b) * kPad + pc * 16), src);
-    }
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (c_begin + s < c_end) stage_chunk(c_begin + s, s);
     cp_async_commit();
-    cp_async_wait_all();
-    __syncthreads();
+  }
+  for (int ch = c_begin; ch < c_end; ++ch) {
+    cp_async_wait_1();
+    __syncthreads();   // chunk ch landed for every thread; chunk ch - 1's buffer is free
+    if (ch + kStages - 1 < c_end) stage_chunk(ch + kStages - 1, (ch + kStages - 1 - c_begin) % kStages);
+    cp_async_commit();
+    const int buf = (ch - c_begin) % kStages;
+    const uint32_t rows_u = base_u + (uint32_t)(buf * STAGE_B), tok_u = rows_u + ROWS_B;
 #pragma unroll
     for (int ks = 0; ks < kKC / 16; ++ks) {
       uint32_t af[NMAT][4];
@@ -174,83 +180,114 @@ __global__ void __launch_bounds__(32 * kBW) rowtok_kernel(const RowTokArgs a) {
         }
       }
     }
-    __syncthreads();   // the stage is refilled next chunk
   }
+  cp_async_wait_all();
 
-  // epilogue: thread holds rows g and g + 8 of the warp's tile, tokens 2t and 2t + 1 of
-  // every 8-token tile
+  // raw partials: thread holds rows g and g + 8 of the warp's tile, tokens 2t and 2t + 1
+  // of every 8-token tile
   const int g = lane >> 2, tq = lane & 3;
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     const int j = row0 + warp * 16 + g + 8 * half;
     if (j >= nrows) continue;
 #pragma unroll
-    for (int n = 0; n < NT; ++n)
+    for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int b = n * 8 + 2 * tq + q;
-        const float v0 = c[0][n][2 * half + q];
-        if (a.mode == ROWS_P1) {
-          if (b < a.B) {
-            __half hi, lo;
-            split_h(v0, hi, lo);
-            a.u_hi[(size_t)b * a.nrows_static + j] = hi;
-            a.u_lo[(size_t)b * a.nrows_static + j] = lo;
-          }
-        } else if (a.mode == ROWS_P2) {
-          if (b < a.B) {
-            const float lg = v0 - __ldg(a.thresh + j);
-            if (a.logits) a.logits[(size_t)b * a.f + j] = lg;
-            if (lg > 0.f) atomicOr(a.mask + (size_t)b * (a.f / 32) + (j >> 5), 1u << (j & 31));
-          }
-        } else {
-          float hv = 0.f;
-          if (b < a.B) {
-            const int i = active_id(j);
-            const uint32_t bit = (__ldg(a.mask_in + (size_t)b * (a.f / 32) + (i >> 5)) >> (i & 31)) & 1u;
-            const float bi = __ldg(a.bias + i);
-            float act;
-            if constexpr (NMAT == 2) act = fmaxf(c[1][n][2 * half + q] + bi, 0.f) * v0;   // gate is matrix 1
-            else act = fmaxf(v0 + bi, 0.f);
-            hv = bit ? act : 0.f;
-          }
-          a.h[(size_t)j * 32 + b] = hv;
-        }
+      for (int n = 0; n < NT; ++n) {
+        float2 v = make_float2(c[m][n][2 * half], c[m][n][2 * half + 1]);
+        *reinterpret_cast<float2*>(a.part + (((size_t)blockIdx.y * NMAT + m) * a.nrows_static + j) * 32 + n * 8 + 2 * tq) = v;
       }
   }
 }
 
+// Sum the splits of part (fixed order) and finish the mode's step, one thread per
+// (row, token).
+struct RowEpiArgs {
+  int mode, nrows_static, B, ksplit, nmat;
+  const int32_t* count;
+  const int32_t* idx;
+  int f;
+  const float* part;
+  __half* u_hi;                // ROWS_P1: [B][r]
+  __half* u_lo;
+  const float* thresh;         // ROWS_P2
+  float* logits;               // [B][f] or null
+  uint32_t* mask;              // [B][f/32], zeroed by the caller
+  const float* bias;           // ROWS_FFN
+  const uint32_t* mask_in;     // [B][f/32]
+  float* h;                    // [count][32]
+};
+
+__global__ void __launch_bounds__(256) rowtok_epilogue(const RowEpiArgs a) {
+  int nrows = a.nrows_static;
+  if (a.mode == ROWS_FFN) {
+    const int cnt = *a.count;
+    if (cnt < 0 || cnt > a.nrows_static) return;   // reported by the row kernel
+    nrows = cnt;
+  }
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = (int)(e / 32), b = (int)(e % 32);
+  if (j >= nrows) return;
+  float v[2] = {0.f, 0.f};
+  for (int s = 0; s < a.ksplit; ++s)
+    for (int m = 0; m < a.nmat; ++m) v[m] += a.part[(((size_t)s * a.nmat + m) * a.nrows_static + j) * 32 + b];
+  if (a.mode == ROWS_P1) {
+    if (b < a.B) {
+      __half hi, lo;
+      split_h(v[0], hi, lo);
+      a.u_hi[(size_t)b * a.nrows_static + j] = hi;
+      a.u_lo[(size_t)b * a.nrows_static + j] = lo;
+    }
+  } else if (a.mode == ROWS_P2) {
+    if (b < a.B) {
+      const float lg = v[0] - __ldg(a.thresh + j);
+      if (a.logits) a.logits[(size_t)b * a.f + j] = lg;
+      if (lg > 0.f) atomicOr(a.mask + (size_t)b * (a.f / 32) + (j >> 5), 1u << (j & 31));
+    }
+  } else {
+    float hv = 0.f;
+    if (b < a.B) {
+      int i = __ldg(a.idx + j);
+      if (i < 0 || i >= a.f) i = 0;   // reported by the row kernel
+      const uint32_t bit = (__ldg(a.mask_in + (size_t)b * (a.f / 32) + (i >> 5)) >> (i & 31)) & 1u;
+      const float bi = __ldg(a.bias + i);
+      const float act = (a.nmat == 2) ? fmaxf(v[1] + bi, 0.f) * v[0] : fmaxf(v[0] + bi, 0.f);   // matrix 1: gate
+      hv = bit ? act : 0.f;
+    }
+    a.h[(size_t)j * 32 + b] = hv;
+  }
+}
+
 // ------------------------------------------------------------------ down projection
-// y[b][c] = sum_j h[j][b] * Wd[idx[j]][c] for a block of 64 columns and all tokens: the
-// columns' slices of the active down rows are staged [neuron][column] and read transposed.
+// ypart[split][b][c] = sum over the split's neurons j of h[j][b] * Wd[idx[j]][c], for a
+// block of 64 columns and all tokens: the columns' slices of the active down rows are
+// staged [neuron][column] and read transposed; then the splits are summed in order.
 struct DownArgs {
   const int32_t* count;
-  int fmax, d, B;
+  int fmax, d, B, nsplit;
   const uint8_t* rec;
   int rec_stride, down_off;
   const int32_t* idx;
-  const float* h;   // [count][32]
-  float* y;         // [B][d]
-  int* err;
+  const float* h;      // [count][32]
+  float* ypart;        // [nsplit][B][d]
 };
 
 template <int NT>
 __global__ void __launch_bounds__(32 * kBW) down_kernel(const DownArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int BP = NT * 8;
-  uint8_t* w_s = smem;                          // [64 neurons][kPad]: 64 columns of each row
-  uint8_t* h_s = smem + kRows * kPad;           // [2][BP][kPad]: h hi / lo per token, 64 neurons
+  constexpr int W_B = kRows * kPad, STAGE_B = W_B + 2 * BP * kPad;   // weights, then h hi / lo [2][BP]
   int count = *a.count;
   if (count < 0 || count > a.fmax) count = 0;   // reported by the gate/up kernel; y becomes 0
+  const int nch = (count + kRows - 1) / kRows;
+  const int c_begin = (int)((long long)blockIdx.y * nch / a.nsplit);
+  const int c_end = (int)((long long)(blockIdx.y + 1) * nch / a.nsplit);
   const int c0 = blockIdx.x * kRows;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  float c[NT][4];
-#pragma unroll
-  for (int n = 0; n < NT; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) c[n][e] = 0.f;
-  const uint32_t w_u = smem_u32(w_s), h_u = smem_u32(h_s);
-  for (int j0 = 0; j0 < count; j0 += kRows) {
+  const uint32_t base_u = smem_u32(smem);
+  auto stage_w = [&](int ch, int buf) {
+    const int j0 = ch * kRows;
+    const uint32_t w_u = base_u + (uint32_t)(buf * STAGE_B);
     for (int e = t; e < kRows * 8; e += 32 * kBW) {
       const int jj = e / 8, pc = e % 8;
       int i = __ldg(a.idx + min(j0 + jj, count - 1));
@@ -258,18 +295,35 @@ __global__ void __launch_bounds__(32 * kBW) down_kernel(const DownArgs a) {
       cp_async16(w_u + (uint32_t)(jj * kPad + pc * 16),
                  a.rec + (size_t)i * a.rec_stride + a.down_off + (size_t)c0 * 2 + pc * 16);
     }
+  };
+  float c[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c[n][e] = 0.f;
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (c_begin + s < c_end) stage_w(c_begin + s, s);
     cp_async_commit();
-    // h of the chunk, split into fp16 hi / lo; neurons past count contribute zero
+  }
+  for (int ch = c_begin; ch < c_end; ++ch) {
+    const int buf = (ch - c_begin) % kStages;
+    const uint32_t w_u = base_u + (uint32_t)(buf * STAGE_B), h_u = w_u + W_B;
+    // h of the chunk, split into fp16 hi / lo (neurons past count contribute zero); this
+    // buffer's previous readers finished before the last barrier
+    const int j0 = ch * kRows;
     for (int e = t; e < BP * kRows; e += 32 * kBW) {
       const int b = e / kRows, jj = e % kRows;
       const float v = (j0 + jj < count && b < a.B) ? a.h[(size_t)(j0 + jj) * 32 + b] : 0.f;
       __half hi, lo;
       split_h(v, hi, lo);
-      reinterpret_cast<__half*>(h_s + (size_t)b * kPad)[jj] = hi;
-      reinterpret_cast<__half*>(h_s + (size_t)(BP + b) * kPad)[jj] = lo;
+      reinterpret_cast<__half*>(smem + buf * STAGE_B + W_B + (size_t)b * kPad)[jj] = hi;
+      reinterpret_cast<__half*>(smem + buf * STAGE_B + W_B + (size_t)(BP + b) * kPad)[jj] = lo;
     }
-    cp_async_wait_all();
-    __syncthreads();
+    cp_async_wait_1();
+    __syncthreads();   // weights and h of chunk ch are in place; chunk ch - 1's buffer is free
+    if (ch + kStages - 1 < c_end) stage_w(ch + kStages - 1, (ch + kStages - 1 - c_begin) % kStages);
+    cp_async_commit();
 #pragma unroll
     for (int ks = 0; ks < kRows / 16; ++ks) {
       uint32_t af[4];
@@ -289,8 +343,9 @@ __global__ void __launch_bounds__(32 * kBW) down_kernel(const DownArgs a) {
           mma16816(c[n], af, bf);
         }
     }
-    __syncthreads();
+    __syncthreads();   // every thread is done with this buffer before its h is rewritten
   }
+  cp_async_wait_all();
   const int g = lane >> 2, tq = lane & 3;
 #pragma unroll
   for (int n = 0; n < NT; ++n)
@@ -298,8 +353,16 @@ __global__ void __launch_bounds__(32 * kBW) down_kernel(const DownArgs a) {
     for (int e = 0; e < 4; ++e) {
       const int col = c0 + warp * 16 + g + 8 * (e >> 1);
       const int b = n * 8 + 2 * tq + (e & 1);
-      if (b < a.B && col < a.d) a.y[(size_t)b * a.d + col] = c[n][e];
+      if (b < a.B && col < a.d) a.ypart[((size_t)blockIdx.y * a.B + b) * a.d + col] = c[n][e];
     }
+}
+
+__global__ void __launch_bounds__(256) down_reduce(const float* ypart, int nsplit, int n, float* y) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= n) return;
+  float v = 0.f;
+  for (int s = 0; s < nsplit; ++s) v += ypart[(size_t)s * n + e];
+  y[e] = v;
 }
 
 // ------------------------------------------------------------------ stack glue
@@ -336,46 +399,68 @@ __global__ void __launch_bounds__(256) glue_kernel(const __half* x, const float*
   }
 }
 
+// K splits: enough blocks to cover the SMs a few times over, at least two chunks each.
+int ksplit_for(int row_blocks, int nch) {
+  const int target = 4 * 148;
+  int s = (target + row_blocks - 1) / max(row_blocks, 1);
+  s = min(s, max(1, nch / 2));
+  return max(1, min(s, kMaxKSplit));
+}
+
 template <int NT>
 cudaError_t launch_rowtok_nt(const RowTokArgs& a, int nmat, int blocks, cudaStream_t s) {
   const bool split = a.tok_lo != nullptr;
   const int ns = split ? 2 : 1;
-  const size_t smem = (size_t)nmat * kRows * kPad + (size_t)ns * NT * 8 * kPad;
+  const size_t smem = (size_t)kStages * ((size_t)nmat * kRows * kPad + (size_t)ns * NT * 8 * kPad);
+  const dim3 grid(blocks, a.ksplit);
   if (nmat == 2) {
     if (split) return cudaErrorNotSupported;
     auto k = rowtok_kernel<NT, 2, false>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<blocks, 32 * kBW, smem, s>>>(a);
+    k<<<grid, 32 * kBW, smem, s>>>(a);
   } else if (split) {
     auto k = rowtok_kernel<NT, 1, true>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<blocks, 32 * kBW, smem, s>>>(a);
+    k<<<grid, 32 * kBW, smem, s>>>(a);
   } else {
     auto k = rowtok_kernel<NT, 1, false>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<blocks, 32 * kBW, smem, s>>>(a);
+    k<<<grid, 32 * kBW, smem, s>>>(a);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_rowtok(const RowTokArgs& a, int nmat, int rows_max, cudaStream_t s) {
+// The row kernel for rows_max rows (an upper bound when the count is on the device), then
+// its epilogue.
+cudaError_t launch_rows(RowTokArgs a, RowEpiArgs ep, int nmat, int rows_max, size_t part_floats, cudaStream_t s) {
   const int blocks = (rows_max + kRows - 1) / kRows;
   if (blocks <= 0) return cudaSuccess;
+  a.ksplit = ksplit_for(blocks, a.K / kKC);
+  const size_t per_split = (size_t)nmat * a.nrows_static * 32;
+  a.ksplit = (int)std::max<size_t>(1, std::min<size_t>(a.ksplit, part_floats / per_split));
+  if (per_split > part_floats) return cudaErrorInvalidValue;
+  cudaError_t e = cudaErrorNotSupported;
   switch ((a.B + 7) / 8) {
-    case 1: return launch_rowtok_nt<1>(a, nmat, blocks, s);
-    case 2: return launch_rowtok_nt<2>(a, nmat, blocks, s);
-    case 3: return launch_rowtok_nt<3>(a, nmat, blocks, s);
-    case 4: return launch_rowtok_nt<4>(a, nmat, blocks, s);
+    case 1: e = launch_rowtok_nt<1>(a, nmat, blocks, s); break;
+    case 2: e = launch_rowtok_nt<2>(a, nmat, blocks, s); break;
+    case 3: e = launch_rowtok_nt<3>(a, nmat, blocks, s); break;
+    case 4: e = launch_rowtok_nt<4>(a, nmat, blocks, s); break;
   }
-  return cudaErrorNotSupported;
+  if (e != cudaSuccess) return e;
+  ep.ksplit = a.ksplit;
+  ep.nmat = nmat;
+  ep.part = a.part;
+  const long long n = (long long)rows_max * 32;
+  rowtok_epilogue<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ep);
+  return cudaGetLastError();
 }
 
 template <int NT>
 cudaError_t launch_down_nt(const DownArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)kRows * kPad + 2 * (size_t)NT * 8 * kPad;
+  const size_t smem = (size_t)kStages * ((size_t)kRows * kPad + 2 * (size_t)NT * 8 * kPad);
   auto k = down_kernel<NT>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  k<<<(a.d + kRows - 1) / kRows, 32 * kBW, smem, s>>>(a);
+  k<<<dim3((a.d + kRows - 1) / kRows, a.nsplit), 32 * kBW, smem, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -386,7 +471,7 @@ bool batched_supported(int family, int B, int d, int r) {
 }
 
 cudaError_t batched_predict(const BatchedLayer& L, const void* x, int B, uint32_t* mask, float* logits,
-                            __half* u_hi, __half* u_lo, cudaStream_t s) {
+                            __half* u_hi, __half* u_lo, float* part, size_t part_floats, cudaStream_t s) {
   RowTokArgs a{};
   a.mode = ROWS_P1;
   a.nrows_static = L.r;
@@ -395,9 +480,14 @@ cudaError_t batched_predict(const BatchedLayer& L, const void* x, int B, uint32_
   a.base = L.p1t;
   a.stride = L.p1_row;
   a.tok = reinterpret_cast<const __half*>(x);
-  a.u_hi = u_hi;
-  a.u_lo = u_lo;
-  cudaError_t e = launch_rowtok(a, 1, L.r, s);
+  a.part = part;
+  RowEpiArgs ea{};
+  ea.mode = ROWS_P1;
+  ea.nrows_static = L.r;
+  ea.B = B;
+  ea.u_hi = u_hi;
+  ea.u_lo = u_lo;
+  cudaError_t e = launch_rows(a, ea, 1, L.r, part_floats, s);
   if (e != cudaSuccess) return e;
   RowTokArgs b{};
   b.mode = ROWS_P2;
@@ -410,15 +500,22 @@ cudaError_t batched_predict(const BatchedLayer& L, const void* x, int B, uint32_
   b.nown_max = L.nown_max;
   b.tok = u_hi;
   b.tok_lo = u_lo;
-  b.thresh = L.thresh;
-  b.logits = logits;
-  b.mask = mask;
-  b.f = L.f;
-  return launch_rowtok(b, 1, L.f, s);
+  b.part = part;
+  RowEpiArgs eb{};
+  eb.mode = ROWS_P2;
+  eb.nrows_static = L.f;
+  eb.B = B;
+  eb.f = L.f;
+  eb.thresh = L.thresh;
+  eb.logits = logits;
+  eb.mask = mask;
+  return launch_rows(b, eb, 1, L.f, part_floats, s);
 }
 
 cudaError_t batched_ffn(const BatchedLayer& L, const void* x, int B, const uint32_t* mask, const int32_t* idx,
-                        const int32_t* count, float* h, float* y, int* err, cudaStream_t s) {
+                        const int32_t* count, float* h, float* y, float* part, size_t part_floats, float* ypart,
+                        int* err, cudaStream_t s) {
+  const int nmat = L.gate_off >= 0 ? 2 : 1;
   RowTokArgs a{};
   a.mode = ROWS_FFN;
   a.nrows_static = L.f;
@@ -430,13 +527,21 @@ cudaError_t batched_ffn(const BatchedLayer& L, const void* x, int B, const uint3
   a.idx = idx;
   a.up_off = L.up_off;
   a.gate_off = L.gate_off;
-  a.tok = reinterpret_cast<const __half*>(x);
-  a.bias = L.bias;
-  a.mask_in = mask;
   a.f = L.f;
-  a.h = h;
+  a.tok = reinterpret_cast<const __half*>(x);
+  a.part = part;
   a.err = err;
-  cudaError_t e = launch_rowtok(a, L.gate_off >= 0 ? 2 : 1, L.f, s);
+  RowEpiArgs ea{};
+  ea.mode = ROWS_FFN;
+  ea.nrows_static = L.f;
+  ea.B = B;
+  ea.count = count;
+  ea.idx = idx;
+  ea.f = L.f;
+  ea.bias = L.bias;
+  ea.mask_in = mask;
+  ea.h = h;
+  cudaError_t e = launch_rows(a, ea, nmat, L.f, part_floats, s);
   if (e != cudaSuccess) return e;
   DownArgs dn{};
   dn.count = count;
@@ -448,16 +553,28 @@ cudaError_t batched_ffn(const BatchedLayer& L, const void* x, int B, const uint3
   dn.down_off = L.down_off;
   dn.idx = idx;
   dn.h = h;
-  dn.y = y;
-  dn.err = err;
+  dn.ypart = ypart;
+  const int col_blocks = (L.d + kRows - 1) / kRows;
+  dn.nsplit = std::min(kMaxDownSplit, std::max(1, (4 * 148 + col_blocks - 1) / col_blocks));
   switch ((B + 7) / 8) {
-    case 1: return launch_down_nt<1>(dn, s);
-    case 2: return launch_down_nt<2>(dn, s);
-    case 3: return launch_down_nt<3>(dn, s);
-    case 4: return launch_down_nt<4>(dn, s);
+    case 1: e = launch_down_nt<1>(dn, s); break;
+    case 2: e = launch_down_nt<2>(dn, s); break;
+    case 3: e = launch_down_nt<3>(dn, s); break;
+    case 4: e = launch_down_nt<4>(dn, s); break;
+    default: e = cudaErrorNotSupported;
   }
-  return cudaErrorNotSupported;
+  if (e != cudaSuccess) return e;
+  const int n = B * L.d;
+  down_reduce<<<(n + 255) / 256, 256, 0, s>>>(ypart, dn.nsplit, n, y);
+  return cudaGetLastError();
 }
+
+size_t batched_part_floats(int d_max, int f_max, int r_max) {
+  // row kernels: up to kMaxKSplit splits of the rank rows, and (bounded by this size)
+  // splits of the d_ff rows for two matrices; 32 token slots per row
+  return std::max((size_t)kMaxKSplit * r_max, (size_t)8 * 2 * f_max) * 32;
+}
+size_t batched_ypart_floats(int d_max) { return (size_t)kMaxDownSplit * 32 * d_max; }
 
 namespace {
 __global__ void count_add_kernel(const int32_t* count, unsigned long long* total, int32_t* layer_count) {

@@ -87,6 +87,9 @@ struct pi_workspace {
   int32_t* bcount;   // [1]
   float* bh;         // [f_max][32] h of the active neurons
   float* by;         // [32][d_max] FFN output
+  float* bpart;      // split partial sums of the row kernels
+  size_t bpart_floats;
+  float* bypart;     // split partial sums of the down kernel
   long long* phase_clk;  // diagnostics: [grid][L_max][12] stamps, or null when off
   int phase_global;      // 1: stamps from the global ns timer
   void* x_host_pinned;
@@ -154,9 +157,12 @@ struct BatchedLayer {
 };
 bool batched_supported(int family, int B, int d, int r);
 cudaError_t batched_predict(const BatchedLayer& L, const void* x, int B, uint32_t* mask, float* logits,
-                            __half* u_hi, __half* u_lo, cudaStream_t s);
+                            __half* u_hi, __half* u_lo, float* part, size_t part_floats, cudaStream_t s);
 cudaError_t batched_ffn(const BatchedLayer& L, const void* x, int B, const uint32_t* mask, const int32_t* idx,
-                        const int32_t* count, float* h, float* y, int* err, cudaStream_t s);
+                        const int32_t* count, float* h, float* y, float* part, size_t part_floats, float* ypart,
+                        int* err, cudaStream_t s);
+size_t batched_part_floats(int d_max, int f_max, int r_max);
+size_t batched_ypart_floats(int d_max);
 cudaError_t batched_glue(const void* x, const float* y, int B, int d, void* x_out, void* trace_x, cudaStream_t s);
 cudaError_t batched_count(const int32_t* count, unsigned long long* total, int32_t* layer_count, cudaStream_t s);
 
