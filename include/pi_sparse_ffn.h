@@ -5,7 +5,8 @@
  * describe it.
  *   - A small per-layer predictor says which FFN neurons will fire. Only those neurons
  *     are computed; the others are skipped (unite.ai "PowerInfer: Mesin Inferensi LLM
- *     Cepat dengan GPU Konsumen", §"Fase Online" and §"Prediktor Kepadatan Adaptif").
+ *     Cepat dengan GPU Konsumen", §"Fase Online: Mesin Inferensi LLM yang Sadar Neuron"
+ *     and §"Prediktor Kepadatan Adaptif").
  *   - Neuron-aware operators read the individual rows (up/gate) and columns (down) of
  *     the active neurons. There is no conversion to a dense format (same page,
  *     §"Operator yang Sadar Neuron").
@@ -13,7 +14,8 @@
  *     maps every placed neuron back to its original position (same page,
  *     §"Penempatan dan Pengelolaan Neuron"; KPD "PowerInfer: Fast Large Language Model
  *     Serving with a Consumer-grade GPU", §"Метод").
- *   - Activations: ReLU and ReGLU (GeekNews "PowerInfer", §"Kısıtlar ve SSS").
+ *   - Activations: ReLU and ReGLU (GeekNews "Tüketici sınıfı GPU takılı PC'lerde yüksek hızlı büyük dil modeli serving",
+ *     §"Kısıtlar ve SSS").
  *     Weights: fp32, fp16 or Q4_0 (same page, §"Kuantizasyon ve uyumluluk").
  *
  * Per layer and token x (d = d_model, f = d_ff, r = rank):

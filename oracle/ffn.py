@@ -5,13 +5,14 @@ baseline leg may import this module; the library never does, and this module nev
 imports the library.  It shares no code with the CUDA path.
 
 Sources (three web pages about PowerInfer; cited by page title and section):
-  [GN]  GeekNews digest "PowerInfer" (tr.news.hada.io), sections
-        "CPU/GPU hibrit çıkarım yöntemi", "Kuantizasyon ve uyumluluk", "Kısıtlar ve SSS".
+  [GN]  GeekNews "Tüketici sınıfı GPU takılı PC'lerde yüksek hızlı büyük dil modeli serving"
+        (tr.news.hada.io), sections "CPU/GPU hibrit çıkarım yöntemi", "Kuantizasyon ve
+        uyumluluk", "Kısıtlar ve SSS".
   [KPD] Telegram channel КПД, "PowerInfer: Fast Large Language Model Serving with a
         Consumer-grade GPU", sections "Введение", "Метод".
   [UAI] unite.ai "PowerInfer: Mesin Inferensi LLM Cepat dengan GPU Konsumen", sections
-        "Fase Online", "Prediktor Kepadatan Adaptif", "Penempatan dan Pengelolaan
-        Neuron", "Operator yang Sadar Neuron".
+        "Fase Online: Mesin Inferensi LLM yang Sadar Neuron", "Prediktor Kepadatan
+        Adaptif", "Penempatan dan Pengelolaan Neuron", "Operator yang Sadar Neuron".
 
 What it computes, for one layer and tokens x[b, :]:
   predictor  u = P1^T x ; logit_i = sum_k P2[k, i] u_k - t_i ; fires iff logit_i > 0
@@ -167,7 +168,7 @@ def sparse_ffn(x: np.ndarray, w: Dict[str, np.ndarray], act: str,
                masks: np.ndarray, idx: np.ndarray) -> np.ndarray:
     """Neuron-aware sparse FFN over the active list.
 
-    [UAI] §"Fase Online" and §"Operator yang Sadar Neuron": predicted-inactive neurons
+    [UAI] §"Fase Online: Mesin Inferensi LLM yang Sadar Neuron" and §"Operator yang Sadar Neuron": predicted-inactive neurons
     are skipped; the active ones are computed row by row (up/gate) and column by column
     (down).  masks: [B, f] bools (per token); idx: ascending union list.
     """

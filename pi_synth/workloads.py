@@ -2,7 +2,7 @@
 
 Each workload is a stack of ReLU or ReGLU FFN layers shaped like a real model, with
 power-law neuron firing probabilities (the locality both PowerInfer pages describe:
-GeekNews digest "PowerInfer" §"PowerInfer'in çözmeye çalıştığı sorun", and unite.ai
+GeekNews "Tüketici sınıfı GPU takılı PC'lerde yüksek hızlı büyük dil modeli serving" §"PowerInfer'in çözmeye çalıştığı sorun", and unite.ai
 "PowerInfer: Mesin Inferensi LLM Cepat dengan GPU Konsumen", introduction).  The
 datasets and trained checkpoints the pages profile are not available; these
 synthetic layers stand in for them.

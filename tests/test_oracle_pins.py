@@ -150,7 +150,8 @@ def test_batch_masks_apply_per_token():
 @pytest.mark.parametrize("act", ["relu", "reglu"])
 def test_sparse_equals_dense_with_true_mask(act):
     """Skipped neurons contribute exact zeros, so with the true mask the sparse FFN
-    is bit-identical to the dense one (unite.ai PowerInfer page, §"Fase Online":
+    is bit-identical to the dense one (unite.ai "PowerInfer: Mesin Inferensi LLM Cepat dengan GPU Konsumen",
+    §"Fase Online: Mesin Inferensi LLM yang Sadar Neuron":
     inactive neurons are skipped)."""
     rng = np.random.default_rng(7)
     d, f = 48, 256
