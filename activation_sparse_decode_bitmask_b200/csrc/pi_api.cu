@@ -115,7 +115,7 @@ pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedPara
   if (p.rec_window < 1) return PI_ERR_UNSUPPORTED;
   smem = fixed + (size_t)p.ring_bytes;
   // ws fields
-  p.ux = ws->ux; p.px = ws->px; p.vx = ws->vx; p.sx = ws->sx;
+  p.ux = ws->ux; p.px = ws->px; p.vx = ws->vx; p.sx = ws->sx; p.cx = ws->cx; p.lx = ws->lx;
   p.bar = ws->bar; p.err = ws->err; p.active_total = ws->active_total;
   p.layer_count = nullptr;
   p.barrier_timeout_ns = kDefaultWaitNs;
@@ -191,7 +191,20 @@ pi_status decode_stack_batched(pi_layer* const* layers, int Lc, void* x_inout, i
   return PI_OK;
 }
 
-LayerDev dev_view(const pi_layer* L, int B = 0) { return LayerDev{L->rec, L->p1t, L->p2o, B > 0 ? hot_len(L, B) : 0, 0}; }
+// Half the expected active records per block at batch B (from the firing frequencies of
+// the reorder): every block keeps that many of its own before balancing, so their
+// records can be fetched while the balancing exchange runs.
+void set_keep_floor(pi_layer* L) {
+  for (int B = 1; B <= 4; ++B) {
+    double expect = 0.0;
+    for (int i = 0; i < L->desc.d_ff; ++i) expect += 1.0 - std::pow(1.0 - (double)L->freq_host[i], (double)B);
+    L->keep_floor[B - 1] = (int)(0.5 * expect / L->G);
+  }
+}
+
+LayerDev dev_view(const pi_layer* L, int B = 0) {
+  return LayerDev{L->rec, L->p1t, L->p2o, B > 0 ? hot_len(L, B) : 0, B > 0 ? L->keep_floor[std::min(B, 4) - 1] : 0};
+}
 
 bool same_desc(const pi_layer_desc& a, const pi_layer_desc& b) {
   return a.d_model == b.d_model && a.d_ff == b.d_ff && a.rank == b.rank && a.act == b.act &&
@@ -362,6 +375,7 @@ pi_status pi_reorder_hot_prefix(pi_layer* L, const float* freq, int hot_count, c
   if (fh && cudaMemcpy(fh, L->freq_sorted, (size_t)F * 4, cudaMemcpyDeviceToHost) == cudaSuccess) {
     delete[] L->freq_host;
     L->freq_host = fh;
+    set_keep_floor(L);
   } else {
     delete[] fh;
   }
@@ -389,6 +403,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
             dmalloc(&ws->px, G * Bm * d_max * 8) == cudaSuccess &&
             dmalloc(&ws->vx, Bm * d_max * 8) == cudaSuccess &&
             dmalloc(&ws->sx, Bm * G * 16) == cudaSuccess &&
+            dmalloc(&ws->cx, G * 8) == cudaSuccess && dmalloc(&ws->lx, G * kMaxOwn * 8) == cudaSuccess &&
             dmalloc(&ws->bar, 64) == cudaSuccess &&
             dmalloc(&ws->err, 16) == cudaSuccess &&
             dmalloc(&ws->active_total, 16) == cudaSuccess &&
@@ -408,6 +423,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
     const uint32_t bar0[4] = {0u, 0u, 1u, 0u};
     ok = cudaMemset(ws->ux, 0, Bm * r_max * 8) == cudaSuccess && cudaMemset(ws->px, 0, G * Bm * d_max * 8) == cudaSuccess &&
          cudaMemset(ws->vx, 0, Bm * d_max * 8) == cudaSuccess && cudaMemset(ws->sx, 0, Bm * G * 16) == cudaSuccess &&
+         cudaMemset(ws->cx, 0, G * 8) == cudaSuccess && cudaMemset(ws->lx, 0, G * kMaxOwn * 8) == cudaSuccess &&
          cudaMemset(ws->bar, 0, 64) == cudaSuccess &&
          cudaMemcpy(ws->bar, bar0, sizeof(bar0), cudaMemcpyHostToDevice) == cudaSuccess &&
          cudaMemset(ws->err, 0, 16) == cudaSuccess && cudaMemset(ws->active_total, 0, 16) == cudaSuccess &&
@@ -424,7 +440,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
 
 void pi_workspace_free(pi_workspace* ws) {
   if (!ws) return;
-  cudaFree(ws->ux); cudaFree(ws->px); cudaFree(ws->vx); cudaFree(ws->sx);
+  cudaFree(ws->ux); cudaFree(ws->px); cudaFree(ws->vx); cudaFree(ws->sx); cudaFree(ws->cx); cudaFree(ws->lx);
   cudaFree(ws->bar); cudaFree(ws->err); cudaFree(ws->active_total);
   cudaFree(ws->layer_count); cudaFree(ws->x_dev); cudaFree(ws->phase_clk);
   cudaFree(ws->u_hi); cudaFree(ws->u_lo); cudaFree(ws->bmask); cudaFree(ws->bidx); cudaFree(ws->bcount);

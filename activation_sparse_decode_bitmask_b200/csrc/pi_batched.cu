@@ -27,10 +27,15 @@ namespace {
 
 constexpr int kBW = 4;                    // warps per block
 constexpr int kRows = 16 * kBW;           // rows (or columns) per block
-constexpr int kKC = 64;                   // K elements staged per chunk
+constexpr int kKC = 128;                  // K elements staged per chunk (256 bytes of each row)
 constexpr int kPad = kKC * 2 + 16;        // bytes per staged row: the 16-byte pad keeps ldmatrix conflict-free
 constexpr int kMaxKSplit = 32;            // K splits of a row kernel at most
 constexpr int kMaxDownSplit = 16;         // neuron splits of the down kernel at most
+constexpr int kDM = 2;                    // 16-column tiles per warp in the down kernel
+constexpr int kDCols = 16 * kDM * kBW;    // columns per down block
+constexpr int kDN = 64;                   // neurons staged per down chunk
+constexpr int kDPad = kDCols * 2 + 16;    // bytes per staged down row slice
+constexpr int kHPad = kDN * 2 + 16;       // bytes per staged token row of h
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -123,16 +128,21 @@ __global__ void __launch_bounds__(32 * kBW) rowtok_kernel(const RowTokArgs a) {
     }
     return a.base + (size_t)i * a.stride + (m == 0 ? a.up_off : a.gate_off);
   };
+  // the block's row addresses, once: the same rows stream through every K chunk
+  __shared__ const uint8_t* rowp[NMAT][kRows];
+  for (int e = t; e < NMAT * kRows; e += 32 * kBW) rowp[e / kRows][e % kRows] = row_ptr(row0 + e % kRows, e / kRows);
+  __syncthreads();
   const uint32_t base_u = smem_u32(smem);
   auto stage_chunk = [&](int ch, int buf) {
     const int k0 = ch * kKC;
     const uint32_t rows_u = base_u + (uint32_t)(buf * STAGE_B), tok_u = rows_u + ROWS_B;
-    for (int e = t; e < NMAT * kRows * 8; e += 32 * kBW) {
-      const int m = e / (kRows * 8), rr = (e / 8) % kRows, pc = e % 8;
-      cp_async16(rows_u + (uint32_t)((m * kRows + rr) * kPad + pc * 16), row_ptr(row0 + rr, m) + (size_t)k0 * 2 + pc * 16);
+    constexpr int PC = kKC * 2 / 16;   // 16-byte pieces per staged row
+    for (int e = t; e < NMAT * kRows * PC; e += 32 * kBW) {
+      const int m = e / (kRows * PC), rr = (e / PC) % kRows, pc = e % PC;
+      cp_async16(rows_u + (uint32_t)((m * kRows + rr) * kPad + pc * 16), rowp[m][rr] + (size_t)k0 * 2 + pc * 16);
     }
-    for (int e = t; e < NS * BP * 8; e += 32 * kBW) {
-      const int s = e / (BP * 8), b = (e / 8) % BP, pc = e % 8;
+    for (int e = t; e < NS * BP * PC; e += 32 * kBW) {
+      const int s = e / (BP * PC), b = (e / PC) % BP, pc = e % PC;
       const __half* src = (s == 0 ? a.tok : a.tok_lo) + (size_t)min(b, a.B - 1) * a.K + k0 + pc * 8;
       cp_async16(tok_u + (uint32_t)((s * BP + b) * kPad + pc * 16), src);
     }
@@ -276,31 +286,34 @@ template <int NT>
 __global__ void __launch_bounds__(32 * kBW) down_kernel(const DownArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int BP = NT * 8;
-  constexpr int W_B = kRows * kPad, STAGE_B = W_B + 2 * BP * kPad;   // weights, then h hi / lo [2][BP]
+  constexpr int W_B = kDN * kDPad, STAGE_B = W_B + 2 * BP * kHPad;   // weights, then h hi / lo [2][BP]
   int count = *a.count;
   if (count < 0 || count > a.fmax) count = 0;   // reported by the gate/up kernel; y becomes 0
-  const int nch = (count + kRows - 1) / kRows;
+  const int nch = (count + kDN - 1) / kDN;
   const int c_begin = (int)((long long)blockIdx.y * nch / a.nsplit);
   const int c_end = (int)((long long)(blockIdx.y + 1) * nch / a.nsplit);
-  const int c0 = blockIdx.x * kRows;
+  const int c0 = blockIdx.x * kDCols;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const uint32_t base_u = smem_u32(smem);
   auto stage_w = [&](int ch, int buf) {
-    const int j0 = ch * kRows;
+    const int j0 = ch * kDN;
+    constexpr int PC = kDCols * 2 / 16;   // 16-byte pieces of a row slice
     const uint32_t w_u = base_u + (uint32_t)(buf * STAGE_B);
-    for (int e = t; e < kRows * 8; e += 32 * kBW) {
-      const int jj = e / 8, pc = e % 8;
+    for (int e = t; e < kDN * PC; e += 32 * kBW) {
+      const int jj = e / PC, pc = e % PC;
       int i = __ldg(a.idx + min(j0 + jj, count - 1));
       if (i < 0 || i >= a.fmax) i = 0;   // reported by the gate/up kernel
-      cp_async16(w_u + (uint32_t)(jj * kPad + pc * 16),
+      cp_async16(w_u + (uint32_t)(jj * kDPad + pc * 16),
                  a.rec + (size_t)i * a.rec_stride + a.down_off + (size_t)c0 * 2 + pc * 16);
     }
   };
-  float c[NT][4];
+  float c[kDM][NT][4];
 #pragma unroll
-  for (int n = 0; n < NT; ++n)
+  for (int mt = 0; mt < kDM; ++mt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) c[n][e] = 0.f;
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) c[mt][n][e] = 0.f;
 #pragma unroll
   for (int s = 0; s < kStages - 1; ++s) {
     if (c_begin + s < c_end) stage_w(c_begin + s, s);
@@ -311,50 +324,57 @@ __global__ void __launch_bounds__(32 * kBW) down_kernel(const DownArgs a) {
     const uint32_t w_u = base_u + (uint32_t)(buf * STAGE_B), h_u = w_u + W_B;
     // h of the chunk, split into fp16 hi / lo (neurons past count contribute zero); this
     // buffer's previous readers finished before the last barrier
-    const int j0 = ch * kRows;
-    for (int e = t; e < BP * kRows; e += 32 * kBW) {
-      const int b = e / kRows, jj = e % kRows;
+    const int j0 = ch * kDN;
+    for (int e = t; e < BP * kDN; e += 32 * kBW) {
+      const int b = e / kDN, jj = e % kDN;
       const float v = (j0 + jj < count && b < a.B) ? a.h[(size_t)(j0 + jj) * 32 + b] : 0.f;
       __half hi, lo;
       split_h(v, hi, lo);
-      reinterpret_cast<__half*>(smem + buf * STAGE_B + W_B + (size_t)b * kPad)[jj] = hi;
-      reinterpret_cast<__half*>(smem + buf * STAGE_B + W_B + (size_t)(BP + b) * kPad)[jj] = lo;
+      reinterpret_cast<__half*>(smem + buf * STAGE_B + W_B + (size_t)b * kHPad)[jj] = hi;
+      reinterpret_cast<__half*>(smem + buf * STAGE_B + W_B + (size_t)(BP + b) * kHPad)[jj] = lo;
     }
     cp_async_wait_1();
     __syncthreads();   // weights and h of chunk ch are in place; chunk ch - 1's buffer is free
     if (ch + kStages - 1 < c_end) stage_w(ch + kStages - 1, (ch + kStages - 1 - c_begin) % kStages);
     cp_async_commit();
 #pragma unroll
-    for (int ks = 0; ks < kRows / 16; ++ks) {
-      uint32_t af[4];
-      {
-        const int jj = ks * 16 + (lane & 7) + 8 * (lane >> 4);   // neuron (K) of this lane's row address
-        const int cc = warp * 16 + 8 * ((lane >> 3) & 1);        // column (M) offset
-        ldsm_x4_t(w_u + (uint32_t)(jj * kPad + cc * 2), af);
-      }
+    for (int ks = 0; ks < kDN / 16; ++ks) {
+      uint32_t bf[NT][2][2];
 #pragma unroll
       for (int n = 0; n < NT; ++n)
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
-          uint32_t bf[2];
           const int b = n * 8 + (lane & 7);
           const int jj = ks * 16 + 8 * ((lane >> 3) & 1);
-          ldsm_x2(h_u + (uint32_t)((s * BP + b) * kPad + jj * 2), bf);
-          mma16816(c[n], af, bf);
+          ldsm_x2(h_u + (uint32_t)((s * BP + b) * kHPad + jj * 2), bf[n][s]);
         }
+#pragma unroll
+      for (int mt = 0; mt < kDM; ++mt) {
+        uint32_t af[4];
+        const int jj = ks * 16 + (lane & 7) + 8 * (lane >> 4);                 // neuron (K) of this lane's row address
+        const int cc = (warp * kDM + mt) * 16 + 8 * ((lane >> 3) & 1);       // column (M) offset
+        ldsm_x4_t(w_u + (uint32_t)(jj * kDPad + cc * 2), af);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          mma16816(c[mt][n], af, bf[n][0]);
+          mma16816(c[mt][n], af, bf[n][1]);
+        }
+      }
     }
     __syncthreads();   // every thread is done with this buffer before its h is rewritten
   }
   cp_async_wait_all();
   const int g = lane >> 2, tq = lane & 3;
 #pragma unroll
-  for (int n = 0; n < NT; ++n)
+  for (int mt = 0; mt < kDM; ++mt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int col = c0 + warp * 16 + g + 8 * (e >> 1);
-      const int b = n * 8 + 2 * tq + (e & 1);
-      if (b < a.B && col < a.d) a.ypart[((size_t)blockIdx.y * a.B + b) * a.d + col] = c[n][e];
-    }
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int col = c0 + (warp * kDM + mt) * 16 + g + 8 * (e >> 1);
+        const int b = n * 8 + 2 * tq + (e & 1);
+        if (b < a.B && col < a.d) a.ypart[((size_t)blockIdx.y * a.B + b) * a.d + col] = c[mt][n][e];
+      }
 }
 
 __global__ void __launch_bounds__(256) down_reduce(const float* ypart, int nsplit, int n, float* y) {
@@ -407,24 +427,36 @@ int ksplit_for(int row_blocks, int nch) {
   return max(1, min(s, kMaxKSplit));
 }
 
+// Raise a kernel's dynamic shared memory limit once (per kernel, per size increase), so
+// the hot launch sequence makes no extra driver calls.
+template <typename K>
+cudaError_t smem_attr_once(K kern, size_t smem, int& configured) {
+  if ((int)smem <= configured) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) configured = (int)smem;
+  return e;
+}
+
 template <int NT>
 cudaError_t launch_rowtok_nt(const RowTokArgs& a, int nmat, int blocks, cudaStream_t s) {
   const bool split = a.tok_lo != nullptr;
   const int ns = split ? 2 : 1;
   const size_t smem = (size_t)kStages * ((size_t)nmat * kRows * kPad + (size_t)ns * NT * 8 * kPad);
   const dim3 grid(blocks, a.ksplit);
+  static int conf2 = 0, conf_split = 0, conf1 = 0;
+  cudaError_t e;
   if (nmat == 2) {
     if (split) return cudaErrorNotSupported;
     auto k = rowtok_kernel<NT, 2, false>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if ((e = smem_attr_once(k, smem, conf2)) != cudaSuccess) return e;
     k<<<grid, 32 * kBW, smem, s>>>(a);
   } else if (split) {
     auto k = rowtok_kernel<NT, 1, true>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if ((e = smem_attr_once(k, smem, conf_split)) != cudaSuccess) return e;
     k<<<grid, 32 * kBW, smem, s>>>(a);
   } else {
     auto k = rowtok_kernel<NT, 1, false>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if ((e = smem_attr_once(k, smem, conf1)) != cudaSuccess) return e;
     k<<<grid, 32 * kBW, smem, s>>>(a);
   }
   return cudaGetLastError();
@@ -457,17 +489,19 @@ cudaError_t launch_rows(RowTokArgs a, RowEpiArgs ep, int nmat, int rows_max, siz
 
 template <int NT>
 cudaError_t launch_down_nt(const DownArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)kStages * ((size_t)kRows * kPad + 2 * (size_t)NT * 8 * kPad);
+  const size_t smem = (size_t)kStages * ((size_t)kDN * kDPad + 2 * (size_t)NT * 8 * kHPad);
   auto k = down_kernel<NT>;
-  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  k<<<dim3((a.d + kRows - 1) / kRows, a.nsplit), 32 * kBW, smem, s>>>(a);
+  static int conf = 0;
+  const cudaError_t e = smem_attr_once(k, smem, conf);
+  if (e != cudaSuccess) return e;
+  k<<<dim3((a.d + kDCols - 1) / kDCols, a.nsplit), 32 * kBW, smem, s>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool batched_supported(int family, int B, int d, int r) {
-  return family == FAM_F16 && B >= 1 && B <= 32 && d % kKC == 0 && r % kKC == 0 && d % kRows == 0;
+  return family == FAM_F16 && B >= 1 && B <= 32 && d % kKC == 0 && r % kKC == 0 && d % kDCols == 0;
 }
 
 cudaError_t batched_predict(const BatchedLayer& L, const void* x, int B, uint32_t* mask, float* logits,
@@ -554,7 +588,7 @@ cudaError_t batched_ffn(const BatchedLayer& L, const void* x, int B, const uint3
   dn.idx = idx;
   dn.h = h;
   dn.ypart = ypart;
-  const int col_blocks = (L.d + kRows - 1) / kRows;
+  const int col_blocks = (L.d + kDCols - 1) / kDCols;
   dn.nsplit = std::min(kMaxDownSplit, std::max(1, (4 * 148 + col_blocks - 1) / col_blocks));
   switch ((B + 7) / 8) {
     case 1: e = launch_down_nt<1>(dn, s); break;

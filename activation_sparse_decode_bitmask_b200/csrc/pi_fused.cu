@@ -47,9 +47,11 @@ constexpr int kItems = 32;          // ring items in flight (mbarrier pairs)
 struct Smem {
   uint64_t full[kItems];
   uint64_t empty[kItems];
-  uint64_t list_ready;
+  uint64_t list_ready;          // the first part of the block's list is in place
+  uint64_t list2_ready;         // the whole list is in place
   uint64_t layer_start;
   int abort_flag;
+  int nlist_a;                  // records of the first part of the list
   int nlist;
   int count;                   // active neurons of the layer (union over tokens)
   int pad;
@@ -63,6 +65,9 @@ struct Smem {
   int32_t list[kMaxList];
   uint8_t list_bits[kMaxList];
   uint8_t own_bits[kMaxOwn];
+  int32_t cnt[kMaxGrid];        // every block's own active count (balance)
+  int32_t xpre[kMaxGrid + 1];   // exclusive prefix of the blocks' excess over the target
+  int32_t bal[4];               // target, this block's deficit start, total excess
 };
 
 // Diagnostics: SM cycle stamps at phase boundaries, [block][layer][kPhases].
@@ -285,6 +290,81 @@ __device__ __forceinline__ float window_dots(uint32_t base, const uint32_t (&pos
   return reduce_scatter<V>(v, lane);
 }
 
+// Balance the active records across blocks.  Every block publishes its own active count
+// and its list entries (id | token bits << 24).  After reading all counts, every block
+// derives the same assignment from them alone: target T = max(ceil(N / G), floor); a
+// block keeps its first min(n_c, T) own records; the records past T of the blocks above
+// the target, in (block, position) order, fill the blocks below it in block order.  So
+// every block ends with T or fewer records and the assignment is a function of the data
+// and the layer's floor only.  A block's first min(n_c, floor) records are its own in
+// any case, so they are fetched while this runs.  Returns the block's new list length;
+// the taken records follow its own in sm.list.
+__device__ __forceinline__ int balance_list(int n_own, int floor, uint32_t tag_c, Smem& sm, const FusedParams& p, int c,
+                                            int G, int t, int warp, int lane) {
+  if (t < n_own) st_tag(p.lx + (size_t)c * kMaxOwn + t, __uint_as_float((uint32_t)sm.list[t] | ((uint32_t)sm.list_bits[t] << 24)), tag_c);
+  if (t == 0) st_tag(p.cx + c, __int_as_float(n_own), tag_c);
+  {
+    uint64_t w[1];
+    poll_words<1>(p.cx, t, kConsumerThreads, G, tag_c, w, sm, p);
+    if (t < G) sm.cnt[t] = __float_as_int(tag_val(w[0]));
+  }
+  named_bar_sync(kRedBar, kConsumerThreads);
+  if (warp == 0) {
+    int n = 0;
+    for (int o = lane; o < G; o += 32) n += sm.cnt[o];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    const int T = max((n + G - 1) / G, floor);
+    // exclusive prefix of the excess max(0, n_o - T), and this block's deficit start
+    int carry = 0, dstart = 0;
+    for (int o0 = 0; o0 < G; o0 += 32) {
+      const int o = o0 + lane;
+      const int ex = (o < G) ? max(0, sm.cnt[o] - T) : 0;
+      const int de = (o < G && o < c) ? max(0, T - sm.cnt[o]) : 0;
+      int incl = ex;
+#pragma unroll
+      for (int k = 1; k < 32; k <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, k);
+        if (lane >= k) incl += v;
+      }
+      if (o < G) sm.xpre[o] = carry + incl - ex;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+      int ds = de;
+#pragma unroll
+      for (int k = 16; k > 0; k >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, k);
+      dstart += ds;
+    }
+    if (lane == 0) {
+      sm.xpre[G] = carry;
+      sm.bal[0] = T;
+      sm.bal[1] = dstart;
+      sm.bal[2] = carry;
+    }
+  }
+  named_bar_sync(kRedBar, kConsumerThreads);
+  const int T = sm.bal[0], dstart = sm.bal[1], xtotal = sm.bal[2];
+  const int keep = min(n_own, T);
+  const int deficit = max(0, T - n_own);
+  const int ntake = max(0, min(dstart + deficit, xtotal) - dstart);
+  if (t < ntake) {
+    const int x = dstart + t;
+    int lo = 0, hi = G;   // owner o: xpre[o] <= x < xpre[o + 1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (sm.xpre[mid] <= x) lo = mid;
+      else hi = mid;
+    }
+    const int k = T + (x - sm.xpre[lo]);
+    uint64_t w[1];
+    poll_words<1>(p.lx + (size_t)lo * kMaxOwn + k, 0, 1, 1, tag_c, w, sm, p);
+    const uint32_t v = (uint32_t)w[0];
+    sm.list[keep + t] = (int32_t)(v & 0xFFFFFFu);
+    sm.list_bits[keep + t] = (uint8_t)(v >> 24);
+  }
+  named_bar_sync(kRedBar, kConsumerThreads);
+  return keep + ntake;
+}
+
 // ------------------------------------------------------------------ the kernel
 template <int FAM, int ACT, int NB, int NU>
 __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p) {
@@ -315,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       mbar_init(&sm.empty[s], kConsumerWarps);
     }
     mbar_init(&sm.list_ready, 1);
+    mbar_init(&sm.list2_ready, 1);
     mbar_init(&sm.layer_start, 1);
     sm.abort_flag = 0;
     sm.nlist = 0;
@@ -399,12 +480,28 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
             if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
           }
           pstamp(p, l, 10);
-          const int n = ok ? sm.nlist : 0;
-          // Ask HBM for every record of the block at once (L2 prefetch needs no shared
-          // memory); the ring copies below then find them in L2 as space frees up.
-          for (int e = 0; e < n && ok; ++e)
+          // Ask HBM for every record at once (L2 prefetch needs no shared memory); the
+          // ring copies then find them in L2 as space frees up.  The first part of the
+          // list is known before the balancing exchange ends, the rest after it.
+          const int na = ok ? sm.nlist_a : 0;
+          for (int e = 0; e < na && ok; ++e)
             prefetch_l2_bulk(Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride);
-          for (int e = 0; e < n && ok; ++e) {
+          int e = 0;
+          for (; e < na && ok; ++e) {
+            if (!(ok = begin_item((uint32_t)p.rec_stride, dst, fb))) break;
+            bulk_g2s(dst, Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride, fb);
+          }
+          if (ok) {
+            const uint64_t t0 = wait_start();
+            while (!mbar_try_wait(&sm.list2_ready, (uint32_t)(l & 1))) {
+              if (aborted(sm)) { ok = false; break; }
+              if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
+            }
+          }
+          const int n = ok ? sm.nlist : 0;
+          for (int q = na; q < n && ok; ++q)
+            prefetch_l2_bulk(Ld.rec + (size_t)sm.list[q] * p.rec_stride, (uint32_t)p.rec_stride);
+          for (; e < n && ok; ++e) {
             if (!(ok = begin_item((uint32_t)p.rec_stride, dst, fb))) break;
             bulk_g2s(dst, Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride, fb);
           }
@@ -456,8 +553,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
 
   int redbuf = 0;   // which half of sm.red the next block reduction uses
   for (int l = 0; l < p.L; ++l) {
-    const uint32_t tag_u = tag_of(epoch, l, 0), tag_p = tag_of(epoch, l, 1), tag_v = tag_of(epoch, l, 2);
+    const uint32_t tag_u = tag_of(epoch, l, 0), tag_p = tag_of(epoch, l, 1), tag_v = tag_of(epoch, l, 2),
+                   tag_c = tag_of(epoch, l, 3);
     int nlist = 0;
+    bool signaled_a = false;   // the first part of the list was handed over already
     stamp(p, l, 0);
     // this layer's x units, fp32, in registers for P-a and F
     uint32_t xr[NU][NB][XW];
@@ -646,6 +745,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         if (p.layer_count) atomicAdd(p.layer_count + l, nlist);
       }
       stamp(p, l, 15);
+      if (do_ffn && p.cx) {
+        // the first part (own records every block keeps) goes to the producer now
+        const int floor = p.layers[l].keep_floor;
+        if (t == 0) {
+          sm.nlist_a = min(nlist, floor);
+          mbar_arrive(&sm.list_ready);
+        }
+        signaled_a = true;
+        nlist = balance_list(nlist, floor, tag_c, sm, p, c, G, t, warp, lane);
+      }
       stamp_val(p, l, 14, nlist);
     } else if (do_ffn) {
       // ---------------------------------------------------------- list from the caller
@@ -674,8 +783,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     if (!do_ffn) break;   // predictor only
     named_bar_sync(kRedBar, kConsumerThreads);
     if (t == 0) {
+      if (!signaled_a) {
+        sm.nlist_a = nlist;
+        mbar_arrive(&sm.list_ready);
+      }
       sm.nlist = nlist;
-      mbar_arrive(&sm.list_ready);
+      mbar_arrive(&sm.list2_ready);
     }
     stamp(p, l, 3);
 

@@ -37,8 +37,8 @@ struct LayerDev {
   const uint8_t* rec;     // [f][rec_stride]   per-neuron record [gate][up][down]
   const uint8_t* p1t;     // [r][p1_row]       P1 transposed, p_dtype
   const uint8_t* p2o;     // [G][nown_max][p2_stride] predictor row + (t, b) of neuron c + m*G
-  int hot;                // hot-prefix length at this call's batch (L2 warm-up), 0 = none
-  int pad;
+  int hot;                // hot-prefix length at this call's batch, 0 = none
+  int keep_floor;         // records every block keeps of its own before balancing (0 = none)
 };
 
 }  // namespace pi
@@ -62,6 +62,7 @@ struct pi_layer {
   int32_t* perm;    // [f] stored position -> original id
   float* freq_sorted;  // [f] firing frequency in stored order (after a reorder), else null
   float* freq_host;    // host copy of freq_sorted (descending), or null
+  int keep_floor[4];   // per batch 1..4: own records every block keeps before balancing
   int hot_count;    // -1: derived per batch from freq_sorted
   int device;
 };
@@ -74,6 +75,8 @@ struct pi_workspace {
   uint64_t* px;      // [grid][B_max][d_max]    tagged y partials
   uint64_t* vx;      // [B_max][d_max]          tagged x + y
   uint64_t* sx;      // [B_max][grid][2]        tagged slice sums and sums of squares
+  uint64_t* cx;      // [grid]                  tagged own active counts (balance)
+  uint64_t* lx;      // [grid][kMaxOwn]         tagged own active list entries (balance)
   uint32_t* bar;     // [0] probe barrier count, [1] exit count, [2] launch epoch (tags)
   int* err;          // device error word
   unsigned long long* active_total;  // running sum of active-list lengths (all calls)
@@ -122,6 +125,8 @@ struct FusedParams {
   uint64_t* px;
   uint64_t* vx;
   uint64_t* sx;
+  uint64_t* cx;        // tagged own active counts [grid]; null: no balancing (each block keeps its own)
+  uint64_t* lx;        // tagged own active list entries [grid][kMaxOwn]
   uint32_t* bar;
   int* err;
   unsigned long long* active_total;
