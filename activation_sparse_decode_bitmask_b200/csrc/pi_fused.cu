@@ -43,6 +43,7 @@ constexpr float kRmsEps = 1e-6f;
 constexpr int kRedBar = 1;          // named barrier id among consumers
 constexpr int kMaxColGroups = 4;    // 32-column groups per reduce slice
 constexpr int kItems = 32;          // ring items in flight (mbarrier pairs)
+constexpr int kBalK = 12;           // list entries every block publishes at least (balance)
 
 struct Smem {
   uint64_t full[kItems];
@@ -66,6 +67,7 @@ struct Smem {
   uint8_t list_bits[kMaxList];
   uint8_t own_bits[kMaxOwn];
   int32_t cnt[kMaxGrid];        // every block's own active count (balance)
+  uint32_t bsnap[kMaxGrid * 12];   // every block's first list entries (balance), kBalK per block
   int32_t xpre[kMaxGrid + 1];   // exclusive prefix of the blocks' excess over the target
   int32_t bal[4];               // target, this block's deficit start, total excess
 };
@@ -301,12 +303,47 @@ __device__ __forceinline__ float window_dots(uint32_t base, const uint32_t (&pos
 // the taken records follow its own in sm.list.
 __device__ __forceinline__ int balance_list(int n_own, int floor, uint32_t tag_c, Smem& sm, const FusedParams& p, int c,
                                             int G, int t, int warp, int lane) {
-  if (t < n_own) st_tag(p.lx + (size_t)c * kMaxOwn + t, __uint_as_float((uint32_t)sm.list[t] | ((uint32_t)sm.list_bits[t] << 24)), tag_c);
+  // publish the count and at least kBalK entries (padded), so that one polling round can
+  // read every count and every block's first kBalK entries
+  if (t < max(n_own, kBalK))
+    st_tag(p.lx + (size_t)c * kMaxOwn + t,
+           __uint_as_float(t < n_own ? ((uint32_t)sm.list[t] | ((uint32_t)sm.list_bits[t] << 24)) : 0u), tag_c);
   if (t == 0) st_tag(p.cx + c, __int_as_float(n_own), tag_c);
   {
-    uint64_t w[1];
-    poll_words<1>(p.cx, t, kConsumerThreads, G, tag_c, w, sm, p);
-    if (t < G) sm.cnt[t] = __float_as_int(tag_val(w[0]));
+    // chunks of 4 words per thread: one round for up to 2048 words (157 blocks)
+    constexpr int MQ = 4;
+    const int nq = G * (1 + kBalK);
+    for (int base = 0; base < nq; base += MQ * kConsumerThreads) {
+      uint64_t w[MQ];
+      uint32_t need = 0;
+#pragma unroll
+      for (int i = 0; i < MQ; ++i) {
+        w[i] = 0;
+        if (base + t + i * kConsumerThreads < nq) need |= 1u << i;
+      }
+      bool started = false;
+      uint64_t tp = 0;
+      while (need) {
+#pragma unroll
+        for (int i = 0; i < MQ; ++i)
+          if (need >> i & 1u) {
+            const int q = base + t + i * kConsumerThreads;
+            const uint64_t* src = (q < G) ? p.cx + q : p.lx + (size_t)((q - G) / kBalK) * kMaxOwn + (q - G) % kBalK;
+            w[i] = ld_tag(src);
+            if (tag_ok(w[i], tag_c)) need &= ~(1u << i);
+          }
+        if (!need || aborted(sm)) break;
+        if (!started) { tp = wait_start(); started = true; }
+        else if (timed_out(tp, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+        if (p.poll_ns) __nanosleep(p.poll_ns);
+      }
+#pragma unroll
+      for (int i = 0; i < MQ; ++i) {
+        const int q = base + t + i * kConsumerThreads;
+        if (q < G) sm.cnt[q] = __float_as_int(tag_val(w[i]));
+        else if (q < nq) sm.bsnap[q - G] = (uint32_t)w[i];
+      }
+    }
   }
   named_bar_sync(kRedBar, kConsumerThreads);
   if (warp == 0) {
@@ -355,9 +392,14 @@ __device__ __forceinline__ int balance_list(int n_own, int floor, uint32_t tag_c
       else hi = mid;
     }
     const int k = T + (x - sm.xpre[lo]);
-    uint64_t w[1];
-    poll_words<1>(p.lx + (size_t)lo * kMaxOwn + k, 0, 1, 1, tag_c, w, sm, p);
-    const uint32_t v = (uint32_t)w[0];
+    uint32_t v;
+    if (k < kBalK) {
+      v = sm.bsnap[lo * kBalK + k];
+    } else {   // past the snapshot (a block far above the target): read it now
+      uint64_t w[1];
+      poll_words<1>(p.lx + (size_t)lo * kMaxOwn + k, 0, 1, 1, tag_c, w, sm, p);
+      v = (uint32_t)w[0];
+    }
     sm.list[keep + t] = (int32_t)(v & 0xFFFFFFu);
     sm.list_bits[keep + t] = (uint8_t)(v >> 24);
   }
@@ -1018,22 +1060,65 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     if (!do_glue) break;
     stamp(p, l, 6);
 
-    // ------------------------------------------------------------ glue: x' = v / rms
+    // ------------------------------------------------------------ glue: x' = (v - mean) / sd
+    // One polling round reads both what the slice owners published: every thread polls its
+    // v pairs of the first chunk and a few of the slices' (sum, sum of squares) words.
     {
-      if (warp < NB) {
-        float s = 0.f;
-        float s2 = 0.f;
-        if (warp < B) {
-          // words (sum, sum of squares) of every slice, interleaved: even lanes read sums,
-          // odd lanes sums of squares (32 is even, so a lane keeps its parity)
-          uint64_t w[2 * kMaxGrid / 32];
-          poll_words<2 * kMaxGrid / 32>(p.sx + (size_t)warp * G * 2, lane, 32, 2 * nslices, tag_v, w, sm, p);
+      const int npairs = B * d / 2;
+      const int nmom = 2 * nslices * B;
+      constexpr int MQ = (2 * kMaxGrid * 4 + kConsumerThreads - 1) / kConsumerThreads;
+      uint64_t w0[8], w1[8], wm[MQ];
+      uint32_t need = 0, needm = 0;
 #pragma unroll
-          for (int k = 0; k < 2 * kMaxGrid / 32; ++k)
-            if (lane + 32 * k < 2 * nslices) s += tag_val(w[k]);
+      for (int k = 0; k < 8; ++k) {
+        w0[k] = w1[k] = 0;
+        if (t + k * kConsumerThreads < npairs) need |= 1u << k;
+      }
+#pragma unroll
+      for (int i = 0; i < MQ; ++i) {
+        wm[i] = 0;
+        if (t + i * kConsumerThreads < nmom) needm |= 1u << i;
+      }
+      {
+        bool started = false;
+        uint64_t tp = 0;
+        while (need | needm) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (need >> k & 1u) {
+              ld_tag2(p.vx + 2 * (size_t)(t + k * kConsumerThreads), w0[k], w1[k]);
+              if (tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
+            }
+#pragma unroll
+          for (int i = 0; i < MQ; ++i)
+            if (needm >> i & 1u) {
+              const int q = t + i * kConsumerThreads;
+              const int bq = q / (2 * nslices), cq = (q >> 1) % nslices;
+              wm[i] = ld_tag(p.sx + ((size_t)bq * G + cq) * 2 + (q & 1));
+              if (tag_ok(wm[i], tag_v)) needm &= ~(1u << i);
+            }
+          if (!(need | needm) || aborted(sm)) break;
+          if (!started) { tp = wait_start(); started = true; }
+          else if (timed_out(tp, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+          if (p.poll_ns) __nanosleep(p.poll_ns);
         }
-        const float sum = warp_sum((lane & 1) ? 0.f : s);
-        s2 = warp_sum((lane & 1) ? s : 0.f);
+      }
+      named_bar_sync(kRedBar, kConsumerThreads);   // the slice reduce is done with red2; nobody reads xs
+      stamp(p, l, 16);
+      float* mom = red2;                            // [B][nslices][2]
+#pragma unroll
+      for (int i = 0; i < MQ; ++i)
+        if (t + i * kConsumerThreads < nmom) mom[t + i * kConsumerThreads] = tag_val(wm[i]);
+      named_bar_sync(kRedBar, kConsumerThreads);
+      if (warp < NB) {
+        float s = 0.f, s2 = 0.f;
+        if (warp < B)
+          for (int cq = lane; cq < nslices; cq += 32) {
+            s += mom[(warp * nslices + cq) * 2];
+            s2 += mom[(warp * nslices + cq) * 2 + 1];
+          }
+        const float sum = warp_sum(s);
+        s2 = warp_sum(s2);
         if (lane == 0) {
           const float mean = sum / (float)d;
           const float var = fmaxf(s2 / (float)d - mean * mean, 0.f);
@@ -1042,40 +1127,46 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         }
       }
       named_bar_sync(kRedBar, kConsumerThreads);
-      stamp(p, l, 16);   // rms known; every warp is done reading xs
-      {
-        const int npairs = B * d / 2;
-        for (int base = 0; base < npairs; base += 8 * kConsumerThreads) {
-          uint64_t w0[8], w1[8];
-          uint32_t need = 0;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            w0[k] = w1[k] = 0;
-            if (base + t + k * kConsumerThreads < npairs) need |= 1u << k;
-          }
-          bool started = false;
-          uint64_t tp = 0;
-          while (need) {
+      for (int k = 0; k < 8; ++k) {
+        const int pr = t + k * kConsumerThreads;
+        if (pr < npairs) {
+          const int idx = 2 * pr, b = idx / d;
+          const float mean = sm.gmean[b], sd = sm.gsd[b];
+          xs[idx] = XT(round_act<FAM>((tag_val(w0[k]) - mean) / sd));
+          xs[idx + 1] = XT(round_act<FAM>((tag_val(w1[k]) - mean) / sd));
+        }
+      }
+      // pairs past the first chunk (wide layers or several tokens): published already
+      for (int base = 8 * kConsumerThreads; base < npairs; base += 8 * kConsumerThreads) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              if (need >> k & 1u) {
-                ld_tag2(p.vx + 2 * (size_t)(base + t + k * kConsumerThreads), w0[k], w1[k]);
-                if (tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
-              }
-            if (!need || aborted(sm)) break;
-            if (!started) { tp = wait_start(); started = true; }
-            else if (timed_out(tp, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
-            if (p.poll_ns) __nanosleep(p.poll_ns);
-          }
+        for (int k = 0; k < 8; ++k) w0[k] = w1[k] = 0;
+        need = 0;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int pr = base + t + k * kConsumerThreads;
-            if (pr < npairs) {
-              const int idx = 2 * pr, b = idx / d;
-              const float mean = sm.gmean[b], sd = sm.gsd[b];
-              xs[idx] = XT(round_act<FAM>((tag_val(w0[k]) - mean) / sd));
-              xs[idx + 1] = XT(round_act<FAM>((tag_val(w1[k]) - mean) / sd));
+        for (int k = 0; k < 8; ++k)
+          if (base + t + k * kConsumerThreads < npairs) need |= 1u << k;
+        bool started = false;
+        uint64_t tp = 0;
+        while (need) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (need >> k & 1u) {
+              ld_tag2(p.vx + 2 * (size_t)(base + t + k * kConsumerThreads), w0[k], w1[k]);
+              if (tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
             }
+          if (!need || aborted(sm)) break;
+          if (!started) { tp = wait_start(); started = true; }
+          else if (timed_out(tp, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+          if (p.poll_ns) __nanosleep(p.poll_ns);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int pr = base + t + k * kConsumerThreads;
+          if (pr < npairs) {
+            const int idx = 2 * pr, b = idx / d;
+            const float mean = sm.gmean[b], sd = sm.gsd[b];
+            xs[idx] = XT(round_act<FAM>((tag_val(w0[k]) - mean) / sd));
+            xs[idx + 1] = XT(round_act<FAM>((tag_val(w1[k]) - mean) / sd));
           }
         }
       }
