@@ -191,14 +191,17 @@ pi_status decode_stack_batched(pi_layer* const* layers, int Lc, void* x_inout, i
   return PI_OK;
 }
 
-// Half the expected active records per block at batch B (from the firing frequencies of
-// the reorder): every block keeps that many of its own before balancing, so their
-// records can be fetched while the balancing exchange runs.
+// A share of the expected active records per block at batch B (from the firing
+// frequencies of the reorder): every block keeps that many of its own before balancing,
+// so their records can be fetched while the balancing exchange runs.  Below the balanced
+// target (the mean count) the floor does not change the assignment, so it sits just
+// under the expected mean.
+constexpr double kKeepShare = 0.85;
 void set_keep_floor(pi_layer* L) {
   for (int B = 1; B <= 4; ++B) {
     double expect = 0.0;
     for (int i = 0; i < L->desc.d_ff; ++i) expect += 1.0 - std::pow(1.0 - (double)L->freq_host[i], (double)B);
-    L->keep_floor[B - 1] = (int)(0.5 * expect / L->G);
+    L->keep_floor[B - 1] = (int)(kKeepShare * expect / L->G);
   }
 }
 

@@ -44,6 +44,7 @@ constexpr int kRedBar = 1;          // named barrier id among consumers
 constexpr int kMaxColGroups = 4;    // 32-column groups per reduce slice
 constexpr int kItems = 32;          // ring items in flight (mbarrier pairs)
 constexpr int kBalK = 12;           // list entries every block publishes at least (balance)
+constexpr uint32_t kSleepNs = 20000;  // suspend hint of blocking mbarrier waits (wakes on completion)
 
 struct Smem {
   uint64_t full[kItems];
@@ -206,7 +207,7 @@ __device__ __forceinline__ void ring_wait_item(uint32_t item, Smem& sm, const Fu
   const uint32_t par = (item / kItems) & 1u;
   if (!aborted(sm) && !mbar_try_wait(bar, par)) {
     const uint64_t t0 = wait_start();
-    while (!mbar_try_wait(bar, par)) {
+    while (!mbar_try_wait_sleep(bar, par, kSleepNs)) {
       if (aborted(sm)) break;
       if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); break; }
     }
@@ -466,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           const uint32_t par = (oldest / kItems) & 1u;
           if (!mbar_try_wait(eb, par)) {
             const uint64_t t0 = wait_start();
-            while (!mbar_try_wait(eb, par)) {
+            while (!mbar_try_wait_sleep(eb, par, kSleepNs)) {
               if (aborted(sm)) return false;
               if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); return false; }
             }
@@ -494,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         if (do_pred && p.gate_producer && l > 0) {
           // experiment: keep the producer quiet until the consumers start this layer
           const uint64_t t0 = wait_start();
-          while (!mbar_try_wait(&sm.layer_start, (uint32_t)(l & 1))) {
+          while (!mbar_try_wait_sleep(&sm.layer_start, (uint32_t)(l & 1), kSleepNs)) {
             if (aborted(sm)) { ok = false; break; }
             if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
           }
@@ -517,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         if (do_ffn && ok) {
           pstamp(p, l, 9);
           const uint64_t t0 = wait_start();
-          while (!mbar_try_wait(&sm.list_ready, (uint32_t)(l & 1))) {
+          while (!mbar_try_wait_sleep(&sm.list_ready, (uint32_t)(l & 1), kSleepNs)) {
             if (aborted(sm)) { ok = false; break; }
             if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
           }
@@ -535,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           }
           if (ok) {
             const uint64_t t0 = wait_start();
-            while (!mbar_try_wait(&sm.list2_ready, (uint32_t)(l & 1))) {
+            while (!mbar_try_wait_sleep(&sm.list2_ready, (uint32_t)(l & 1), kSleepNs)) {
               if (aborted(sm)) { ok = false; break; }
               if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
             }
@@ -556,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         uint64_t* fb = &sm.full[s % kItems];
         const uint32_t par = (s / kItems) & 1u;
         const uint64_t t0 = wait_start();
-        while (!mbar_try_wait(fb, par)) {
+        while (!mbar_try_wait_sleep(fb, par, kSleepNs)) {
           if (timed_out(t0, p.wait_cycles)) { atomicExch(p.err, DEV_ERR_RING_TIMEOUT); break; }
         }
       }

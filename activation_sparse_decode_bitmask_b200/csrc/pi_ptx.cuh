@@ -47,6 +47,19 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Blocking form for wait loops: the thread may be suspended until the phase completes or
+// about `hint_ns` pass, instead of spinning and taking issue slots from the warps that
+// share its scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* b, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
   uint32_t ok;
   asm volatile(
