@@ -71,6 +71,7 @@ struct Smem {
   uint32_t bsnap[kMaxGrid * 12];   // every block's first list entries (balance), kBalK per block
   int32_t xpre[kMaxGrid + 1];   // exclusive prefix of the blocks' excess over the target
   int32_t bal[4];               // target, this block's deficit start, total excess
+  int32_t wsum[3][kConsumerWarps];   // per-warp partials of the balance's block scans
 };
 
 // Diagnostics: SM cycle stamps at phase boundaries, [block][layer][kPhases].
@@ -166,12 +167,14 @@ __device__ __forceinline__ void poll_words(const uint64_t* base, int first, int 
   uint64_t t0 = 0;
   bool started = false;
   while (need) {
+    // every load of the round is issued before any tag is looked at, so the round costs
+    // one L2 round trip whatever the number of words
 #pragma unroll
     for (int k = 0; k < MAXK; ++k)
-      if (need >> k & 1u) {
-        w[k] = ld_tag(base + first + k * stride);
-        if (tag_ok(w[k], tag)) need &= ~(1u << k);
-      }
+      if (need >> k & 1u) w[k] = ld_tag(base + first + k * stride);
+#pragma unroll
+    for (int k = 0; k < MAXK; ++k)
+      if ((need >> k & 1u) && tag_ok(w[k], tag)) need &= ~(1u << k);
     if (!need || aborted(sm)) break;
     if (!started) {
       t0 = wait_start();
@@ -331,8 +334,10 @@ __device__ __forceinline__ int balance_list(int n_own, int floor, uint32_t tag_c
             const int q = base + t + i * kConsumerThreads;
             const uint64_t* src = (q < G) ? p.cx + q : p.lx + (size_t)((q - G) / kBalK) * kMaxOwn + (q - G) % kBalK;
             w[i] = ld_tag(src);
-            if (tag_ok(w[i], tag_c)) need &= ~(1u << i);
           }
+#pragma unroll
+        for (int i = 0; i < MQ; ++i)
+          if ((need >> i & 1u) && tag_ok(w[i], tag_c)) need &= ~(1u << i);
         if (!need || aborted(sm)) break;
         if (!started) { tp = wait_start(); started = true; }
         else if (timed_out(tp, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
@@ -347,36 +352,47 @@ __device__ __forceinline__ int balance_list(int n_own, int floor, uint32_t tag_c
     }
   }
   named_bar_sync(kRedBar, kConsumerThreads);
-  if (warp == 0) {
-    int n = 0;
-    for (int o = lane; o < G; o += 32) n += sm.cnt[o];
+  // block-wide: N = sum of the counts, T, the exclusive prefix of the excess over T, and
+  // this block's deficit start (the deficits of the blocks before it), in fixed orders
+  const int cv = (t < G) ? sm.cnt[t] : 0;
+  {
+    int v = cv;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-    const int T = max((n + G - 1) / G, floor);
-    // exclusive prefix of the excess max(0, n_o - T), and this block's deficit start
-    int carry = 0, dstart = 0;
-    for (int o0 = 0; o0 < G; o0 += 32) {
-      const int o = o0 + lane;
-      const int ex = (o < G) ? max(0, sm.cnt[o] - T) : 0;
-      const int de = (o < G && o < c) ? max(0, T - sm.cnt[o]) : 0;
-      int incl = ex;
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) sm.wsum[0][warp] = v;
+  }
+  named_bar_sync(kRedBar, kConsumerThreads);
+  int n = 0;
 #pragma unroll
-      for (int k = 1; k < 32; k <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, k);
-        if (lane >= k) incl += v;
-      }
-      if (o < G) sm.xpre[o] = carry + incl - ex;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-      int ds = de;
+  for (int w = 0; w < kConsumerWarps; ++w) n += sm.wsum[0][w];
+  const int Tb = max((n + G - 1) / G, floor);
+  const int ex = (t < G) ? max(0, cv - Tb) : 0;
+  const int de = (t < c) ? max(0, Tb - cv) : 0;
+  int incl = ex, dsum = de;
 #pragma unroll
-      for (int k = 16; k > 0; k >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, k);
-      dstart += ds;
+  for (int k = 1; k < 32; k <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, k);
+    if (lane >= k) incl += v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+  if (lane == 31) sm.wsum[1][warp] = incl;
+  if (lane == 0) sm.wsum[2][warp] = dsum;
+  named_bar_sync(kRedBar, kConsumerThreads);
+  {
+    int off = 0, total = 0, dstart_all = 0;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      if (w < warp) off += sm.wsum[1][w];
+      total += sm.wsum[1][w];
+      dstart_all += sm.wsum[2][w];
     }
-    if (lane == 0) {
-      sm.xpre[G] = carry;
-      sm.bal[0] = T;
-      sm.bal[1] = dstart;
-      sm.bal[2] = carry;
+    if (t < G) sm.xpre[t] = off + incl - ex;
+    if (t == 0) {
+      sm.xpre[G] = total;
+      sm.bal[0] = Tb;
+      sm.bal[1] = dstart_all;
+      sm.bal[2] = total;
     }
   }
   named_bar_sync(kRedBar, kConsumerThreads);
@@ -981,7 +997,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     if (slice_owner) {
       // warp w sums partial rows cc = w, w+8, ...; KU rows' words are read together so
       // the L2 round trips overlap; sums run in ascending cc (fixed order)
-      constexpr int KU = 20 / NB;
+      constexpr int KU = 10 / NB;   // 16 warps x 10 rows: all 148 partials in one round at one token
       float acc[NB][kMaxColGroups];
 #pragma unroll
       for (int b = 0; b < NB; ++b)
@@ -1000,14 +1016,22 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
               if (cc0 + kConsumerWarps * k < G && b < B) need |= 1u << (k * NB + b);
             }
           while (need) {
+            uint64_t wk[KU][NB];
+#pragma unroll
+            for (int k = 0; k < KU; ++k)
+#pragma unroll
+              for (int b = 0; b < NB; ++b) {
+                wk[k][b] = 0;
+                if (need >> (k * NB + b) & 1u)
+                  wk[k][b] = ld_tag(p.px + ((size_t)(cc0 + kConsumerWarps * k) * B + b) * d + col0 + 32 * gq + lane);
+              }
 #pragma unroll
             for (int k = 0; k < KU; ++k)
 #pragma unroll
               for (int b = 0; b < NB; ++b)
-                if (need >> (k * NB + b) & 1u) {
-                  const int cc = cc0 + kConsumerWarps * k;
-                  const uint64_t w = ld_tag(p.px + ((size_t)cc * B + b) * d + col0 + 32 * gq + lane);
-                  if (tag_ok(w, tag_p)) { tmp[k][b] = tag_val(w); need &= ~(1u << (k * NB + b)); }
+                if ((need >> (k * NB + b) & 1u) && tag_ok(wk[k][b], tag_p)) {
+                  tmp[k][b] = tag_val(wk[k][b]);
+                  need &= ~(1u << (k * NB + b));
                 }
             if (need && aborted(sm)) break;
             if (need && timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
@@ -1086,18 +1110,20 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         while (need | needm) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            if (need >> k & 1u) {
-              ld_tag2(p.vx + 2 * (size_t)(t + k * kConsumerThreads), w0[k], w1[k]);
-              if (tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
-            }
+            if (need >> k & 1u) ld_tag2(p.vx + 2 * (size_t)(t + k * kConsumerThreads), w0[k], w1[k]);
 #pragma unroll
           for (int i = 0; i < MQ; ++i)
             if (needm >> i & 1u) {
               const int q = t + i * kConsumerThreads;
               const int bq = q / (2 * nslices), cq = (q >> 1) % nslices;
               wm[i] = ld_tag(p.sx + ((size_t)bq * G + cq) * 2 + (q & 1));
-              if (tag_ok(wm[i], tag_v)) needm &= ~(1u << i);
             }
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if ((need >> k & 1u) && tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
+#pragma unroll
+          for (int i = 0; i < MQ; ++i)
+            if ((needm >> i & 1u) && tag_ok(wm[i], tag_v)) needm &= ~(1u << i);
           if (!(need | needm) || aborted(sm)) break;
           if (!started) { tp = wait_start(); started = true; }
           else if (timed_out(tp, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
@@ -1151,10 +1177,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         while (need) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            if (need >> k & 1u) {
-              ld_tag2(p.vx + 2 * (size_t)(base + t + k * kConsumerThreads), w0[k], w1[k]);
-              if (tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
-            }
+            if (need >> k & 1u) ld_tag2(p.vx + 2 * (size_t)(base + t + k * kConsumerThreads), w0[k], w1[k]);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if ((need >> k & 1u) && tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
           if (!need || aborted(sm)) break;
           if (!started) { tp = wait_start(); started = true; }
           else if (timed_out(tp, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
