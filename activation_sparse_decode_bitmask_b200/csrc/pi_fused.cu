@@ -45,6 +45,7 @@ constexpr int kMaxColGroups = 4;    // 32-column groups per reduce slice
 constexpr int kItems = 32;          // ring items in flight (mbarrier pairs)
 constexpr int kBalK = 12;           // list entries every block publishes at least (balance)
 constexpr uint32_t kSleepNs = 20000;  // suspend hint of blocking mbarrier waits (wakes on completion)
+constexpr int kHr = 48;             // F h slots: >= kItems + the dot lookahead (16)
 
 struct Smem {
   uint64_t full[kItems];
@@ -62,8 +63,8 @@ struct Smem {
   float gmean[4];   // glue: mean and standard deviation of v per token
   float gsd[4];
   float red[2][kConsumerWarps][16];   // block reductions: warp partials (double-buffered)
-  float hbuf[2][16][4];         // h of the records of an F window (double-buffered)
-  int win[2];                   // records in an F window; 0: not chosen yet
+  uint64_t hready[kHr];         // F: the dot partials of record s (mod kHr) are in hpart[s]
+  float hpart[kHr][16];         // [warp of the record's group][token][gate/up]
   int32_t list[kMaxList];
   uint8_t list_bits[kMaxList];
   uint8_t own_bits[kMaxOwn];
@@ -205,9 +206,8 @@ __device__ __forceinline__ const uint8_t* ring_next(ConsumerRing& r, uint32_t si
   return r.base + ring_place(r.head, size, r.cap);
 }
 // Wait until ring item `item` has landed (bounded).
-__device__ __forceinline__ void ring_wait_item(uint32_t item, Smem& sm, const FusedParams& p) {
-  uint64_t* bar = &sm.full[item % kItems];
-  const uint32_t par = (item / kItems) & 1u;
+// Wait until phase `par` of `bar` has completed (bounded).
+__device__ __forceinline__ void bar_wait(uint64_t* bar, uint32_t par, Smem& sm, const FusedParams& p) {
   if (!aborted(sm) && !mbar_try_wait(bar, par)) {
     const uint64_t t0 = wait_start();
     while (!mbar_try_wait_sleep(bar, par, kSleepNs)) {
@@ -216,17 +216,15 @@ __device__ __forceinline__ void ring_wait_item(uint32_t item, Smem& sm, const Fu
     }
   }
 }
+__device__ __forceinline__ void ring_wait_item(uint32_t item, Smem& sm, const FusedParams& p) {
+  bar_wait(&sm.full[item % kItems], (item / kItems) & 1u, sm, p);
+}
 // Warp-collective wait for ring item `item`: lane 0 waits on the barrier (acquire) and
 // __syncwarp passes the visibility of the landed bytes on to the other lanes, so the
 // mbarrier sees one waiter per warp instead of 32.
 __device__ __forceinline__ void ring_wait_item_warp(uint32_t item, Smem& sm, const FusedParams& p) {
   if ((threadIdx.x & 31) == 0) ring_wait_item(item, sm, p);
   __syncwarp();
-}
-// Has ring item `item` landed?  (Non-blocking; valid for items fewer than kItems ahead
-// of the oldest item not yet released.)
-__device__ __forceinline__ bool ring_item_ready(uint32_t item, Smem& sm) {
-  return mbar_test_wait(&sm.full[item % kItems], (item / kItems) & 1u);
 }
 __device__ __forceinline__ void ring_release_item(uint32_t item, Smem& sm) {
   __syncwarp();
@@ -257,43 +255,50 @@ __device__ __forceinline__ uint32_t tag_of(uint32_t epoch, int l, int e) {
   return epoch * 1024u + (uint32_t)l * 8u + (uint32_t)e;
 }
 
-// The gate/up dot products of an F window of N records (ring positions pos) over this
-// thread's units, reduced across the warp: returns this lane's share of the reduce-scatter
-// of the window's N * NB * NV values and sets lg = log2 of their padded count.
 __host__ __device__ constexpr int pow2_ceil(int v) { return v <= 1 ? 1 : 2 * pow2_ceil((v + 1) / 2); }
 __host__ __device__ constexpr int log2_exact(int v) { return v <= 1 ? 0 : 1 + log2_exact(v / 2); }
 
-template <int FAM, int ACT, int NB, int NU, int N, int KW>
-__device__ __forceinline__ float window_dots(uint32_t base, const uint32_t (&pos)[KW], const FusedParams& p,
-                                             int t, int nunits, const uint32_t (&xr)[NU][NB][Fam<FAM>::XW], int lane,
-                                             int& lg) {
-  constexpr int NV = (ACT == PI_REGLU) ? 2 : 1;
-  constexpr int V = pow2_ceil(N * NB * NV);
-  float v[V];
+// Warps that share the gate/up dots of one F record: 4 (8 for Q4_0, whose units cost
+// more arithmetic), fewer where the partials of the group would not fit a 16-float slot.
+__host__ __device__ constexpr int f_group_warps(int fam, int act, int nb) {
+  return (fam == FAM_Q4 ? 8 : 4) * nb * (act == PI_REGLU ? 2 : 1) <= 16 ? (fam == FAM_Q4 ? 8 : 4)
+                                                                        : 16 / (nb * (act == PI_REGLU ? 2 : 1));
+}
+
+// This lane's partial gate/up dot products of one F record (at shared address rec) with
+// every token's x (xs: [NB][d] at shared address xs) over the units q0, q0 + qs, ... in
+// ascending order.
+template <int FAM, int ACT, int NB>
+__device__ __forceinline__ void record_dot(uint32_t rec, uint32_t xs, const FusedParams& p, int nunits, int q0,
+                                           int qs, float (&au)[NB], float (&ag)[NB]) {
+  constexpr int XW = Fam<FAM>::XW;
 #pragma unroll
-  for (int i = 0; i < V; ++i) v[i] = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < N; ++kk) {
-    const uint32_t rec = base + pos[kk];
-    float au[NB], ag[NB];
-#pragma unroll
-    for (int b = 0; b < NB; ++b) au[b] = ag[b] = 0.f;
-#pragma unroll
-    for (int j = 0; j < NU; ++j) {
-      const int q = t + kConsumerThreads * j;
-      if (q < nunits) {
-        unit_dot<FAM, NB>(rec + (uint32_t)p.up_off, p.d, q, xr[j], au);
-        if constexpr (ACT == PI_REGLU) unit_dot<FAM, NB>(rec + (uint32_t)p.gate_off, p.d, q, xr[j], ag);
-      }
-    }
+  for (int b = 0; b < NB; ++b) au[b] = ag[b] = 0.f;
+  const uint32_t up = rec + (uint32_t)p.up_off, gate = rec + (uint32_t)p.gate_off;
+  if constexpr (FAM == FAM_Q4) {
+    // x units widen to 16 fp32 values: one token at a time keeps them in registers
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      v[(kk * NB + b) * NV] = au[b];
-      if constexpr (ACT == PI_REGLU) v[(kk * NB + b) * NV + 1] = ag[b];
+      float su[1] = {0.f}, sg[1] = {0.f};
+#pragma unroll 2
+      for (int q = q0; q < nunits; q += qs) {
+        uint32_t xu[1][XW];
+        lds_x_unit<FAM, 1>(xs + (uint32_t)(b * p.d * 2), p.d, q, xu);
+        unit_dot<FAM, 1>(up, p.d, q, xu, su);
+        if constexpr (ACT == PI_REGLU) unit_dot<FAM, 1>(gate, p.d, q, xu, sg);
+      }
+      au[b] = su[0];
+      ag[b] = sg[0];
+    }
+  } else {
+#pragma unroll 4
+    for (int q = q0; q < nunits; q += qs) {
+      uint32_t xu[NB][XW];
+      lds_x_unit<FAM, NB>(xs, p.d, q, xu);
+      unit_dot<FAM, NB>(up, p.d, q, xu, au);
+      if constexpr (ACT == PI_REGLU) unit_dot<FAM, NB>(gate, p.d, q, xu, ag);
     }
   }
-  lg = log2_exact(V);
-  return reduce_scatter<V>(v, lane);
 }
 
 // Balance the active records across blocks.  Every block publishes its own active count
@@ -456,6 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     mbar_init(&sm.list_ready, 1);
     mbar_init(&sm.list2_ready, 1);
     mbar_init(&sm.layer_start, 1);
+    for (int s = 0; s < kHr; ++s) mbar_init(&sm.hready[s], f_group_warps(FAM, ACT, NB));
     sm.abort_flag = 0;
     sm.nlist = 0;
     mbar_fence_init();
@@ -611,6 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
   named_bar_sync(kRedBar, kConsumerThreads);
 
   int redbuf = 0;   // which half of sm.red the next block reduction uses
+  uint32_t fseq = 0;  // F records of earlier layers (h slot of record e: (fseq + e) % kHr)
   for (int l = 0; l < p.L; ++l) {
     const uint32_t tag_u = tag_of(epoch, l, 0), tag_p = tag_of(epoch, l, 1), tag_v = tag_of(epoch, l, 2),
                    tag_c = tag_of(epoch, l, 3);
@@ -851,14 +858,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     }
     stamp(p, l, 3);
 
-    // ------------------------------------------------------------ F: windows of landed records
-    // A window is the next record and the ones after it that have already landed (up
-    // to KW).  Every thread dots its units of the window's gate/up rows with its x units
-    // and a block reduction gives the window's dot products.  Windows are pipelined with
-    // one barrier each: after window w's barrier, 16 threads form h of window w while
-    // every thread adds h * (its units of each down row) of window w-1 into its y units.
-    // Thread 0 chooses window w+1 before that barrier.  A record's sums do not depend on
-    // how the records fall into windows.
+    // ------------------------------------------------------------ F: records
+    // The 16 consumer warps form groups of KG; group g takes the gate/up dots of records
+    // g, g + 16/KG, ... with no block barrier: each warp of the group waits for the record
+    // to land, dots its slice of the units with x from shared memory, reduces across its
+    // lanes, posts its partial sums in the record's h slot and arrives on the slot's
+    // barrier.  Every thread then adds h * (its units of each down row) into its y units
+    // in list order: it waits on each record's slot, sums the KG partials in a fixed order,
+    // forms h and releases the record.  A warp dots a record only while it is fewer than R
+    // records ahead of its own down-row cursor, so the records a warp waits for always
+    // fit in the ring beside the ones not yet released.  Sums run in a fixed order
+    // whatever the timing.
     float y[NU][NB][UE];
 #pragma unroll
     for (int j = 0; j < NU; ++j)
@@ -866,115 +876,86 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       for (int b = 0; b < NB; ++b)
 #pragma unroll
         for (int e = 0; e < UE; ++e) y[j][b][e] = 0.f;
-    constexpr int NV = (ACT == PI_REGLU) ? 2 : 1;
-    constexpr int KW = (16 / (NB * NV) < 8) ? 16 / (NB * NV) : 8;   // 16 reduced values, 8 records
-    // window cap: one window and one more record always fit in the ring together, so
-    // waiting for a record while a window is held can never block the producer
-    const int kw = min(KW, p.rec_window);
-    long long f_wait = 0;   // diagnostics: cycles thread 0 waits for records
-    // thread 0: the window that starts at list position e (ring item `item`): the records
-    // from there that have landed, 0 if none has
-    auto choose = [&](int e, uint32_t item) {
-      int nb = 0;
-      while (nb < kw && e + nb < nlist && ring_item_ready(item + nb, sm)) ++nb;
-      return nb;
-    };
-    uint32_t item_e = ring.item;
-    bool first = true;   // the first window is always chosen with a wait
-    int nwin = 0;        // diagnostics: windows so far
-    int wb = 0;          // buffer of the current window
-    int nb_prev = 0;     // records of the previous window, whose down rows are still to add
-    uint32_t pos_prev[KW];
-#pragma unroll
-    for (int kk = 0; kk < KW; ++kk) pos_prev[kk] = 0;
-    for (int e = 0; e < nlist || nb_prev > 0;) {
-      if (e < nlist && (first || *(volatile int*)&sm.win[wb] == 0)) {
-        // not chosen before the last barrier: wait for its first record (only the previous
-        // window is held, so the producer can place it), then choose
-        named_bar_sync(kRedBar, kConsumerThreads);   // everyone has read sm.win[wb]
-        if (t == 0) {
+    {
+      constexpr int NV = (ACT == PI_REGLU) ? 2 : 1;
+      constexpr int NVAL = NB * NV;                 // partial sums per warp and record
+      constexpr int V = pow2_ceil(NVAL);
+      constexpr int LG = log2_exact(V);
+      constexpr int KG = f_group_warps(FAM, ACT, NB);
+      constexpr int NG = kConsumerWarps / KG;       // records dotted at once
+      static_assert(KG * NVAL <= 16 && kConsumerWarps % KG == 0, "h slot layout");
+      // records E .. E + R - 1 fit in the ring together (at most one record's worth of
+      // space is lost where the placement wraps)
+      const int R = max(1, min((int)(ring.cap / (uint32_t)p.rec_stride) - 1, kConsumerWarps));
+      const uint32_t base = smem_u32(ring.base), xsa = smem_u32(xs);
+      const uint32_t item0 = ring.item;
+      const int kq = warp % KG;
+      long long f_wait = 0, d_wait = 0;   // diagnostics: cycles thread 0 waits for h / for records
+      int ed = warp / KG;                  // next record this warp's group dots
+      uint32_t hd = ring.head;             // ring head before record id (dot cursor)
+      int id = 0;
+      for (int ea = 0; ea < nlist; ++ea) {
+        while (ed < nlist && ed < ea + R) {
+          uint32_t pos = 0;
+          for (; id <= ed; ++id) pos = ring_place(hd, (uint32_t)p.rec_stride, ring.cap);
           const long long wt0 = diag_clock(p);
-          ring_wait_item(item_e, sm, p);
-          f_wait += diag_clock(p) - wt0;
-          if (e == 0) stamp(p, l, 5);
-          sm.win[wb] = max(1, choose(e, item_e));
+          ring_wait_item_warp(item0 + ed, sm, p);
+          d_wait += diag_clock(p) - wt0;
+          if (ed == 0) stamp(p, l, 5);
+          float au[NB], ag[NB];
+          record_dot<FAM, ACT, NB>(base + pos, xsa, p, nunits, 32 * kq + lane, 32 * KG, au, ag);
+          float v[V];
+#pragma unroll
+          for (int i = 0; i < V; ++i) v[i] = 0.f;
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            v[b * NV] = au[b];
+            if constexpr (ACT == PI_REGLU) v[b * NV + 1] = ag[b];
+          }
+          const float sw = reduce_scatter<V>(v, lane);   // lane k: value k >> (5 - LG)
+          const uint32_t s = (fseq + (uint32_t)ed) % kHr;
+          if ((lane & ((32 >> LG) - 1)) == 0 && (lane >> (5 - LG)) < NVAL) sm.hpart[s][kq * NVAL + (lane >> (5 - LG))] = sw;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.hready[s]);
+          ed += NG;
         }
-        named_bar_sync(kRedBar, kConsumerThreads);
-      }
-      first = false;
-      const int nb = (e < nlist) ? *(volatile int*)&sm.win[wb] : 0;
-      if (p.phase_clk && nwin < 16 && nb > 0) {
-        stamp(p, l, 32 + 2 * nwin);
-        stamp_val(p, l, 33 + 2 * nwin, nb);
-      }
-      nwin += (nb > 0);
-      uint32_t pos[KW];
+        const uint32_t pa = ring_place(ring.head, (uint32_t)p.rec_stride, ring.cap);
+        const uint32_t sq = fseq + (uint32_t)ea;
+        const long long wt0 = diag_clock(p);
+        if (lane == 0) bar_wait(&sm.hready[sq % kHr], (sq / kHr) & 1u, sm, p);
+        __syncwarp();
+        f_wait += diag_clock(p) - wt0;
+        const float* hp = sm.hpart[sq % kHr];
+        float sv[NVAL];
 #pragma unroll
-      for (int kk = 0; kk < KW; ++kk) {
-        pos[kk] = 0;
-        // thread 0 saw these records land (acquire) before the barrier that precedes this
-        if (kk < nb) pos[kk] = ring_place(ring.head, (uint32_t)p.rec_stride, ring.cap);
-      }
-      float* red = &sm.red[redbuf][0][0];
-      if (nb > 0) {
-        float sw = 0.f;
-        int lg = 0;   // log2 of the number of reduced values
-        switch (nb) {
-#define PI_WIN(N) case N: if constexpr (N <= KW) sw = window_dots<FAM, ACT, NB, NU, N>(smem_u32(ring.base), pos, p, t, nunits, xr, lane, lg); break;
-          PI_WIN(1) PI_WIN(2) PI_WIN(3) PI_WIN(4) PI_WIN(5) PI_WIN(6) PI_WIN(7) PI_WIN(8)
-#undef PI_WIN
+        for (int i = 0; i < NVAL; ++i) {
+          float a = hp[i];
+#pragma unroll
+          for (int k = 1; k < KG; ++k) a += hp[k * NVAL + i];
+          sv[i] = a;
         }
-        redbuf ^= 1;
-        if ((lane & ((32 >> lg) - 1)) == 0) red[warp * 16 + (lane >> (5 - lg))] = sw;
-      }
-      const int dw = (nwin == 2 || nwin == 3) ? 22 + 3 * (nwin - 2) : -1;   // diagnostics: windows 1, 2
-      if (dw >= 0) stamp(p, l, dw);
-      // the next window, if its records have landed already (never blocks)
-      if (t == 0) sm.win[wb ^ 1] = (e + nb < nlist) ? choose(e + nb, item_e + nb) : 0;
-      named_bar_sync(kRedBar, kConsumerThreads);
-      if (dw >= 0) stamp(p, l, dw + 1);
-      if (t < nb * NB) {
-        const int kk = t / NB, b = t % NB;
-        float su = 0.f, sg = 0.f;
+        const float bi = lds_f32(base + pa + (uint32_t)p.bias_off);
+        const uint32_t bits = sm.list_bits[ea];
+        float h[NB];
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          su += red[w * 16 + (kk * NB + b) * NV];
-          if constexpr (ACT == PI_REGLU) sg += red[w * 16 + (kk * NB + b) * NV + 1];
+        for (int b = 0; b < NB; ++b) {
+          float a;
+          if constexpr (ACT == PI_REGLU) a = fmaxf(sv[b * NV + 1] + bi, 0.f) * sv[b * NV];
+          else a = fmaxf(sv[b * NV] + bi, 0.f);
+          h[b] = (b < B && ((bits >> b) & 1u)) ? a : 0.f;
         }
-        uint32_t mypos = pos[0];
+        const uint32_t drow = base + pa + (uint32_t)p.down_off;
 #pragma unroll
-        for (int k2 = 1; k2 < KW; ++k2) if (k2 == kk) mypos = pos[k2];
-        const float bi = lds_f32(smem_u32(ring.base) + mypos + (uint32_t)p.bias_off);
-        float a;
-        if constexpr (ACT == PI_REGLU) a = fmaxf(sg + bi, 0.f) * su;
-        else a = fmaxf(su + bi, 0.f);
-        sm.hbuf[wb][kk][b] = (b < B && ((sm.list_bits[e + kk] >> b) & 1u)) ? a : 0.f;
+        for (int j = 0; j < NU; ++j)
+          if (t + kConsumerThreads * j < nunits) unit_axpy<FAM, NB>(drow, d, t + kConsumerThreads * j, h, y[j]);
+        ring_release_item(item0 + ea, sm);
       }
-      // down rows of the previous window (its h was formed before this barrier)
-#pragma unroll
-      for (int kk = 0; kk < KW; ++kk) {
-        if (kk < nb_prev) {
-          float h[NB];
-#pragma unroll
-          for (int b = 0; b < NB; ++b) h[b] = sm.hbuf[wb ^ 1][kk][b];
-          const uint32_t drow = smem_u32(ring.base) + pos_prev[kk] + (uint32_t)p.down_off;
-#pragma unroll
-          for (int j = 0; j < NU; ++j)
-            if (t + kConsumerThreads * j < nunits) unit_axpy<FAM, NB>(drow, d, t + kConsumerThreads * j, h, y[j]);
-          ring_release_item(item_e - nb_prev + kk, sm);
-        }
-      }
-      if (dw >= 0) stamp(p, l, dw + 2);
-#pragma unroll
-      for (int kk = 0; kk < KW; ++kk) pos_prev[kk] = pos[kk];
-      nb_prev = nb;
-      item_e += nb;
-      e += nb;
-      wb ^= 1;
+      ring.item = item0 + (uint32_t)nlist;
+      fseq += (uint32_t)nlist;
+      stamp(p, l, 20);
+      stamp_val(p, l, 19, f_wait);
+      stamp_val(p, l, 21, d_wait);
     }
-    ring.item = item_e;
-    stamp(p, l, 20);
-    stamp_val(p, l, 21, nwin);
     // publish the partial y of this block as tagged words
     {
       uint64_t* part = p.px + (size_t)c * B * d;
@@ -991,7 +972,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         }
     }
     stamp(p, l, 4);
-    stamp_val(p, l, 19, f_wait);
 
     // ------------------------------------------------------------ R: slice reduce
     if (slice_owner) {

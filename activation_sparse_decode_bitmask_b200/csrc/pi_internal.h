@@ -107,7 +107,7 @@ struct FusedParams {
   int grid;
   int row_bytes, rec_stride, gate_off, up_off, down_off, bias_off, p1_row, p2_stride;
   int ring_bytes, p1_rows_per_item, p2_rows_per_item, nown_max;
-  int rec_window;      // records per F window at most (one window and one record fit in the ring)
+  int rec_window;      // ring_bytes / rec_stride - 2: at least 1, so three records fit in the ring
   int nslices;
   LayerDev layers[kMaxLayers];
   // inputs / outputs

@@ -99,6 +99,29 @@ __device__ __forceinline__ void load_x_unit(const void* xs, int d, int q, uint32
   }
 }
 
+// The same from shared memory (xs: shared address of [NB][d] in the family's x type)
+template <int FAM, int NB>
+__device__ __forceinline__ void lds_x_unit(uint32_t xs, int d, int q, uint32_t (&xu)[NB][Fam<FAM>::XW]) {
+  constexpr int UE = Fam<FAM>::UE;
+  constexpr uint32_t XB = FAM == FAM_F32 ? 4u : 2u;   // bytes per x element
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const uint32_t a = xs + XB * (uint32_t)(b * d + UE * q);
+    if constexpr (FAM == FAM_F32 || FAM == FAM_F16) {
+      const uint4 v = lds128(a);
+      xu[b][0] = v.x; xu[b][1] = v.y; xu[b][2] = v.z; xu[b][3] = v.w;
+    } else {
+#pragma unroll
+      for (int c = 0; c < UE / 8; ++c) {
+        float w[8];
+        widen8(lds128(a + 16u * c), w);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xu[b][8 * c + e] = __float_as_uint(w[e]);
+      }
+    }
+  }
+}
+
 // acc[b] += (unit q of a weight row) . xu[b]
 template <int FAM, int NB>
 __device__ __forceinline__ void unit_dot(uint32_t row, int d, int q, const uint32_t (&xu)[NB][Fam<FAM>::XW],
