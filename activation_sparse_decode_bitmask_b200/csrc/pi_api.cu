@@ -122,7 +122,6 @@ pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedPara
   p.wait_cycles = kDefaultWaitNs * 3;   // cycles at up to 3 GHz: at least the nominal budget
   p.barrier_extra = 0;
   p.poll_ns = 64;          // back-off between exchange polling rounds
-  p.gate_producer = 0;
   return PI_OK;
 }
 

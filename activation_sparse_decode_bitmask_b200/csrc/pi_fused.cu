@@ -52,7 +52,7 @@ struct Smem {
   uint64_t empty[kItems];
   uint64_t list_ready;          // the first part of the block's list is in place
   uint64_t list2_ready;         // the whole list is in place
-  uint64_t layer_start;
+  uint64_t f_done;              // the consumers have taken every F record of the layer
   int abort_flag;
   int nlist_a;                  // records of the first part of the list
   int nlist;
@@ -311,13 +311,14 @@ __device__ __forceinline__ void record_dot(uint32_t rec, uint32_t xs, const Fuse
 // any case, so they are fetched while this runs.  Returns the block's new list length;
 // the taken records follow its own in sm.list.
 __device__ __forceinline__ int balance_list(int n_own, int floor, uint32_t tag_c, Smem& sm, const FusedParams& p, int c,
-                                            int G, int t, int warp, int lane) {
+                                            int G, int t, int warp, int lane, int l) {
   // publish the count and at least kBalK entries (padded), so that one polling round can
   // read every count and every block's first kBalK entries
   if (t < max(n_own, kBalK))
     st_tag(p.lx + (size_t)c * kMaxOwn + t,
            __uint_as_float(t < n_own ? ((uint32_t)sm.list[t] | ((uint32_t)sm.list_bits[t] << 24)) : 0u), tag_c);
   if (t == 0) st_tag(p.cx + c, __int_as_float(n_own), tag_c);
+  stamp(p, l, 22);
   {
     // chunks of 4 words per thread: one round for up to 2048 words (157 blocks)
     constexpr int MQ = 4;
@@ -356,7 +357,9 @@ __device__ __forceinline__ int balance_list(int n_own, int floor, uint32_t tag_c
       }
     }
   }
+  stamp(p, l, 23);
   named_bar_sync(kRedBar, kConsumerThreads);
+  stamp(p, l, 24);
   // block-wide: N = sum of the counts, T, the exclusive prefix of the excess over T, and
   // this block's deficit start (the deficits of the blocks before it), in fixed orders
   const int cv = (t < G) ? sm.cnt[t] : 0;
@@ -405,6 +408,7 @@ __device__ __forceinline__ int balance_list(int n_own, int floor, uint32_t tag_c
   const int keep = min(n_own, T);
   const int deficit = max(0, T - n_own);
   const int ntake = max(0, min(dstart + deficit, xtotal) - dstart);
+  stamp(p, l, 25);
   if (t < ntake) {
     const int x = dstart + t;
     int lo = 0, hi = G;   // owner o: xpre[o] <= x < xpre[o + 1]
@@ -460,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     }
     mbar_init(&sm.list_ready, 1);
     mbar_init(&sm.list2_ready, 1);
-    mbar_init(&sm.layer_start, 1);
+    mbar_init(&sm.f_done, 1);
     for (int s = 0; s < kHr; ++s) mbar_init(&sm.hready[s], f_group_warps(FAM, ACT, NB));
     sm.abort_flag = 0;
     sm.nlist = 0;
@@ -514,13 +518,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         const LayerDev Ld = p.layers[l];
         uint8_t* dst;
         uint64_t* fb;
-        if (do_pred && p.gate_producer && l > 0) {
-          // experiment: keep the producer quiet until the consumers start this layer
+        if (do_pred && do_ffn && l > 0) {
+          // the predictor rows of this layer are not needed before the glue of the last
+          // one ends: start their copies once this block has taken its last F record, so
+          // that they do not compete with the F records other blocks still wait for
           const uint64_t t0 = wait_start();
-          while (!mbar_try_wait_sleep(&sm.layer_start, (uint32_t)(l & 1), kSleepNs)) {
+          while (!mbar_try_wait_sleep(&sm.f_done, (uint32_t)((l - 1) & 1), kSleepNs)) {
             if (aborted(sm)) { ok = false; break; }
             if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
           }
+          if (!ok) break;
         }
         if (do_pred) {
           for (int k = k0; k < k1 && ok; k += p.p1_rows_per_item) {
@@ -638,7 +645,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           for (int e = 0; e < XW; ++e) xr[j][b][e] = 0u;
       }
     }
-    if (t == 0) mbar_arrive(&sm.layer_start);
 
     if (do_pred) {
       // ---------------------------------------------------------- P-a: u rows of this block
@@ -819,7 +825,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           mbar_arrive(&sm.list_ready);
         }
         signaled_a = true;
-        nlist = balance_list(nlist, floor, tag_c, sm, p, c, G, t, warp, lane);
+        nlist = balance_list(nlist, floor, tag_c, sm, p, c, G, t, warp, lane, l);
       }
       stamp_val(p, l, 14, nlist);
     } else if (do_ffn) {
@@ -952,6 +958,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       }
       ring.item = item0 + (uint32_t)nlist;
       fseq += (uint32_t)nlist;
+      if (t == 0) mbar_arrive(&sm.f_done);
       stamp(p, l, 20);
       stamp_val(p, l, 19, f_wait);
       stamp_val(p, l, 21, d_wait);

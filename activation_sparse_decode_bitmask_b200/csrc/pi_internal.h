@@ -137,7 +137,6 @@ struct FusedParams {
   long long* phase_clk;  // diagnostics: SM cycle stamps per block, layer and phase, or null
   int phase_global;      // stamps from the global ns timer instead of the SM cycle counter
   unsigned poll_ns;      // back-off between polling rounds of the cross-block exchanges
-  int gate_producer;     // 1: the producer starts a layer's copies only when the consumers do
 };
 
 enum : int { MODE_PREDICT = 1, MODE_FFN = 2, MODE_GLUE = 4 };
