@@ -7,8 +7,8 @@ PyTorch fallback; importing it fails if libpi.so has not been built.
 """
 from ._abi import (PI_F16, PI_F32, PI_MAX_BATCH, PI_NOALLOC_SCRATCH_BYTES, PI_Q4_0, PI_RELU, PI_REGLU, EXPORTS,
                    Layer, LayerDesc, LayerWeights, PiError, Trace, Workspace, abi_version, compact_active,
-                   decode_stack, decode_stack_host, diag_barrier_timeout, get_perm, lib, load_layer, make_desc,
-                   predict, predict_noalloc, reorder_hot_prefix, sparse_ffn, status_str)
+                   decode_stack, decode_stack_host, diag_barrier_timeout, get_perm, kernel_launches, lib, load_layer,
+                   make_desc, predict, predict_noalloc, reorder_hot_prefix, sparse_ffn, status_str)
 
 # the C names, for readers coming from the header
 pi_load_layer = load_layer
@@ -21,3 +21,4 @@ pi_sparse_ffn = sparse_ffn
 pi_decode_stack = decode_stack
 pi_decode_stack_host = decode_stack_host
 pi_status_str = status_str
+pi_kernel_launches = kernel_launches

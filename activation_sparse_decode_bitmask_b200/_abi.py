@@ -29,7 +29,8 @@ EXPORTS = ["pi_load_layer", "pi_reorder_hot_prefix", "pi_get_perm", "pi_layer_ge
            "pi_workspace_create", "pi_workspace_free", "pi_stream_status", "pi_workspace_active_total",
            "pi_workspace_layer_counts", "pi_diag_phase_clocks_enable", "pi_diag_phase_clocks_read",
            "pi_device_grid", "pi_diag_barrier_timeout", "pi_predict", "pi_predict_noalloc", "pi_compact_active",
-           "pi_sparse_ffn", "pi_decode_stack", "pi_decode_stack_host", "pi_status_str", "pi_abi_version"]
+           "pi_sparse_ffn", "pi_decode_stack", "pi_decode_stack_host", "pi_status_str", "pi_abi_version",
+           "pi_kernel_launches"]
 
 
 class PiError(RuntimeError):
@@ -80,6 +81,7 @@ def _load() -> ctypes.CDLL:
         "pi_decode_stack_host": (i, [vp, i, vp, vp, i, vp, vp]),
         "pi_status_str": (ctypes.c_char_p, [i]),
         "pi_abi_version": (i, []),
+        "pi_kernel_launches": (ctypes.c_ulonglong, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -273,3 +275,8 @@ def status_str(st: int) -> str:
 
 def abi_version() -> int:
     return _lib.pi_abi_version()
+
+
+def kernel_launches() -> int:
+    """Kernels this library has launched in this process so far (host-side count)."""
+    return int(_lib.pi_kernel_launches())

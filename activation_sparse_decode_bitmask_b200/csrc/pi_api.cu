@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -215,9 +216,19 @@ bool same_desc(const pi_layer_desc& a, const pi_layer_desc& b) {
 
 }  // namespace
 
+namespace pi {
+std::atomic<uint64_t>& launch_counter() {
+  static std::atomic<uint64_t> n{0};
+  return n;
+}
+void note_launch() { launch_counter().fetch_add(1, std::memory_order_relaxed); }
+}  // namespace pi
+
 extern "C" {
 
 int pi_abi_version(void) { return 10000; }
+
+uint64_t pi_kernel_launches(void) { return pi::launch_counter().load(std::memory_order_relaxed); }
 
 const char* pi_status_str(pi_status s) {
   switch (s) {
@@ -503,6 +514,7 @@ pi_status pi_predict(const pi_layer* L, const void* x, int B, uint32_t* mask, fl
   p.logits_out = logits;
   PI_TRY(cudaMemsetAsync(mask, 0, (size_t)B * (L->desc.d_ff / 32) * 4, stream));   // bits are OR-ed in
   PI_TRY(launch_fused(L->family, L->desc.act, B, p, smem, stream));
+  note_launch();
   return PI_OK;
 }
 
@@ -537,6 +549,7 @@ pi_status pi_sparse_ffn(const pi_layer* L, const void* x, int B, const uint32_t*
   p.count_in = count;
   p.y_out = y;
   PI_TRY(launch_fused(L->family, L->desc.act, B, p, smem, stream));
+  note_launch();
   return PI_OK;
 }
 
@@ -574,6 +587,7 @@ pi_status pi_decode_stack(pi_layer* const* layers, int Lc, void* x_inout, int B,
   PI_TRY(cudaMemsetAsync(ws->layer_count, 0, (size_t)Lc * 4, stream));
   if (trace && trace->mask) PI_TRY(cudaMemsetAsync(trace->mask, 0, (size_t)Lc * B * words * 4, stream));
   PI_TRY(launch_fused(L0->family, L0->desc.act, B, p, smem, stream));
+  note_launch();
   if (trace && trace->idx)
     for (int l = 0; l < Lc; ++l)
       PI_TRY(launch_compact(trace->mask + (size_t)l * B * words, B, L0->desc.d_ff, trace->idx + (size_t)l * L0->desc.d_ff,
@@ -629,6 +643,7 @@ pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaSt
   p.wait_cycles = timeout_ns * 2;   // SM cycles, about 2 per ns
   p.barrier_extra = 1;   // one arrival more than the grid has: no wait can complete
   PI_TRY(launch_barrier_probe(p, 2, stream));
+  note_launch();
   return PI_OK;
 }
 
@@ -683,6 +698,7 @@ pi_status noalloc_scratch(int dev, cudaStream_t stream, unsigned char** out) {
     void* ptr = nullptr;
     PI_TRY(cudaGetSymbolAddress(&ptr, g_noalloc_scratch));
     PI_TRY(cudaMemsetAsync(ptr, 0, PI_NOALLOC_SCRATCH_BYTES, stream));
+    note_launch();
     noalloc_init_kernel<<<1, 1, 0, stream>>>(static_cast<uint32_t*>(ptr));
     PI_TRY(cudaGetLastError());
     PI_TRY(cudaStreamSynchronize(stream));
@@ -730,6 +746,9 @@ pi_status pi_predict_noalloc(const pi_layer* L, const void* x, int B, uint32_t* 
   p.logits_out = logits;
   PI_TRY(cudaMemsetAsync(mask, 0, (size_t)B * (L->desc.d_ff / 32) * 4, stream));   // bits are OR-ed in
   PI_TRY(launch_fused(L->family, L->desc.act, B, p, smem, stream));
+  note_launch();
+
+  note_launch();
   noalloc_status_kernel<<<1, 1, 0, stream>>>(w.bar, w.err, status);
   PI_TRY(cudaGetLastError());
   return PI_OK;

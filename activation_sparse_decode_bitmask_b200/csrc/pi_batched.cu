@@ -449,14 +449,17 @@ cudaError_t launch_rowtok_nt(const RowTokArgs& a, int nmat, int blocks, cudaStre
     if (split) return cudaErrorNotSupported;
     auto k = rowtok_kernel<NT, 2, false>;
     if ((e = smem_attr_once(k, smem, conf2)) != cudaSuccess) return e;
+    note_launch();
     k<<<grid, 32 * kBW, smem, s>>>(a);
   } else if (split) {
     auto k = rowtok_kernel<NT, 1, true>;
     if ((e = smem_attr_once(k, smem, conf_split)) != cudaSuccess) return e;
+    note_launch();
     k<<<grid, 32 * kBW, smem, s>>>(a);
   } else {
     auto k = rowtok_kernel<NT, 1, false>;
     if ((e = smem_attr_once(k, smem, conf1)) != cudaSuccess) return e;
+    note_launch();
     k<<<grid, 32 * kBW, smem, s>>>(a);
   }
   return cudaGetLastError();
@@ -483,6 +486,7 @@ cudaError_t launch_rows(RowTokArgs a, RowEpiArgs ep, int nmat, int rows_max, siz
   ep.nmat = nmat;
   ep.part = a.part;
   const long long n = (long long)rows_max * 32;
+  note_launch();
   rowtok_epilogue<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ep);
   return cudaGetLastError();
 }
@@ -494,6 +498,7 @@ cudaError_t launch_down_nt(const DownArgs& a, cudaStream_t s) {
   static int conf = 0;
   const cudaError_t e = smem_attr_once(k, smem, conf);
   if (e != cudaSuccess) return e;
+  note_launch();
   k<<<dim3((a.d + kDCols - 1) / kDCols, a.nsplit), 32 * kBW, smem, s>>>(a);
   return cudaGetLastError();
 }
@@ -599,6 +604,7 @@ cudaError_t batched_ffn(const BatchedLayer& L, const void* x, int B, const uint3
   }
   if (e != cudaSuccess) return e;
   const int n = B * L.d;
+  note_launch();
   down_reduce<<<(n + 255) / 256, 256, 0, s>>>(ypart, dn.nsplit, n, y);
   return cudaGetLastError();
 }
@@ -619,11 +625,13 @@ __global__ void count_add_kernel(const int32_t* count, unsigned long long* total
 }  // namespace
 
 cudaError_t batched_count(const int32_t* count, unsigned long long* total, int32_t* layer_count, cudaStream_t s) {
+  note_launch();
   count_add_kernel<<<1, 1, 0, s>>>(count, total, layer_count);
   return cudaGetLastError();
 }
 
 cudaError_t batched_glue(const void* x, const float* y, int B, int d, void* x_out, void* trace_x, cudaStream_t s) {
+  note_launch();
   glue_kernel<<<B, 256, 0, s>>>(reinterpret_cast<const __half*>(x), y, d, reinterpret_cast<__half*>(x_out),
                                 reinterpret_cast<__half*>(trace_x));
   return cudaGetLastError();

@@ -100,6 +100,9 @@ struct pi_workspace {
 
 namespace pi {
 
+// Counts one kernel launch of this library (read by pi_kernel_launches).
+void note_launch();
+
 // Parameters of one launch of the fused kernel.
 struct FusedParams {
   int mode;            // bit 1: predictor, bit 2: FFN, bit 4: stack glue (layer loop)

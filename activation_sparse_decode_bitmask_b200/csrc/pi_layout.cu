@@ -177,14 +177,14 @@ cudaError_t relayout_transpose(const void* src, int esize, int rows, int cols, l
                                uint8_t* dst, long long dst_stride, long long dst_off, cudaStream_t s,
                                int G, int nmax) {
   const dim3 blk(32, 8);
+  if (esize != 4 && esize != 2) return cudaErrorInvalidValue;
+  note_launch();
   if (esize == 4)
     transpose_kernel<uint32_t><<<tgrid(rows, cols), blk, 0, s>>>(static_cast<const uint32_t*>(src), rows, cols,
                                                                   src_ld, dst, dst_stride, dst_off, G, nmax);
-  else if (esize == 2)
+  else
     transpose_kernel<uint16_t><<<tgrid(rows, cols), blk, 0, s>>>(static_cast<const uint16_t*>(src), rows, cols,
                                                                   src_ld, dst, dst_stride, dst_off, G, nmax);
-  else
-    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
@@ -192,6 +192,7 @@ cudaError_t relayout_copy_rows(const void* src, long long src_stride, long long 
                                long long dst_stride, long long dst_off, int rows, int bytes,
                                const int32_t* order, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
+  note_launch();
   copy_rows_kernel<<<rows, 128, 0, s>>>(static_cast<const uint8_t*>(src), src_stride, src_off, dst, dst_stride,
                                         dst_off, rows, bytes, order);
   return cudaGetLastError();
@@ -199,40 +200,48 @@ cudaError_t relayout_copy_rows(const void* src, long long src_stride, long long 
 
 cudaError_t relayout_p2_header(const float* thresh, const float* bias, int f, uint8_t* p2o, int p2_stride,
                                int hdr_off, int G, int nmax, cudaStream_t s) {
+  note_launch();
   p2_header_kernel<<<(f + 255) / 256, 256, 0, s>>>(thresh, bias, f, p2o, p2_stride, hdr_off, G, nmax);
   return cudaGetLastError();
 }
 
 cudaError_t relayout_row_scalar(const float* v, int f, uint8_t* dst, long long stride, long long off, cudaStream_t s) {
+  note_launch();
   row_scalar_kernel<<<(f + 255) / 256, 256, 0, s>>>(v, f, dst, stride, off);
   return cudaGetLastError();
 }
 
 cudaError_t gather_owner_rows(const uint8_t* src, uint8_t* dst, const int32_t* order, int f, int G, int nmax,
                               int stride, cudaStream_t s) {
+  note_launch();
   gather_owner_rows_kernel<<<f, 128, 0, s>>>(src, dst, order, f, G, nmax, stride);
   return cudaGetLastError();
 }
 
 cudaError_t hot_order(const float* freq, int n, int32_t* order, int* bad, cudaStream_t s) {
+  note_launch();
   hot_rank_kernel<<<(n + 255) / 256, 256, 0, s>>>(freq, n, order, bad);
   return cudaGetLastError();
 }
 
 cudaError_t gather_f32(const float* src, const int32_t* order, int n, float* dst, cudaStream_t s) {
+  note_launch();
   gather_f32_kernel<<<(n + 255) / 256, 256, 0, s>>>(src, order, n, dst);
   return cudaGetLastError();
 }
 cudaError_t gather_i32(const int32_t* src, const int32_t* order, int n, int32_t* dst, cudaStream_t s) {
+  note_launch();
   gather_i32_kernel<<<(n + 255) / 256, 256, 0, s>>>(src, order, n, dst);
   return cudaGetLastError();
 }
 cudaError_t iota_i32(int32_t* p, int n, cudaStream_t s) {
+  note_launch();
   iota_kernel<<<(n + 255) / 256, 256, 0, s>>>(p, n);
   return cudaGetLastError();
 }
 
 cudaError_t launch_compact(const uint32_t* mask, int B, int f, int32_t* idx, int32_t* count, cudaStream_t s) {
+  note_launch();
   compact_kernel<<<1, 1024, 0, s>>>(mask, B, f, idx, count);
   return cudaGetLastError();
 }

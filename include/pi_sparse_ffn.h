@@ -290,6 +290,13 @@ const char* pi_status_str(pi_status s);
 /* Compile-time version of this ABI (major * 10000 + minor * 100 + patch). */
 int pi_abi_version(void);
 
+/* Number of kernels this library has launched in the calling process so far, on any
+ * device and stream (layout, predictor, compaction, FFN and service kernels alike;
+ * memsets and copies are not kernels of this library and are not counted).  The count is
+ * taken on the host at each launch, so the difference between two reads brackets the
+ * launches of the calls made in between.  Thread-safe; never fails. */
+uint64_t pi_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -51,6 +51,7 @@ def test_host_validation_without_gpu(lib):
     assert L.pi_abi_version() == 10000
     assert L.pi_status_str(0) == b"ok"
     assert L.pi_status_str(5) == b"a device-side wait timed out"
+    assert pi.kernel_launches() == 0       # nothing has launched in this CPU-only process
     # argument errors are returned before any CUDA call
     h = ctypes.c_void_p()
     assert L.pi_workspace_create(0, 1024, 64, 1, 1, ctypes.byref(h)) == 1

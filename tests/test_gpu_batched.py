@@ -144,3 +144,20 @@ def test_batched_fullsize_opt_layer(B):
     err = H.rel_err(y.cpu().double().numpy(), y_ref)
     assert err <= H.y_tol(wl.w_dtype), err
     print(f"OPT-175B layer B={B}: union {cnt}/{wl.d_ff}, in-band flips {flips}, y rel err {err:.2e}")
+
+
+def test_kernel_launch_count_per_step():
+    """pi_kernel_launches brackets the launches of a call: one persistent launch per decode
+    step at one token, eleven launches per layer on the batched path (predictor rows and
+    epilogue twice, compaction, count, gate/up rows and epilogue, down, down reduce, glue)."""
+    wl = W_OPT_SMALL
+    gl, _ = H.build_layers(pi, wl, keep_host=False)
+    L = wl.n_layers
+    for B, per_step in [(1, 1), (8, 11 * L)]:
+        ws = _ws(wl, B, L)
+        x = S.make_inputs(wl, B, "cuda", stream_id=170 + B)
+        n0 = pi.kernel_launches()
+        pi.decode_stack(gl, x, B, ws)
+        n1 = pi.kernel_launches()
+        assert ws.status() == 0
+        assert n1 - n0 == per_step, (B, n1 - n0)
