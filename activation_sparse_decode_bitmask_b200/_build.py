@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpi.so")
 SOURCES = ["pi_fused.cu", "pi_batched.cu", "pi_layout.cu", "pi_api.cu"]
-DEPS = SOURCES + ["pi_internal.h", "pi_layout.h", "pi_ptx.cuh"]
+DEPS = SOURCES + ["pi_internal.h", "pi_layout.h", "pi_ptx.cuh", "pi_rowmath.cuh"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "pi_sparse_ffn.h")
 
 NVCC_FLAGS = [
