@@ -286,7 +286,12 @@ template <int NT>
 __global__ void __launch_bounds__(32 * kBW) down_kernel(const DownArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int BP = NT * 8;
-  constexpr int W_B = kDN * kDPad, STAGE_B = W_B + 2 * BP * kHPad;   // weights, then h hi / lo [2][BP]
+  // a stage: the chunk's down-row slices, h as fp16 hi / lo [2][BP], and h as copied (fp32 [kDN][BP])
+  constexpr int W_B = kDN * kDPad, HS_B = 2 * BP * kHPad, STAGE_B = W_B + HS_B + kDN * BP * 4;
+  constexpr int PC = kDCols * 2 / 16;          // 16-byte pieces of a row slice
+  constexpr int PW = kDN * PC / (32 * kBW);    // row-slice pieces per thread and chunk
+  constexpr int PH = BP / 4;                   // 16-byte pieces of a neuron's h
+  static_assert(kDN * PC % (32 * kBW) == 0 && kDN * PH % (32 * kBW) == 0, "down staging");
   int count = *a.count;
   if (count < 0 || count > a.fmax) count = 0;   // reported by the gate/up kernel; y becomes 0
   const int nch = (count + kDN - 1) / kDN;
@@ -295,16 +300,31 @@ __global__ void __launch_bounds__(32 * kBW) down_kernel(const DownArgs a) {
   const int c0 = blockIdx.x * kDCols;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const uint32_t base_u = smem_u32(smem);
-  auto stage_w = [&](int ch, int buf) {
+  // The neuron index of each of this thread's row-slice pieces of a chunk is loaded one
+  // chunk before the copies that need it, so no copy waits on a global load.
+  auto load_idx = [&](int ch, int (&iv)[PW]) {
+#pragma unroll
+    for (int u = 0; u < PW; ++u) {
+      const int jj = (t + u * 32 * kBW) / PC;
+      iv[u] = ch < c_end ? __ldg(a.idx + min(ch * kDN + jj, count - 1)) : 0;
+    }
+  };
+  auto stage = [&](int ch, int buf, const int (&iv)[PW]) {
     const int j0 = ch * kDN;
-    constexpr int PC = kDCols * 2 / 16;   // 16-byte pieces of a row slice
-    const uint32_t w_u = base_u + (uint32_t)(buf * STAGE_B);
-    for (int e = t; e < kDN * PC; e += 32 * kBW) {
-      const int jj = e / PC, pc = e % PC;
-      int i = __ldg(a.idx + min(j0 + jj, count - 1));
+    const uint32_t w_u = base_u + (uint32_t)(buf * STAGE_B), hr_u = w_u + W_B + HS_B;
+#pragma unroll
+    for (int u = 0; u < PW; ++u) {
+      const int e = t + u * 32 * kBW, jj = e / PC, pc = e % PC;
+      int i = iv[u];
       if (i < 0 || i >= a.fmax) i = 0;   // reported by the gate/up kernel
       cp_async16(w_u + (uint32_t)(jj * kDPad + pc * 16),
                  a.rec + (size_t)i * a.rec_stride + a.down_off + (size_t)c0 * 2 + pc * 16);
+    }
+    // h rows past count are clamped to the last one and zeroed when converted
+#pragma unroll
+    for (int u = 0; u < kDN * PH / (32 * kBW); ++u) {
+      const int e = t + u * 32 * kBW, jj = e / PH, pc = e % PH;
+      cp_async16(hr_u + (uint32_t)((jj * BP + pc * 4) * 4), a.h + (size_t)min(j0 + jj, count - 1) * 32 + pc * 4);
     }
   };
   float c[kDM][NT][4];
@@ -314,29 +334,38 @@ __global__ void __launch_bounds__(32 * kBW) down_kernel(const DownArgs a) {
     for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e) c[mt][n][e] = 0.f;
+  int iv[PW];
 #pragma unroll
   for (int s = 0; s < kStages - 1; ++s) {
-    if (c_begin + s < c_end) stage_w(c_begin + s, s);
+    if (c_begin + s < c_end) {
+      load_idx(c_begin + s, iv);
+      stage(c_begin + s, s, iv);
+    }
     cp_async_commit();
   }
+  load_idx(c_begin + kStages - 1, iv);
   for (int ch = c_begin; ch < c_end; ++ch) {
     const int buf = (ch - c_begin) % kStages;
     const uint32_t w_u = base_u + (uint32_t)(buf * STAGE_B), h_u = w_u + W_B;
-    // h of the chunk, split into fp16 hi / lo (neurons past count contribute zero); this
-    // buffer's previous readers finished before the last barrier
-    const int j0 = ch * kDN;
-    for (int e = t; e < BP * kDN; e += 32 * kBW) {
-      const int b = e / kDN, jj = e % kDN;
-      const float v = (j0 + jj < count && b < a.B) ? a.h[(size_t)(j0 + jj) * 32 + b] : 0.f;
-      __half hi, lo;
-      split_h(v, hi, lo);
-      reinterpret_cast<__half*>(smem + buf * STAGE_B + W_B + (size_t)b * kHPad)[jj] = hi;
-      reinterpret_cast<__half*>(smem + buf * STAGE_B + W_B + (size_t)(BP + b) * kHPad)[jj] = lo;
-    }
     cp_async_wait_1();
     __syncthreads();   // weights and h of chunk ch are in place; chunk ch - 1's buffer is free
-    if (ch + kStages - 1 < c_end) stage_w(ch + kStages - 1, (ch + kStages - 1 - c_begin) % kStages);
+    if (ch + kStages - 1 < c_end) stage(ch + kStages - 1, (ch + kStages - 1 - c_begin) % kStages, iv);
     cp_async_commit();
+    load_idx(ch + kStages, iv);   // consumed by the next iteration's copies
+    // h of the chunk, split into fp16 hi / lo (neurons past count contribute zero)
+    {
+      const int j0 = ch * kDN;
+      const float* hr = reinterpret_cast<const float*>(smem + buf * STAGE_B + W_B + HS_B);
+      for (int e = t; e < BP * kDN; e += 32 * kBW) {
+        const int b = e / kDN, jj = e % kDN;
+        const float v = (j0 + jj < count && b < a.B) ? hr[jj * BP + b] : 0.f;
+        __half hi, lo;
+        split_h(v, hi, lo);
+        reinterpret_cast<__half*>(smem + buf * STAGE_B + W_B + (size_t)b * kHPad)[jj] = hi;
+        reinterpret_cast<__half*>(smem + buf * STAGE_B + W_B + (size_t)(BP + b) * kHPad)[jj] = lo;
+      }
+    }
+    __syncthreads();   // h of chunk ch is split
 #pragma unroll
     for (int ks = 0; ks < kDN / 16; ++ks) {
       uint32_t bf[NT][2][2];
@@ -493,7 +522,7 @@ cudaError_t launch_rows(RowTokArgs a, RowEpiArgs ep, int nmat, int rows_max, siz
 
 template <int NT>
 cudaError_t launch_down_nt(const DownArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)kStages * ((size_t)kDN * kDPad + 2 * (size_t)NT * 8 * kHPad);
+  const size_t smem = (size_t)kStages * ((size_t)kDN * kDPad + 2 * (size_t)NT * 8 * kHPad + (size_t)kDN * NT * 8 * 4);
   auto k = down_kernel<NT>;
   static int conf = 0;
   const cudaError_t e = smem_attr_once(k, smem, conf);
