@@ -110,8 +110,8 @@ pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedPara
   const long long max_item = std::max({(long long)L->rec_stride, (long long)p.p1_rows_per_item * L->p1_row,
                                        (long long)p.p2_rows_per_item * L->p2_stride});
   if (p.ring_bytes < 2 * max_item || max_item >= (1 << 20)) return PI_ERR_UNSUPPORTED;
-  // records outstanding at once: floor(ring / stride) - 1 (an item never wraps); a
-  // window plus the record after it must fit
+  // records outstanding at once: floor(ring / stride) - 1 (an item never wraps); the F
+  // phase needs room for at least two records beside the one it waits for
   p.rec_window = p.ring_bytes / L->rec_stride - 2;
   if (p.rec_window < 1) return PI_ERR_UNSUPPORTED;
   smem = fixed + (size_t)p.ring_bytes;

@@ -205,9 +205,11 @@ pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaSt
  * 3 list handed to the producer, 5 first record landed, 4 FFN partials published,
  * 6 slice reduce done, 16 moments read, 17 v read, 8 glue done. Producer warp: 9 waits
  * for the list, 10 list received, 11 all records issued; 12 and 13 mark the first
- * predictor item landing (P2, P1). Slot 14 holds the block's record count, 18 the
- * cycles spent waiting for P2 rows, 19 those spent waiting for records, and 32-63 the
- * start and size of up to 16 F windows. With `on` = 2
+ * predictor item landing (P2, P1), 20 F loop done, 22-25 the balancing steps (list
+ * published, thread 0's words read, every thread's words read, targets computed).
+ * Slot 14 holds the block's record count, 18 the cycles spent waiting for P2 rows, 19
+ * the cycles thread 0 waits for the h of records and 21 those warp 0 waits for records
+ * to land. With `on` = 2
  * the stamps come from the GPU's global nanosecond timer instead, so blocks can be
  * compared with one another. With `on` = 0 recording stops and the buffer is freed. */
 pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on);
