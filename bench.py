@@ -140,8 +140,8 @@ class ClockSampler:
         if not self.ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
         names = [n for n, b in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
-                "reasons": names, "samples": len(self.samples)}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_min_mhz": float(min(self.samples)),
+                "sm_max_mhz": float(self.max_mhz), "reasons": names, "samples": len(self.samples)}
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -290,11 +290,12 @@ def run_ours(args, world, rank, local):
         pi.decode_stack_host(layers, xh[k], xo, B, ws)
     dist_barrier(world)
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for k in range(Ke):
-        pi.decode_stack_host(layers, xh[k], xo, B, ws)
-    f1.record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(local) as clk_e2e:
+        f0.record(stream)
+        for k in range(Ke):
+            pi.decode_stack_host(layers, xh[k], xo, B, ws)
+        f1.record(stream)
+        torch.cuda.synchronize()
     e2e_ms = dist_max(f0.elapsed_time(f1), world)
     xbytes = B * wl.d_model * (4 if wl.x_dtype == "f32" else 2)
 
@@ -316,7 +317,8 @@ def run_ours(args, world, rank, local):
                                 f"whole step: {launches // K} launches of the batched kernels per step"),
                      "peak_source": peak_kind},
         "e2e": {"value": round(world * Ke * B / (e2e_ms / 1e3), 2), "unit": "tokens/s",
-                "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": xbytes, "steps": Ke},
+                "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": xbytes, "steps": Ke,
+                "clocks": clk_e2e.summary()},
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
