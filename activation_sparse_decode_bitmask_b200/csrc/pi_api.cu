@@ -134,14 +134,18 @@ pi_status check_ws(const pi_workspace* ws, const pi_layer_desc& d, int B, int L)
 }
 
 // Hot-prefix length at batch B: the neurons (in hot order) whose union firing probability
-// 1 - (1 - f)^B is at least 1/2, or the count fixed by pi_reorder_hot_prefix.
-int hot_len(const pi_layer* L, int B) {
-  if (!L->freq_host) return 0;
+// 1 - (1 - f)^B is at least 1/2, or the count fixed by pi_reorder_hot_prefix.  Computed
+// once per batch size when the frequencies arrive (the scan would otherwise run for every
+// layer of every call).
+int hot_len_scan(const pi_layer* L, int B) {
   if (L->hot_count >= 0) return L->hot_count;
   int n = 0;
   const int F = L->desc.d_ff;
   while (n < F && 1.0 - std::pow(1.0 - (double)L->freq_host[n], (double)B) >= 0.5) ++n;
   return n;
+}
+int hot_len(const pi_layer* L, int B) {
+  return (L->freq_host && B >= 1 && B <= 32) ? L->hot_len_b[B] : 0;
 }
 
 BatchedLayer bview(const pi_layer* L) {
@@ -191,18 +195,20 @@ pi_status decode_stack_batched(pi_layer* const* layers, int Lc, void* x_inout, i
   return PI_OK;
 }
 
-// A share of the expected active records per block at batch B (from the firing
-// frequencies of the reorder): every block keeps that many of its own before balancing,
-// so their records can be fetched while the balancing exchange runs.  Below the balanced
-// target (the mean count) the floor does not change the assignment, so it sits just
-// under the expected mean.
+// Per-batch tables from the firing frequencies of the reorder.  The keep floor is a share
+// of the expected active records per block at batch B: every block keeps that many of its
+// own before balancing, so their records can be fetched while the balancing exchange
+// runs.  Below the balanced target (the mean count) the floor does not change the
+// assignment, so it sits just under the expected mean.  The hot-prefix lengths are the
+// scans of hot_len_scan.
 constexpr double kKeepShare = 0.85;
-void set_keep_floor(pi_layer* L) {
+void set_batch_tables(pi_layer* L) {
   for (int B = 1; B <= 4; ++B) {
     double expect = 0.0;
     for (int i = 0; i < L->desc.d_ff; ++i) expect += 1.0 - std::pow(1.0 - (double)L->freq_host[i], (double)B);
     L->keep_floor[B - 1] = (int)(kKeepShare * expect / L->G);
   }
+  for (int B = 1; B <= 32; ++B) L->hot_len_b[B] = hot_len_scan(L, B);
 }
 
 LayerDev dev_view(const pi_layer* L, int B = 0) {
@@ -388,7 +394,7 @@ pi_status pi_reorder_hot_prefix(pi_layer* L, const float* freq, int hot_count, c
   if (fh && cudaMemcpy(fh, L->freq_sorted, (size_t)F * 4, cudaMemcpyDeviceToHost) == cudaSuccess) {
     delete[] L->freq_host;
     L->freq_host = fh;
-    set_keep_floor(L);
+    set_batch_tables(L);
   } else {
     delete[] fh;
   }

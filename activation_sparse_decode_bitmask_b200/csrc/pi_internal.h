@@ -64,6 +64,7 @@ struct pi_layer {
   float* freq_host;    // host copy of freq_sorted (descending), or null
   int keep_floor[4];   // per batch 1..4: own records every block keeps before balancing
   int hot_count;    // -1: derived per batch from freq_sorted
+  int hot_len_b[33];   // per batch 1..32: hot-prefix length (set with freq_host)
   int device;
 };
 
