@@ -70,7 +70,7 @@ extern "C" {
 typedef enum {
   PI_OK = 0,
   PI_ERR_ARG = 1,          /* bad pointer, size, shape or combination */
-  PI_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+  PI_ERR_UNSUPPORTED = 2,  /* valid request the library does not implement */
   PI_ERR_OOM = 3,          /* device allocation failed */
   PI_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, copy, sync) */
   PI_ERR_TIMEOUT = 5,      /* a device-side wait gave up (see pi_stream_status) */

@@ -84,7 +84,7 @@ def predictor_logits(x: np.ndarray, p1: np.ndarray, p2: np.ndarray,
     [UAI] §"Prediktor Kepadatan Adaptif": each layer has a small predictor, kept on
     the GPU, that says which neurons will be active; only those are processed.  The
     pages give no architecture; the linear low-rank form with a per-neuron threshold
-    is this build's reading.
+    is the reading taken here.
     """
     x = np.atleast_2d(np.asarray(x, np.float64))
     u = x @ p1
