@@ -134,7 +134,7 @@ def compact(words: np.ndarray, f: int):
 def _preacts(x: np.ndarray, w: Dict[str, np.ndarray], act: str, rows):
     """Per-token pre-activations of the given neuron rows (fp64)."""
     up = x @ w["w_up"][rows].T
-    if act == "relu":
+    if act in ("relu", "relu2"):
         return up + w["bias"][rows], None
     gate = x @ w["w_gate"][rows].T
     return gate + w["bias"][rows], up
@@ -143,6 +143,7 @@ def _preacts(x: np.ndarray, w: Dict[str, np.ndarray], act: str, rows):
 def activations(x: np.ndarray, w: Dict[str, np.ndarray], act: str,
                 rows: np.ndarray) -> np.ndarray:
     """a[b, k] for neuron rows[k].  ReLU: max(0, up + b).  ReGLU: max(0, gate + b) * up.
+    Squared ReLU ("relu2"): max(0, up + b)^2.
 
     [GN] §"Kısıtlar ve SSS": only ReLU / ReGLU / squared-ReLU models are supported,
     because those activations give exact zeros that can be skipped.
@@ -151,6 +152,8 @@ def activations(x: np.ndarray, w: Dict[str, np.ndarray], act: str,
     a = np.maximum(fire, 0.0)
     if act == "reglu":
         a = a * up
+    elif act == "relu2":
+        a = a * a
     return a
 
 
@@ -180,7 +183,7 @@ def sparse_ffn(x: np.ndarray, w: Dict[str, np.ndarray], act: str,
 
 
 def dense_ffn(x: np.ndarray, w: Dict[str, np.ndarray], act: str) -> np.ndarray:
-    """The dense ReLU/ReGLU FFN: every neuron, no predictor."""
+    """The dense FFN (ReLU, ReGLU or squared ReLU): every neuron, no predictor."""
     f = w["bias"].shape[0]
     rows = np.arange(f)
     return down_accumulate(activations(np.atleast_2d(x), w, act, rows), w["w_down"], rows)

@@ -16,6 +16,8 @@ def _pins():
     yield lambda: P.test_brute_force_exact("reglu", 1)
     yield P.test_relu_single_neuron_by_hand
     yield P.test_reglu_single_neuron_by_hand
+    yield P.test_relu2_single_neuron_by_hand
+    yield lambda: P.test_brute_force_exact("relu2", 2)
     yield P.test_one_hot_input_selects_predictor_row
     yield P.test_logit_zero_is_inactive
     yield P.test_batch_masks_apply_per_token
@@ -59,6 +61,18 @@ def _mut_act_bias_on_up(x, w, act, rows):
     gate = x @ w["w_gate"][rows].T
     up = x @ w["w_up"][rows].T + w["bias"][rows]
     return np.maximum(gate, 0.0) * up
+
+
+def _mut_relu2_unsquared(x, w, act, rows):
+    return _orig["activations"](x, w, "relu" if act == "relu2" else act, rows)
+
+
+def _mut_relu2_square_before_clamp(x, w, act, rows):
+    if act != "relu2":
+        return _orig["activations"](x, w, act, rows)
+    x = np.atleast_2d(x)
+    pre = x @ w["w_up"][rows].T + w["bias"][rows]
+    return pre * pre
 
 
 def _mut_sparse_ignores_token_mask(x, w, act, masks, idx):
@@ -114,6 +128,8 @@ MUTANTS = {
     "act without bias": ("activations", _mut_act_no_bias),
     "reglu relu on up": ("activations", _mut_act_relu_on_up),
     "reglu bias on up": ("activations", _mut_act_bias_on_up),
+    "relu2 not squared": ("activations", _mut_relu2_unsquared),
+    "relu2 squared before the clamp": ("activations", _mut_relu2_square_before_clamp),
     "token mask ignored": ("sparse_ffn", _mut_sparse_ignores_token_mask),
     "mask words msb-first": ("pack_mask", _mut_pack_msb),
     "compact intersection": ("compact", _mut_compact_intersection),

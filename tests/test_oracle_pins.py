@@ -43,6 +43,8 @@ def brute_act(x_row, w, act, i):
     up = sum((Fr(w["w_up"][i, j]) * Fr(x_row[j]) for j in range(d)), Fr(0))
     if act == "relu":
         return max(Fr(0), up + Fr(w["bias"][i]))
+    if act == "relu2":
+        return max(Fr(0), up + Fr(w["bias"][i])) ** 2
     gate = sum((Fr(w["w_gate"][i, j]) * Fr(x_row[j]) for j in range(d)), Fr(0))
     return max(Fr(0), gate + Fr(w["bias"][i])) * up
 
@@ -58,7 +60,7 @@ def brute_y(x_row, w, act, active):
     return out
 
 
-@pytest.mark.parametrize("act", ["relu", "reglu"])
+@pytest.mark.parametrize("act", ["relu", "reglu", "relu2"])
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_brute_force_exact(act, seed):
     w, x = tiny_layer(act, seed)
@@ -106,6 +108,20 @@ def test_relu_single_neuron_by_hand():
     assert np.array_equal(y, np.zeros((1, 4)))
 
 
+def test_relu2_single_neuron_by_hand():
+    w = _one_neuron_layer("relu")
+    x = np.array([[1.0, 1.0, 2.0, 0.5]])
+    # up + bias = 1.25 as in the ReLU case; squared -> 1.5625
+    y = O.sparse_ffn(x, w, "relu2", np.ones((1, 32), bool), np.array([5]))
+    assert np.array_equal(y, [[3.125, 0.0, -1.5625, 6.25]])
+    # below the kink the square of the ReLU is still exactly zero
+    y = O.sparse_ffn(-x, w, "relu2", np.ones((1, 32), bool), np.array([5]))
+    assert np.array_equal(y, np.zeros((1, 4)))
+    # a pre-activation under 1 shrinks: (0.5)^2 = 0.25
+    x3 = np.array([[0.0, 0.0, 0.0, 0.25]])   # up = 0.75, + bias -> 0.5
+    assert O.activations(x3, w, "relu2", np.array([5]))[0, 0] == 0.25
+
+
 def test_reglu_single_neuron_by_hand():
     w = _one_neuron_layer("reglu")
     x = np.array([[2.0, 1.0, 0.0, -1.0]])
@@ -147,7 +163,7 @@ def test_batch_masks_apply_per_token():
 
 
 # ----------------------------------------------------------------- invariants
-@pytest.mark.parametrize("act", ["relu", "reglu"])
+@pytest.mark.parametrize("act", ["relu", "reglu", "relu2"])
 def test_sparse_equals_dense_with_true_mask(act):
     """Skipped neurons contribute exact zeros, so with the true mask the sparse FFN
     is bit-identical to the dense one (unite.ai "PowerInfer: Mesin Inferensi LLM Cepat dengan GPU Konsumen",
