@@ -22,7 +22,7 @@ class Workload:
     d_model: int
     d_ff: int
     rank: int
-    act: str                 # "relu" (bias on up) or "reglu" (bias on gate)
+    act: str                 # "relu" or "relu2" (bias on up), or "reglu" (bias on gate)
     w_dtype: str             # "f32" | "f16" | "q4_0"
     x_dtype: str             # "f32" | "f16"
     p_dtype: str             # "f32" | "f16"
