@@ -271,9 +271,12 @@ pi_status pi_sparse_ffn(const pi_layer* layer, const void* x, int B, const uint3
                         pi_workspace* ws, cudaStream_t stream);
 
 /* A whole decode step through L layers: predictor, compaction, sparse FFN and stack
- * glue for each layer. One persistent kernel runs on the device and the host does not
- * synchronise inside. x_inout: device [B][d] in the activation dtype. It holds x_0
- * on entry and x_L on return. All layers must share one descriptor. trace may be NULL. */
+ * glue for each layer. At 1-4 tokens, when the layer fits the persistent kernel, one
+ * launch runs the whole step. Otherwise (5-32 tokens, or layers too wide for it) each
+ * layer runs a fixed sequence of kernels: tensor-core row tiles for the predictor and
+ * gate/up, compaction, the down columns and the glue. The host does not synchronise
+ * inside either way. x_inout: device [B][d] in the activation dtype. It holds x_0 on
+ * entry and x_L on return. All layers must share one descriptor. trace may be NULL. */
 pi_status pi_decode_stack(pi_layer* const* layers, int L, void* x_inout, int B,
                           const pi_trace* trace, pi_workspace* ws, cudaStream_t stream);
 
