@@ -19,7 +19,13 @@ def declared_functions():
 
 @pytest.fixture(scope="module")
 def lib():
-    from activation_sparse_decode_bitmask_b200 import _build
+    # the build script is loaded by path: importing the package loads libpi.so, which
+    # fails when an older library lacks a symbol the binding binds
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_pi_build_for_tests", os.path.join(ROOT, "activation_sparse_decode_bitmask_b200", "_build.py"))
+    _build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(_build)
     path = _build.build()
     return ctypes.CDLL(path), path
 
