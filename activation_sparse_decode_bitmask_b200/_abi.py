@@ -84,7 +84,10 @@ def _load() -> ctypes.CDLL:
         "pi_kernel_launches": (ctypes.c_ulonglong, []),
     }
     for name, (res, args) in sig.items():
-        fn = getattr(lib, name)
+        try:
+            fn = getattr(lib, name)
+        except AttributeError as e:
+            raise ImportError(f"{_build.LIB} lacks {name}; rebuild it with __graft_entry__.build()") from e
         fn.restype = res
         fn.argtypes = args
     return lib
