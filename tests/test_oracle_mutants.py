@@ -5,10 +5,12 @@ import pytest
 
 from oracle import ffn as O
 import test_oracle_pins as P
+import test_oracle_stack_pins as SP
 
 _orig = {name: getattr(O, name) for name in
          ("predictor_logits", "fire_bits", "activations", "sparse_ffn", "pack_mask",
-          "compact", "q4_0_unpack", "stack_glue", "hot_order", "down_accumulate")}
+          "compact", "q4_0_unpack", "stack_glue", "hot_order", "down_accumulate",
+          "layer_weights_f64", "layer_step", "decode_stack")}
 
 
 def _pins():
@@ -29,6 +31,11 @@ def _pins():
     yield P.test_stack_glue_closed_form
     yield P.test_hot_order_and_prefix
     yield P.test_permuted_layer_same_output
+    yield SP.test_q4_down_plane_is_transposed
+    yield SP.test_q4_layer_output_by_hand
+    yield lambda: SP.test_two_layer_two_token_stack("relu")
+    yield lambda: SP.test_two_layer_two_token_stack("reglu")
+    yield SP.test_layer_step_record
 
 
 def _mut_logits_plus_t(x, p1, p2, t):
@@ -122,7 +129,39 @@ def _mut_down_reverse(a, w_down, rows):
     return _orig["down_accumulate"](a[:, ::-1], w_down, list(rows))
 
 
+def _mut_q4_down_not_transposed(t, act):
+    out = _orig["layer_weights_f64"](t, act)
+    if "q_down" in t:
+        out["w_down"] = O.q4_0_unpack(t["q_down"], t["s_down"])
+    return out
+
+
+def _mut_step_union_bits(x, w, act, x_dtype):
+    f = w["bias"].shape[0]
+    logits = O.predictor_logits(x, w["p1"], w["p2"], w["thresh"])
+    bits = O.fire_bits(logits)
+    words = O.pack_mask(bits)
+    idx, count = O.compact(words, f)
+    union = np.broadcast_to(np.atleast_2d(bits).any(axis=0), np.atleast_2d(bits).shape)
+    y = O.sparse_ffn(x, w, act, union, idx)
+    return {"logits": logits, "bits": bits, "words": words, "idx": idx, "count": count, "y": y,
+            "x_next": O.stack_glue(x, y, x_dtype)}
+
+
+def _mut_stack_keeps_x_in(x0, layers, act, x_dtype):
+    x = np.atleast_2d(x0)
+    trace = []
+    for w in layers:
+        rec = O.layer_step(x, w, act, x_dtype)
+        rec["x_in"] = x
+        trace.append(rec)
+    return trace
+
+
 MUTANTS = {
+    "q4 down plane not transposed": ("layer_weights_f64", _mut_q4_down_not_transposed),
+    "union mask as per-token bits": ("layer_step", _mut_step_union_bits),
+    "next layer gets x_in": ("decode_stack", _mut_stack_keeps_x_in),
     "logit +t": ("predictor_logits", _mut_logits_plus_t),
     "fire >=": ("fire_bits", _mut_fire_ge),
     "act without bias": ("activations", _mut_act_no_bias),
