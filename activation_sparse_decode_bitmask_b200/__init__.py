@@ -5,7 +5,7 @@ include/pi_sparse_ffn.h (libpi.so).  This package is the thin Python binding: it
 torch tensors' device pointers and the current stream to the library.  It has no CPU or
 PyTorch fallback; importing it fails if libpi.so has not been built.
 """
-from ._abi import (PI_F16, PI_F32, PI_MAX_BATCH, PI_NOALLOC_SCRATCH_BYTES, PI_Q4_0, PI_RELU, PI_REGLU, EXPORTS,
+from ._abi import (PI_F16, PI_F32, PI_MAX_BATCH, PI_NOALLOC_SCRATCH_BYTES, PI_Q4_0, PI_RELU, PI_RELU2, PI_REGLU, EXPORTS,
                    Layer, LayerDesc, LayerWeights, PiError, Trace, Workspace, abi_version, compact_active,
                    decode_stack, decode_stack_host, diag_barrier_timeout, get_perm, kernel_launches, lib, load_layer,
                    make_desc, predict, predict_noalloc, reorder_hot_prefix, sparse_ffn, status_str)

@@ -16,7 +16,7 @@ import torch
 from . import _build
 
 PI_F32, PI_F16, PI_Q4_0 = 0, 1, 2
-PI_RELU, PI_REGLU = 0, 1
+PI_RELU, PI_REGLU, PI_RELU2 = 0, 1, 2
 PI_MAX_BATCH = 32
 PI_NOALLOC_SCRATCH_BYTES = 256 * 1024
 DIAG_SLOTS = 64   # diagnostic stamps per block and layer
@@ -121,7 +121,7 @@ def _stream(stream=None) -> int:
 
 
 _DT = {"f32": PI_F32, "f16": PI_F16, "q4_0": PI_Q4_0}
-_ACT = {"relu": PI_RELU, "reglu": PI_REGLU}
+_ACT = {"relu": PI_RELU, "reglu": PI_REGLU, "relu2": PI_RELU2}
 
 
 def make_desc(d_model: int, d_ff: int, rank: int, act: str, w_dtype: str, x_dtype: str,

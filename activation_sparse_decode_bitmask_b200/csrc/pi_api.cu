@@ -45,7 +45,7 @@ int smem_optin(int dev) {
 }
 
 pi_status check_desc(const pi_layer_desc& d) {
-  if (d.act != PI_RELU && d.act != PI_REGLU) return PI_ERR_ARG;
+  if (d.act != PI_RELU && d.act != PI_REGLU && d.act != PI_RELU2) return PI_ERR_ARG;
   if ((unsigned)d.w_dtype > PI_Q4_0 || (unsigned)d.x_dtype > PI_Q4_0 || (unsigned)d.p_dtype > PI_Q4_0) return PI_ERR_ARG;
   if (d.d_model <= 0 || d.d_ff < 32 || d.rank <= 0) return PI_ERR_ARG;
   if (d.d_ff % 32 || d.d_model % 64 || d.rank % 8 || d.rank > d.d_model) return PI_ERR_ARG;
@@ -80,49 +80,46 @@ void free_layer_buffers(pi_layer* L) {
   L->freq_host = nullptr;
 }
 
+// Bytes of bulk copies each block of the fused kernel keeps in flight: enough to keep its
+// share of HBM busy (about the SM's share of bandwidth times the unloaded latency), and no
+// more, since every byte beyond that only lengthens the queue the exchange words wait in.
+// PI_FUSED_INFLIGHT_KB in the environment (read once) overrides the default of 64 KB.
+int inflight_budget_bytes() {
+  static const int v = [] {
+    const char* e = std::getenv("PI_FUSED_INFLIGHT_KB");
+    const int kb = e ? std::atoi(e) : 0;
+    return (kb > 0 && kb <= 4096 ? kb : 64) * 1024;
+  }();
+  return v;
+}
+
 // Geometry of the fused kernel for one layer shape.
-pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedParams& p, size_t& smem) {
+// r_max: the largest predictor rank of the launch's layers (the layer's own when <= 0).
+pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedParams& p, size_t& smem, int r_max = 0) {
   const pi_layer_desc& d = L->desc;
   std::memset(&p, 0, sizeof(p));
-  p.B = B; p.d = d.d_model; p.f = d.d_ff; p.r = d.rank;
+  p.B = B; p.d = d.d_model; p.f = d.d_ff; p.r = r_max > 0 ? r_max : d.rank;
+  if (p.r > 3072) return PI_ERR_UNSUPPORTED;   // the u exchange polls at most 3072 words per token
   p.grid = ws->grid;
   p.row_bytes = L->row_bytes; p.rec_stride = L->rec_stride;
-  p.gate_off = L->gate_off; p.up_off = L->up_off; p.down_off = L->down_off; p.bias_off = L->bias_off;
-  p.p1_row = L->p1_row; p.p2_stride = L->p2_stride;
+  p.gate_off = L->gate_off; p.up_off = L->up_off; p.bias_off = L->bias_off;
+  p.dn_stride = L->dn_stride; p.dn_off = (long long)L->dn_off;
+  p.p1_row = L->p1_row; p.p2_stride = p2_stride_of(p.r, L->family == FAM_F32 ? 4 : 2);
   p.nown_max = L->nown_max;
-  const int ngroups = d.d_model / 32;
-  p.nslices = std::min(ws->grid, ngroups);
-  if ((ngroups + p.nslices - 1) / p.nslices > 4) return PI_ERR_UNSUPPORTED;
+  p.act_square = d.act == PI_RELU2;
   if (L->G != ws->grid) return PI_ERR_ARG;   // layer laid out for another device
   if (L->nown_max > kMaxOwn) return PI_ERR_UNSUPPORTED;
   if (!fused_supported(L->family, B, d.d_model)) return PI_ERR_UNSUPPORTED;
-  const size_t budget = (size_t)smem_optin(ws->device);
-  const size_t fixed = fused_fixed_smem(B, d.d_model, d.rank, ws->grid, L->nown_max, L->family);
-  if (budget <= fixed) return PI_ERR_UNSUPPORTED;
-  p.ring_bytes = (int)((budget - fixed) / 128 * 128);
-  // ring items: whole neuron records; P1^T rows grouped into ~32 KB copies; the block's
-  // own P2 rows in as few copies as fit twice in the ring (up to 96 KB each), so that
-  // every consumer warp has rows to work on in the logits pass
-  const int cap = std::max(L->rec_stride, 32 * 1024);
-  const int cap_p2 = std::max(cap, std::min(96 * 1024, p.ring_bytes / 2 - 128));
-  p.p1_rows_per_item = std::max(1, cap / L->p1_row);
-  p.p2_rows_per_item = std::max(1, std::min(L->nown_max, cap_p2 / L->p2_stride));
-  const long long max_item = std::max({(long long)L->rec_stride, (long long)p.p1_rows_per_item * L->p1_row,
-                                       (long long)p.p2_rows_per_item * L->p2_stride});
-  if (p.ring_bytes < 2 * max_item || max_item >= (1 << 20)) return PI_ERR_UNSUPPORTED;
-  // records outstanding at once: floor(ring / stride) - 1 (an item never wraps); the F
-  // phase needs room for at least two records beside the one it waits for
-  p.rec_window = p.ring_bytes / L->rec_stride - 2;
-  if (p.rec_window < 1) return PI_ERR_UNSUPPORTED;
-  smem = fixed + (size_t)p.ring_bytes;
+  if (!fused_plan_smem(p, L->family, (size_t)smem_optin(ws->device), smem)) return PI_ERR_UNSUPPORTED;
   // ws fields
-  p.ux = ws->ux; p.px = ws->px; p.vx = ws->vx; p.sx = ws->sx; p.cx = ws->cx; p.lx = ws->lx;
+  p.ux = ws->ux; p.mx = ws->mx; p.hx = ws->hx; p.vx = ws->vx; p.sx = ws->sx;
   p.bar = ws->bar; p.err = ws->err; p.active_total = ws->active_total;
   p.layer_count = nullptr;
   p.barrier_timeout_ns = kDefaultWaitNs;
   p.wait_cycles = kDefaultWaitNs * 3;   // cycles at up to 3 GHz: at least the nominal budget
   p.barrier_extra = 0;
   p.poll_ns = 64;          // back-off between exchange polling rounds
+  p.inflight_budget = inflight_budget_bytes();
   return PI_OK;
 }
 
@@ -133,27 +130,14 @@ pi_status check_ws(const pi_workspace* ws, const pi_layer_desc& d, int B, int L)
   return PI_OK;
 }
 
-// Hot-prefix length at batch B: the neurons (in hot order) whose union firing probability
-// 1 - (1 - f)^B is at least 1/2, or the count fixed by pi_reorder_hot_prefix.  Computed
-// once per batch size when the frequencies arrive (the scan would otherwise run for every
-// layer of every call).
-int hot_len_scan(const pi_layer* L, int B) {
-  if (L->hot_count >= 0) return L->hot_count;
-  int n = 0;
-  const int F = L->desc.d_ff;
-  while (n < F && 1.0 - std::pow(1.0 - (double)L->freq_host[n], (double)B) >= 0.5) ++n;
-  return n;
-}
-int hot_len(const pi_layer* L, int B) {
-  return (L->freq_host && B >= 1 && B <= 32) ? L->hot_len_b[B] : 0;
-}
-
 BatchedLayer bview(const pi_layer* L) {
   BatchedLayer b;
   b.d = L->desc.d_model; b.f = L->desc.d_ff; b.r = L->desc.rank; b.G = L->G; b.nown_max = L->nown_max;
-  b.rec = L->rec; b.rec_stride = L->rec_stride; b.up_off = L->up_off; b.gate_off = L->gate_off; b.down_off = L->down_off;
+  b.rec = L->rec; b.rec_stride = L->rec_stride; b.up_off = L->up_off; b.gate_off = L->gate_off;
+  b.dn = L->rec + L->dn_off; b.dn_stride = L->dn_stride;
   b.p1t = L->p1t; b.p1_row = L->p1_row; b.p2o = L->p2o; b.p2_stride = L->p2_stride;
   b.thresh = L->thresh; b.bias = L->bias;
+  b.act_square = L->desc.act == PI_RELU2;
   return b;
 }
 // Calls the fused kernel does not serve take the batched path: more than 4 tokens, or
@@ -171,7 +155,8 @@ pi_status decode_stack_batched(pi_layer* const* layers, int Lc, void* x_inout, i
                                pi_workspace* ws, cudaStream_t stream) {
   const pi_layer* L0 = layers[0];
   const int d = L0->desc.d_model, f = L0->desc.d_ff, words = f / 32;
-  if (!batched_supported(L0->family, B, d, L0->desc.rank) || !ws->u_hi) return PI_ERR_UNSUPPORTED;
+  for (int l = 0; l < Lc; ++l)
+    if (!batched_supported(L0->family, B, d, layers[l]->desc.rank) || !ws->u_hi) return PI_ERR_UNSUPPORTED;
   if (trace && (trace->idx || trace->count) && !(trace->idx && trace->count && trace->mask)) return PI_ERR_ARG;
   PI_TRY(cudaMemsetAsync(ws->layer_count, 0, (size_t)Lc * 4, stream));
   if (trace && trace->x)
@@ -195,12 +180,11 @@ pi_status decode_stack_batched(pi_layer* const* layers, int Lc, void* x_inout, i
   return PI_OK;
 }
 
-// Per-batch tables from the firing frequencies of the reorder.  The keep floor is a share
-// of the expected active records per block at batch B: every block keeps that many of its
-// own before balancing, so their records can be fetched while the balancing exchange
-// runs.  Below the balanced target (the mean count) the floor does not change the
-// assignment, so it sits just under the expected mean.  The hot-prefix lengths are the
-// scans of hot_len_scan.
+// Per-batch keep floors from the firing frequencies of the reorder: a share of the
+// expected active records per block at batch B.  Every block keeps that many of its own
+// active neurons whatever the counts say, so their records are fetched while the mask
+// exchange runs.  Below the balanced target (the mean count) the floor does not change
+// the assignment, so it sits just under the expected mean.
 constexpr double kKeepShare = 0.85;
 void set_batch_tables(pi_layer* L) {
   for (int B = 1; B <= 4; ++B) {
@@ -208,16 +192,16 @@ void set_batch_tables(pi_layer* L) {
     for (int i = 0; i < L->desc.d_ff; ++i) expect += 1.0 - std::pow(1.0 - (double)L->freq_host[i], (double)B);
     L->keep_floor[B - 1] = (int)(kKeepShare * expect / L->G);
   }
-  for (int B = 1; B <= 32; ++B) L->hot_len_b[B] = hot_len_scan(L, B);
 }
 
 LayerDev dev_view(const pi_layer* L, int B = 0) {
-  return LayerDev{L->rec, L->p1t, L->p2o, B > 0 ? hot_len(L, B) : 0, B > 0 ? L->keep_floor[std::min(B, 4) - 1] : 0};
+  return LayerDev{L->rec, L->p1t, L->p2o, B > 0 ? L->keep_floor[std::min(B, 4) - 1] : 0, L->desc.rank};
 }
 
-bool same_desc(const pi_layer_desc& a, const pi_layer_desc& b) {
-  return a.d_model == b.d_model && a.d_ff == b.d_ff && a.rank == b.rank && a.act == b.act &&
-         a.w_dtype == b.w_dtype && a.x_dtype == b.x_dtype && a.p_dtype == b.p_dtype;
+// Layers of one stack share everything but the predictor rank, which may differ per layer.
+bool same_desc_but_rank(const pi_layer_desc& a, const pi_layer_desc& b) {
+  return a.d_model == b.d_model && a.d_ff == b.d_ff && a.act == b.act && a.w_dtype == b.w_dtype &&
+         a.x_dtype == b.x_dtype && a.p_dtype == b.p_dtype;
 }
 
 }  // namespace
@@ -274,12 +258,12 @@ pi_status pi_load_layer(const pi_layer_desc* desc, const pi_layer_weights* w, cu
   const int D = d.d_model, F = d.d_ff, R = d.rank;
   const int pb = wbytes(fam == FAM_Q4 ? FAM_F16 : fam);
   L->row_bytes = fam == FAM_Q4 ? round16((long long)D / 2 + D / 16) : D * wbytes(fam);
-  const int nrows = reglu ? 3 : 2;
-  L->rec_stride = L->row_bytes * nrows + 16;   // rows, then a 16-byte header with the bias
+  L->rec_stride = L->row_bytes * (reglu ? 2 : 1) + 16;   // gate?, up, then a 16-byte header with the bias
   L->gate_off = reglu ? 0 : -1;
   L->up_off = reglu ? L->row_bytes : 0;
-  L->down_off = L->up_off + L->row_bytes;
-  L->bias_off = L->down_off + L->row_bytes;
+  L->bias_off = L->up_off + L->row_bytes;
+  L->dn_stride = L->row_bytes;
+  L->dn_off = (size_t)d.d_ff * L->rec_stride;
   L->p1_row = D * pb;
   L->p2_stride = round16((long long)R * pb + 8);
   L->G = sm_count(L->device);
@@ -287,7 +271,8 @@ pi_status pi_load_layer(const pi_layer_desc* desc, const pi_layer_weights* w, cu
   L->nown_max = (F + L->G - 1) / L->G;
 
   auto fail = [&](pi_status s) { free_layer_buffers(L); delete L; return s; };
-  if (dmalloc(&L->rec, (size_t)F * L->rec_stride) != cudaSuccess) return fail(PI_ERR_OOM);
+  const size_t rec_bytes = L->dn_off + (size_t)F * L->dn_stride;
+  if (dmalloc(&L->rec, rec_bytes) != cudaSuccess) return fail(PI_ERR_OOM);
   if (dmalloc(&L->p1t, (size_t)R * L->p1_row) != cudaSuccess) return fail(PI_ERR_OOM);
   if (dmalloc(&L->p2o, (size_t)L->G * L->nown_max * L->p2_stride) != cudaSuccess) return fail(PI_ERR_OOM);
   if (dmalloc(&L->bias, (size_t)F * 4) != cudaSuccess) return fail(PI_ERR_OOM);
@@ -296,23 +281,25 @@ pi_status pi_load_layer(const pi_layer_desc* desc, const pi_layer_weights* w, cu
 
   cudaError_t e = cudaSuccess;
   auto step = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
-  step(cudaMemsetAsync(L->rec, 0, (size_t)F * L->rec_stride, stream));
+  step(cudaMemsetAsync(L->rec, 0, rec_bytes, stream));
   step(cudaMemsetAsync(L->p2o, 0, (size_t)L->G * L->nown_max * L->p2_stride, stream));
   if (fam == FAM_Q4) {
     const int nb = D / 32;
     const void* nib[3] = {w->w_gate, w->w_up, w->w_down};
     const void* scl[3] = {w->s_gate, w->s_up, w->s_down};
-    const int off[3] = {L->gate_off, L->up_off, L->down_off};
+    uint8_t* const base[3] = {L->rec, L->rec, L->rec + L->dn_off};
+    const int stride[3] = {L->rec_stride, L->rec_stride, L->dn_stride};
+    const int off[3] = {L->gate_off, L->up_off, 0};
     for (int m = reglu ? 0 : 1; m < 3; ++m) {
-      step(relayout_copy_rows(nib[m], nb * 16, 0, L->rec, L->rec_stride, off[m], F, nb * 16, nullptr, stream));
-      step(relayout_copy_rows(scl[m], nb * 2, 0, L->rec, L->rec_stride, off[m] + D / 2, F, nb * 2, nullptr, stream));
+      step(relayout_copy_rows(nib[m], nb * 16, 0, base[m], stride[m], off[m], F, nb * 16, nullptr, stream));
+      step(relayout_copy_rows(scl[m], nb * 2, 0, base[m], stride[m], off[m] + D / 2, F, nb * 2, nullptr, stream));
     }
   } else {
     const int wb = wbytes(fam);
     if (reglu) step(relayout_copy_rows(w->w_gate, (long long)D * wb, 0, L->rec, L->rec_stride, L->gate_off, F, D * wb, nullptr, stream));
     step(relayout_copy_rows(w->w_up, (long long)D * wb, 0, L->rec, L->rec_stride, L->up_off, F, D * wb, nullptr, stream));
     // down: caller's [d x f] row-major -> neuron-major rows
-    step(relayout_transpose(w->w_down, wb, D, F, F, L->rec, L->rec_stride, L->down_off, stream));
+    step(relayout_transpose(w->w_down, wb, D, F, F, L->rec + L->dn_off, L->dn_stride, 0, stream));
   }
   // P1 [d x r] -> P1^T [r x d];  P2 [r x f] -> per-neuron rows [f][r] + (t, b)
   step(relayout_transpose(w->p1, pb, D, R, R, L->p1t, L->p1_row, 0, stream));
@@ -359,7 +346,8 @@ pi_status pi_reorder_hot_prefix(pi_layer* L, const float* freq, int hot_count, c
     cudaFree(order); cudaFree(bad); cudaFree(rec); cudaFree(p2o); cudaFree(bias); cudaFree(thresh);
     cudaFree(fs); cudaFree(perm);
   };
-  if (dmalloc(&order, (size_t)F * 4) || dmalloc(&bad, 4) || dmalloc(&rec, (size_t)F * L->rec_stride) ||
+  const size_t rec_bytes = L->dn_off + (size_t)F * L->dn_stride;
+  if (dmalloc(&order, (size_t)F * 4) || dmalloc(&bad, 4) || dmalloc(&rec, rec_bytes) ||
       dmalloc(&p2o, p2_bytes) || dmalloc(&bias, (size_t)F * 4) || dmalloc(&thresh, (size_t)F * 4) ||
       dmalloc(&fs, (size_t)F * 4) || dmalloc(&perm, (size_t)F * 4)) {
     cleanup();
@@ -375,6 +363,8 @@ pi_status pi_reorder_hot_prefix(pi_layer* L, const float* freq, int hot_count, c
   if (e != cudaSuccess) { cleanup(); return cuda_status(e); }
   if (hbad) { cleanup(); return PI_ERR_ARG; }
   step(relayout_copy_rows(L->rec, L->rec_stride, 0, rec, L->rec_stride, 0, F, L->rec_stride, order, stream));
+  step(relayout_copy_rows(L->rec + L->dn_off, L->dn_stride, 0, rec + L->dn_off, L->dn_stride, 0, F, L->dn_stride, order,
+                          stream));
   step(cudaMemsetAsync(p2o, 0, p2_bytes, stream));
   step(gather_owner_rows(L->p2o, p2o, order, F, L->G, L->nown_max, L->p2_stride, stream));
   step(gather_f32(L->bias, order, F, bias, stream));
@@ -418,11 +408,12 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
   if (ws->grid <= 0) { delete ws; return PI_ERR_CUDA; }
   if (ws->grid > kMaxGrid) { delete ws; return PI_ERR_UNSUPPORTED; }
   const size_t G = ws->grid, Bm = B_max;
+  const size_t mx_bytes = G * 4 * kMaxOwnWords * 8, hx_bytes = (size_t)f_max * Bm * 8;
   bool ok = dmalloc(&ws->ux, Bm * r_max * 8) == cudaSuccess &&
-            dmalloc(&ws->px, G * Bm * d_max * 8) == cudaSuccess &&
+            dmalloc(&ws->mx, mx_bytes) == cudaSuccess &&
+            dmalloc(&ws->hx, hx_bytes) == cudaSuccess &&
             dmalloc(&ws->vx, Bm * d_max * 8) == cudaSuccess &&
             dmalloc(&ws->sx, Bm * G * 16) == cudaSuccess &&
-            dmalloc(&ws->cx, G * 8) == cudaSuccess && dmalloc(&ws->lx, G * kMaxOwn * 8) == cudaSuccess &&
             dmalloc(&ws->bar, 64) == cudaSuccess &&
             dmalloc(&ws->err, 16) == cudaSuccess &&
             dmalloc(&ws->active_total, 16) == cudaSuccess &&
@@ -440,9 +431,9 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
   if (ok) {
     // tagged words start with tag 0; launch epochs start at 1, so no stale word matches
     const uint32_t bar0[4] = {0u, 0u, 1u, 0u};
-    ok = cudaMemset(ws->ux, 0, Bm * r_max * 8) == cudaSuccess && cudaMemset(ws->px, 0, G * Bm * d_max * 8) == cudaSuccess &&
+    ok = cudaMemset(ws->ux, 0, Bm * r_max * 8) == cudaSuccess && cudaMemset(ws->mx, 0, mx_bytes) == cudaSuccess &&
+         cudaMemset(ws->hx, 0, hx_bytes) == cudaSuccess &&
          cudaMemset(ws->vx, 0, Bm * d_max * 8) == cudaSuccess && cudaMemset(ws->sx, 0, Bm * G * 16) == cudaSuccess &&
-         cudaMemset(ws->cx, 0, G * 8) == cudaSuccess && cudaMemset(ws->lx, 0, G * kMaxOwn * 8) == cudaSuccess &&
          cudaMemset(ws->bar, 0, 64) == cudaSuccess &&
          cudaMemcpy(ws->bar, bar0, sizeof(bar0), cudaMemcpyHostToDevice) == cudaSuccess &&
          cudaMemset(ws->err, 0, 16) == cudaSuccess && cudaMemset(ws->active_total, 0, 16) == cudaSuccess &&
@@ -459,7 +450,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
 
 void pi_workspace_free(pi_workspace* ws) {
   if (!ws) return;
-  cudaFree(ws->ux); cudaFree(ws->px); cudaFree(ws->vx); cudaFree(ws->sx); cudaFree(ws->cx); cudaFree(ws->lx);
+  cudaFree(ws->ux); cudaFree(ws->mx); cudaFree(ws->hx); cudaFree(ws->vx); cudaFree(ws->sx);
   cudaFree(ws->bar); cudaFree(ws->err); cudaFree(ws->active_total);
   cudaFree(ws->layer_count); cudaFree(ws->x_dev); cudaFree(ws->phase_clk);
   cudaFree(ws->u_hi); cudaFree(ws->u_lo); cudaFree(ws->bmask); cudaFree(ws->bidx); cudaFree(ws->bcount);
@@ -477,7 +468,7 @@ pi_status pi_stream_status(pi_workspace* ws, cudaStream_t stream) {
   PI_TRY(cudaMemcpy(bar, ws->bar, sizeof(bar), cudaMemcpyDeviceToHost));
   bar[0] = 0u;
   bar[1] = 0u;
-  bar[2] += 1u;   // fresh tags: nothing an aborted launch left behind can match
+  bar[2] = next_launch_epoch(bar[2]);   // fresh tags: nothing an aborted launch left behind can match
   PI_TRY(cudaMemcpy(ws->bar, bar, sizeof(bar), cudaMemcpyHostToDevice));
   PI_TRY(cudaMemset(ws->err, 0, 16));
   PI_TRY(cudaDeviceSynchronize());
@@ -562,17 +553,20 @@ pi_status pi_sparse_ffn(const pi_layer* L, const void* x, int B, const uint32_t*
 pi_status pi_decode_stack(pi_layer* const* layers, int Lc, void* x_inout, int B, const pi_trace* trace,
                           pi_workspace* ws, cudaStream_t stream) {
   if (!layers || Lc < 1 || Lc > kMaxLayers || !x_inout || B < 1 || B > PI_MAX_BATCH) return PI_ERR_ARG;
+  int r_max = 0;
   for (int l = 0; l < Lc; ++l) {
     if (!layers[l]) return PI_ERR_ARG;
-    if (!same_desc(layers[l]->desc, layers[0]->desc)) return PI_ERR_ARG;
+    if (!same_desc_but_rank(layers[l]->desc, layers[0]->desc)) return PI_ERR_ARG;
+    r_max = std::max(r_max, layers[l]->desc.rank);
   }
   const pi_layer* L0 = layers[0];
   pi_status st = check_ws(ws, L0->desc, B, Lc);
   if (st != PI_OK) return st;
+  if (r_max > ws->r_max) return PI_ERR_ARG;
   if (use_batched(L0, B)) return decode_stack_batched(layers, Lc, x_inout, B, trace, ws, stream);
   FusedParams p;
   size_t smem = 0;
-  st = plan_fused(L0, B, ws, p, smem);
+  st = plan_fused(L0, B, ws, p, smem, r_max);
   if (st != PI_OK) return st;
   p.mode = MODE_PREDICT | MODE_FFN | MODE_GLUE;
   p.L = Lc;
@@ -689,7 +683,7 @@ __global__ void noalloc_status_kernel(uint32_t* ctl, int* err, int32_t* status) 
   if (e != 0) {
     ctl[0] = 0u;
     ctl[1] = 0u;
-    ctl[2] += 1u;
+    ctl[2] = next_launch_epoch(ctl[2]);
     *err = 0;
   }
 }
@@ -728,22 +722,23 @@ pi_status pi_predict_noalloc(const pi_layer* L, const void* x, int B, uint32_t* 
   if (L->G != G) return PI_ERR_ARG;   // layer laid out for another device
   const size_t u_bytes = round256((size_t)B * L->desc.rank * 8);
   if (kNoallocCtlBytes + u_bytes > PI_NOALLOC_SCRATCH_BYTES) return PI_ERR_UNSUPPORTED;
-  unsigned char* s = nullptr;
-  pi_status st = noalloc_scratch(dev, stream, &s);
-  if (st != PI_OK) return st;
   pi_workspace w;   // a view of the static scratch; nothing is allocated
   std::memset(&w, 0, sizeof(w));
   w.d_max = L->desc.d_model; w.f_max = L->desc.d_ff; w.r_max = L->desc.rank; w.B_max = B; w.L_max = 1;
   w.grid = G;
   w.device = dev;
-  w.bar = reinterpret_cast<uint32_t*>(s);
-  w.err = reinterpret_cast<int*>(s + 64);
-  w.active_total = reinterpret_cast<unsigned long long*>(s + 128);
-  w.ux = reinterpret_cast<uint64_t*>(s + kNoallocCtlBytes);
+  // the shape check comes first: a refused shape enqueues nothing, not even the set-up
   FusedParams p;
   size_t smem = 0;
-  st = plan_fused(L, B, &w, p, smem);
+  pi_status st = plan_fused(L, B, &w, p, smem);
   if (st != PI_OK) return st;
+  unsigned char* s = nullptr;
+  st = noalloc_scratch(dev, stream, &s);
+  if (st != PI_OK) return st;
+  p.bar = reinterpret_cast<uint32_t*>(s);
+  p.err = reinterpret_cast<int*>(s + 64);
+  p.active_total = reinterpret_cast<unsigned long long*>(s + 128);
+  p.ux = reinterpret_cast<uint64_t*>(s + kNoallocCtlBytes);
   p.mode = MODE_PREDICT;
   p.L = 1;
   p.layers[0] = dev_view(L);
@@ -755,7 +750,7 @@ pi_status pi_predict_noalloc(const pi_layer* L, const void* x, int B, uint32_t* 
   note_launch();
 
   note_launch();
-  noalloc_status_kernel<<<1, 1, 0, stream>>>(w.bar, w.err, status);
+  noalloc_status_kernel<<<1, 1, 0, stream>>>(p.bar, p.err, status);
   PI_TRY(cudaGetLastError());
   return PI_OK;
 }

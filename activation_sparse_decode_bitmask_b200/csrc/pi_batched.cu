@@ -214,6 +214,7 @@ __global__ void __launch_bounds__(32 * kBW) rowtok_kernel(const RowTokArgs a) {
 // (row, token).
 struct RowEpiArgs {
   int mode, nrows_static, B, ksplit, nmat;
+  int squared;                 // ROWS_FFN: squared ReLU
   const int32_t* count;
   const int32_t* idx;
   int f;
@@ -261,7 +262,8 @@ __global__ void __launch_bounds__(256) rowtok_epilogue(const RowEpiArgs a) {
       if (i < 0 || i >= a.f) i = 0;   // reported by the row kernel
       const uint32_t bit = (__ldg(a.mask_in + (size_t)b * (a.f / 32) + (i >> 5)) >> (i & 31)) & 1u;
       const float bi = __ldg(a.bias + i);
-      const float act = (a.nmat == 2) ? fmaxf(v[1] + bi, 0.f) * v[0] : fmaxf(v[0] + bi, 0.f);   // matrix 1: gate
+      float act = (a.nmat == 2) ? fmaxf(v[1] + bi, 0.f) * v[0] : fmaxf(v[0] + bi, 0.f);   // matrix 1: gate
+      if (a.squared) act *= act;   // squared ReLU
       hv = bit ? act : 0.f;
     }
     a.h[(size_t)j * 32 + b] = hv;
@@ -607,6 +609,7 @@ cudaError_t batched_ffn(const BatchedLayer& L, const void* x, int B, const uint3
   ea.idx = idx;
   ea.f = L.f;
   ea.bias = L.bias;
+  ea.squared = L.act_square;
   ea.mask_in = mask;
   ea.h = h;
   cudaError_t e = launch_rows(a, ea, nmat, L.f, part_floats, s);
@@ -616,9 +619,9 @@ cudaError_t batched_ffn(const BatchedLayer& L, const void* x, int B, const uint3
   dn.fmax = L.f;
   dn.d = L.d;
   dn.B = B;
-  dn.rec = L.rec;
-  dn.rec_stride = L.rec_stride;
-  dn.down_off = L.down_off;
+  dn.rec = L.dn;
+  dn.rec_stride = L.dn_stride;
+  dn.down_off = 0;
   dn.idx = idx;
   dn.h = h;
   dn.ypart = ypart;

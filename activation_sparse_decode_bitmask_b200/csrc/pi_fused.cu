@@ -1,27 +1,35 @@
 // The fused persistent kernel of the activation-sparse FFN decode path.
 //
-// One block per SM: 8 consumer warps and 1 producer warp.  The producer streams every
-// byte the block needs from HBM into a byte ring in shared memory, as a few large bulk
-// copies per item: the block's P1^T rows, its own neurons' predictor rows (stored
-// contiguously per block), and one [gate | up | down] record per active neuron it
-// processes.  It runs ahead of the consumers as far as the ring allows, so the next
-// layer's predictor is in flight while the consumers wait on cross-block exchanges.
+// One block per SM: 16 consumer warps and 1 producer warp.  The producer streams the
+// block's predictor rows and the [gate | up | bias] record of every active neuron the
+// block dots from HBM into a byte ring in shared memory, as bulk copies completing on
+// mbarriers.  It runs ahead of the consumers as far as the ring allows, so the next
+// layer's predictor is in flight while the consumers finish the current one.
 //
 // Per layer, for block c of G (stack mode):
-//   P-a  u_k = P1^T[k] . x for the block's rank rows k (one warp per row) -> u exchange
-//   P-b  logit_i = P2^T[i] . u - t_i for the block's own neurons i = c, c+G, c+2G, ...
-//        (8 rows per warp pass); bit = logit > 0
-//   list the block's own active neurons, ascending: nothing is exchanged, so the
-//        producer starts on the records as soon as the block's own bits are known
-//   F    for each of its records: one warp forms the gate/up dot products with x
-//          ReLU : h = max(0, w_up_i . x + b_i)    ReGLU: max(0, w_gate_i . x + b_i) * (w_up_i . x)
-//          h[b] = 0 where token b's bit is 0
-//        then all threads add h * w_down_i into y (registers, fp32, one thread per 16 B)
-//        -> partial exchange
-//   R    block s < nslices owns a column slice: v = x + sum_c partial_c in ascending c,
-//        and the slice's sum and sum of squares -> v / moments exchange
-//   glue x' = (v - mean(v)) / sqrt(var(v) + 1e-6) from the slices' sums and sums of
-//        squares, rounded to the activation dtype
+//   P-a   u_k = P1^T[k] . x for the block's rank rows k -> u exchange
+//   P-b   logit_i = P2^T[i] . u - t_i for the block's own neurons i = c, c+G, c+2G, ...;
+//         bit = logit > 0.  The block lists its own active neurons and hands the first
+//         of them (a floor set from the firing frequencies) to the producer at once.
+//   mask  every block publishes its own bit words; one polling round gives every block
+//         every bit.  From the union counts each block derives the same balanced
+//         assignment: it keeps up to T of its own active neurons and takes the excess of
+//         the blocks above T, so every block dots at most T = max(ceil(N/G), floor).
+//   F     gate/up dot products of the assigned records (a group of warps per record):
+//           ReLU : h = max(0, w_up_i . x + b_i)    ReGLU: max(0, w_gate_i . x + b_i) * (w_up_i . x)
+//           squared ReLU: h = max(0, w_up_i . x + b_i)^2
+//           h[b] = 0 where token b's bit is 0
+//         -> h exchange (one tagged word per neuron and token)
+//   down  block c owns a slice of the d output columns.  While F runs, its threads copy
+//         their slice of every active neuron's down row into shared memory (cp.async);
+//         then y[slice] = sum over the active neurons of h_i * W_down[i][slice], in a fixed
+//         order, and v = x + y with the slice's sum and sum of squares -> v exchange
+//   glue  x' = (v - mean(v)) / sqrt(var(v) + 1e-6) from every slice's v and moments,
+//         rounded to the activation dtype
+// The down projection is column-owned: a block reads only its slice of each active down
+// row, so nothing like a d-long partial sum per block is ever exchanged; the exchanges
+// carry r values (u), f/32 bit words (mask), one value per active neuron (h) and d
+// values (v) per token.
 // Mask words (predict output, trace) are OR-ed in by the owner blocks of their bits.
 // Cross-block exchanges use 64-bit words {tag, value}: a reader polls the words
 // themselves until every tag matches, so data and completion arrive together and no grid
@@ -29,6 +37,7 @@
 // block out), per layer and per exchange.  Every sum runs in a fixed order, so results
 // are bitwise reproducible.
 #include <cuda_fp16.h>
+#include <algorithm>
 #include <cstdint>
 
 #include "pi_internal.h"
@@ -39,43 +48,43 @@ namespace pi {
 
 namespace {
 
-constexpr float kRmsEps = 1e-6f;
+constexpr float kNormEps = 1e-6f;
 constexpr int kRedBar = 1;          // named barrier id among consumers
-constexpr int kMaxColGroups = 4;    // 32-column groups per reduce slice
 constexpr int kItems = 32;          // ring items in flight (mbarrier pairs)
-constexpr int kBalK = 12;           // list entries every block publishes at least (balance)
 constexpr uint32_t kSleepNs = 20000;  // suspend hint of blocking mbarrier waits (wakes on completion)
-constexpr int kHr = 48;             // F h slots: >= kItems + the dot lookahead (16)
+constexpr int kHr = 48;             // F h slots: more than kItems, so a slot is free before its reuse
+constexpr int kMaxDch = 1024;       // entries per down chunk
+
+enum Exchange : int { EX_U = 0, EX_M = 1, EX_H = 2, EX_V = 3 };
 
 struct Smem {
   uint64_t full[kItems];
   uint64_t empty[kItems];
-  uint64_t list_ready;          // the first part of the block's list is in place
+  uint64_t list_ready;          // the kept part of the block's list is in place
   uint64_t list2_ready;         // the whole list is in place
-  uint64_t f_done;              // the consumers have taken every F record of the layer
   int abort_flag;
-  int nlist_a;                  // records of the first part of the list
+  int nlist_a;                  // records of the kept part of the list
   int nlist;
-  int count;                   // active neurons of the layer (union over tokens)
-  int pad;
-  uint32_t item_pos[kItems];   // producer bookkeeping of items in flight
+  int count;                    // own active neurons of the layer (union over tokens)
+  uint32_t item_pos[kItems];    // producer bookkeeping of items in flight
   uint32_t item_size[kItems];
-  float gmean[4];   // glue: mean and standard deviation of v per token
+  float gmean[4];               // glue: mean and standard deviation of v per token
   float gsd[4];
   float red[2][kConsumerWarps][16];   // block reductions: warp partials (double-buffered)
-  uint64_t hready[kHr];         // F: the dot partials of record s (mod kHr) are in hpart[s]
+  int hcnt[kHr];                // F: warps of the record's group that posted partials
   float hpart[kHr][16];         // [warp of the record's group][token][gate/up]
-  int32_t list[kMaxList];
+  int32_t list[kMaxList];       // the neurons this block dots, kept ones first
+  int32_t list_ent[kMaxList];   // their positions in the layer's entry order (h word index)
   uint8_t list_bits[kMaxList];
   uint8_t own_bits[kMaxOwn];
-  int32_t cnt[kMaxGrid];        // every block's own active count (balance)
-  uint32_t bsnap[kMaxGrid * 12];   // every block's first list entries (balance), kBalK per block
+  int32_t cnt[kMaxGrid];        // union active count of every block's own neurons
+  int32_t pre[kMaxGrid + 1];    // exclusive prefix of cnt: entries in owner-major order
   int32_t xpre[kMaxGrid + 1];   // exclusive prefix of the blocks' excess over the target
   int32_t bal[4];               // target, this block's deficit start, total excess
-  int32_t wsum[3][kConsumerWarps];   // per-warp partials of the balance's block scans
+  int32_t wsum[3][kConsumerWarps];   // per-warp partials of block scans
 };
 
-// Diagnostics: SM cycle stamps at phase boundaries, [block][layer][kPhases].
+// Diagnostics: SM cycle (or global ns) stamps at phase boundaries, [block][layer][slot].
 constexpr int kPhases = kDiagSlots;
 __device__ __forceinline__ long long stamp_now(const FusedParams& p) {
   return p.phase_global ? (long long)globaltimer_ns() : clock64();
@@ -109,10 +118,8 @@ __device__ __forceinline__ uint64_t tagged(uint32_t bits, uint32_t tag) { return
 __device__ __forceinline__ void st_tag(uint64_t* p, float v, uint32_t tag) {
   asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(tagged(__float_as_uint(v), tag)) : "memory");
 }
-__device__ __forceinline__ void st_tag2(uint64_t* p, float v0, float v1, uint32_t tag) {
-  asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(p), "l"(tagged(__float_as_uint(v0), tag)),
-               "l"(tagged(__float_as_uint(v1), tag))
-               : "memory");
+__device__ __forceinline__ void st_tag_u(uint64_t* p, uint32_t v, uint32_t tag) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(tagged(v, tag)) : "memory");
 }
 __device__ __forceinline__ uint64_t ld_tag(const uint64_t* p) {
   uint64_t w;
@@ -124,6 +131,12 @@ __device__ __forceinline__ void ld_tag2(const uint64_t* p, uint64_t& a, uint64_t
 }
 __device__ __forceinline__ bool tag_ok(uint64_t w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
 __device__ __forceinline__ float tag_val(uint64_t w) { return __uint_as_float((uint32_t)w); }
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
 
 // Butterfly reduce-scatter of 8 per-lane partial sums (per token) across the warp: on
 // return, out[b] in every lane is the full sum of row (lane >> 2) & 7.  The order of
@@ -168,8 +181,6 @@ __device__ __forceinline__ void poll_words(const uint64_t* base, int first, int 
   uint64_t t0 = 0;
   bool started = false;
   while (need) {
-    // every load of the round is issued before any tag is looked at, so the round costs
-    // one L2 round trip whatever the number of words
 #pragma unroll
     for (int k = 0; k < MAXK; ++k)
       if (need >> k & 1u) w[k] = ld_tag(base + first + k * stride);
@@ -205,7 +216,6 @@ struct ConsumerRing {
 __device__ __forceinline__ const uint8_t* ring_next(ConsumerRing& r, uint32_t size) {
   return r.base + ring_place(r.head, size, r.cap);
 }
-// Wait until ring item `item` has landed (bounded).
 // Wait until phase `par` of `bar` has completed (bounded).
 __device__ __forceinline__ void bar_wait(uint64_t* bar, uint32_t par, Smem& sm, const FusedParams& p) {
   if (!aborted(sm) && !mbar_try_wait(bar, par)) {
@@ -226,9 +236,14 @@ __device__ __forceinline__ void ring_wait_item_warp(uint32_t item, Smem& sm, con
   if ((threadIdx.x & 31) == 0) ring_wait_item(item, sm, p);
   __syncwarp();
 }
-__device__ __forceinline__ void ring_release_item(uint32_t item, Smem& sm) {
+// Release an item: the 16 consumer warps owe 16 arrivals per item; a warp that stands
+// for `cnt` of them arrives with that count.
+__device__ __forceinline__ void ring_release_item(uint32_t item, Smem& sm, uint32_t cnt = 1) {
   __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.empty[item % kItems]);
+  if ((threadIdx.x & 31) == 0) {
+    if (cnt == 1) mbar_arrive(&sm.empty[item % kItems]);
+    else mbar_arrive_cnt(&sm.empty[item % kItems], cnt);
+  }
 }
 
 // ------------------------------------------------------------------ activations
@@ -247,10 +262,12 @@ __device__ __forceinline__ float load_act(const void* base, size_t idx) {
   if constexpr (FAM == FAM_F32) return reinterpret_cast<const float*>(base)[idx];
   else return __half2float(reinterpret_cast<const __half*>(base)[idx]);
 }
-
-__device__ __forceinline__ int slice_begin(int s, int ns, int ngroups) {
-  return (int)((long long)s * ngroups / ns) * 32;
+template <int FAM, typename XT>
+__device__ __forceinline__ float xs_val(const XT* xs, int idx) {
+  if constexpr (FAM == FAM_F32) return xs[idx];
+  else return __half2float(xs[idx]);
 }
+
 __device__ __forceinline__ uint32_t tag_of(uint32_t epoch, int l, int e) {
   return epoch * 1024u + (uint32_t)l * 8u + (uint32_t)e;
 }
@@ -265,6 +282,85 @@ __host__ __device__ constexpr int f_group_warps(int fam, int act, int nb) {
                                                                         : 16 / (nb * (act == PI_REGLU ? 2 : 1));
 }
 
+// Elements of one 16-byte down unit: 4 fp32, 8 fp16, or the 32 weights of a Q4_0 block.
+__host__ __device__ constexpr int down_unit_elems(int fam) { return fam == FAM_F32 ? 4 : fam == FAM_F16 ? 8 : 32; }
+
+// Position of the k-th (from 0) set bit of u; u has more than k set bits.
+__device__ __forceinline__ int select_bit(uint32_t u, int k) {
+  int pos = 0, n = __popc(u & 0xFFFFu);
+  if (k >= n) { k -= n; u >>= 16; pos += 16; }
+  n = __popc(u & 0xFFu);
+  if (k >= n) { k -= n; u >>= 8; pos += 8; }
+  n = __popc(u & 0xFu);
+  if (k >= n) { k -= n; u >>= 4; pos += 4; }
+  n = __popc(u & 0x3u);
+  if (k >= n) { k -= n; u >>= 2; pos += 2; }
+  if (k >= (int)(u & 1u)) pos += 1;
+  return pos;
+}
+
+// Exclusive prefix sums over the consumer threads of K values per thread (thread order),
+// with the totals.  Integer sums: the result is exact.
+template <int K>
+__device__ __forceinline__ void block_excl_scan(const int (&v)[K], int (&excl)[K], int (&tot)[K], Smem& sm, int warp,
+                                                int lane) {
+  int incl[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    incl[k] = v[k];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, incl[k], o);
+      if (lane >= o) incl[k] += x;
+    }
+    if (lane == 31) sm.wsum[k][warp] = incl[k];
+  }
+  named_bar_sync(kRedBar, kConsumerThreads);
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    int off = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const int s = sm.wsum[k][w];
+      if (w < warp) off += s;
+      total += s;
+    }
+    excl[k] = off + incl[k] - v[k];
+    tot[k] = total;
+  }
+  named_bar_sync(kRedBar, kConsumerThreads);   // sm.wsum is free again
+}
+
+// Union over the tokens of block o's own bit word w (ob: [G][NB][nw]).
+template <int NB>
+__device__ __forceinline__ uint32_t union_word(const uint32_t* ob, int o, int w, int nw) {
+  uint32_t u = 0;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) u |= ob[((size_t)o * NB + b) * nw + w];
+  return u;
+}
+
+// Own index m of the k-th active neuron of block o, from the union of its bit words.
+template <int NB>
+__device__ __forceinline__ int owner_select(const uint32_t* ob, int o, int k, int nw) {
+  for (int w = 0; w < nw; ++w) {
+    const uint32_t u = union_word<NB>(ob, o, w, nw);
+    const int n = __popc(u);
+    if (k < n) return 32 * w + select_bit(u, k);
+    k -= n;
+  }
+  return -1;   // unreachable with consistent counts
+}
+
+template <int NB>
+__device__ __forceinline__ uint32_t owner_token_bits(const uint32_t* ob, int o, int m, int nw) {
+  uint32_t bits = 0;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) bits |= ((ob[((size_t)o * NB + b) * nw + (m >> 5)] >> (m & 31)) & 1u) << b;
+  return bits;
+}
+
+// ------------------------------------------------------------------ gate/up dots
 // This lane's partial gate/up dot products of one F record (at shared address rec) with
 // every token's x (xs: [NB][d] at shared address xs) over the units q0, q0 + qs, ... in
 // ascending order.
@@ -275,162 +371,56 @@ __device__ __forceinline__ void record_dot(uint32_t rec, uint32_t xs, const Fuse
 #pragma unroll
   for (int b = 0; b < NB; ++b) au[b] = ag[b] = 0.f;
   const uint32_t up = rec + (uint32_t)p.up_off, gate = rec + (uint32_t)p.gate_off;
-  if constexpr (FAM == FAM_Q4) {
-    // x units widen to 16 fp32 values: one token at a time keeps them in registers
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      float su[1] = {0.f}, sg[1] = {0.f};
-#pragma unroll 2
-      for (int q = q0; q < nunits; q += qs) {
-        uint32_t xu[1][XW];
-        lds_x_unit<FAM, 1>(xs + (uint32_t)(b * p.d * 2), p.d, q, xu);
-        unit_dot<FAM, 1>(up, p.d, q, xu, su);
-        if constexpr (ACT == PI_REGLU) unit_dot<FAM, 1>(gate, p.d, q, xu, sg);
-      }
-      au[b] = su[0];
-      ag[b] = sg[0];
-    }
-  } else {
 #pragma unroll 4
-    for (int q = q0; q < nunits; q += qs) {
-      uint32_t xu[NB][XW];
-      lds_x_unit<FAM, NB>(xs, p.d, q, xu);
-      unit_dot<FAM, NB>(up, p.d, q, xu, au);
-      if constexpr (ACT == PI_REGLU) unit_dot<FAM, NB>(gate, p.d, q, xu, ag);
-    }
+  for (int q = q0; q < nunits; q += qs) {
+    uint32_t xu[NB][XW];
+    lds_x_unit<FAM, NB>(xs, p.d, q, xu);
+    unit_dot<FAM, NB>(up, p.d, q, xu, au);
+    if constexpr (ACT == PI_REGLU) unit_dot<FAM, NB>(gate, p.d, q, xu, ag);
   }
 }
 
-// Balance the active records across blocks.  Every block publishes its own active count
-// and its list entries (id | token bits << 24).  After reading all counts, every block
-// derives the same assignment from them alone: target T = max(ceil(N / G), floor); a
-// block keeps its first min(n_c, T) own records; the records past T of the blocks above
-// the target, in (block, position) order, fill the blocks below it in block order.  So
-// every block ends with T or fewer records and the assignment is a function of the data
-// and the layer's floor only.  A block's first min(n_c, floor) records are its own in
-// any case, so they are fetched while this runs.  Returns the block's new list length;
-// the taken records follow its own in sm.list.
-__device__ __forceinline__ int balance_list(int n_own, int floor, uint32_t tag_c, Smem& sm, const FusedParams& p, int c,
-                                            int G, int t, int warp, int lane, int l) {
-  // publish the count and at least kBalK entries (padded), so that one polling round can
-  // read every count and every block's first kBalK entries
-  if (t < max(n_own, kBalK))
-    st_tag(p.lx + (size_t)c * kMaxOwn + t,
-           __uint_as_float(t < n_own ? ((uint32_t)sm.list[t] | ((uint32_t)sm.list_bits[t] << 24)) : 0u), tag_c);
-  if (t == 0) st_tag(p.cx + c, __int_as_float(n_own), tag_c);
-  stamp(p, l, 22);
-  {
-    // chunks of 4 words per thread: one round for up to 2048 words (157 blocks)
-    constexpr int MQ = 4;
-    const int nq = G * (1 + kBalK);
-    for (int base = 0; base < nq; base += MQ * kConsumerThreads) {
-      uint64_t w[MQ];
-      uint32_t need = 0;
+// ------------------------------------------------------------------ down units
+// acc[b][e] += h[b] * (element e of a 16-byte down unit at shared address a); Q4_0 units
+// are whole 32-weight blocks whose fp16 scale is `sc`.
+template <int FAM, int NB>
+__device__ __forceinline__ void down_unit_fma(uint32_t a, float sc, const float (&h)[NB],
+                                              float (&acc)[NB][down_unit_elems(FAM)]) {
+  if constexpr (FAM == FAM_F32) {
+    const float4 w = u4f(lds128(a));
 #pragma unroll
-      for (int i = 0; i < MQ; ++i) {
-        w[i] = 0;
-        if (base + t + i * kConsumerThreads < nq) need |= 1u << i;
-      }
-      bool started = false;
-      uint64_t tp = 0;
-      while (need) {
+    for (int b = 0; b < NB; ++b) {
+      acc[b][0] = fmaf(h[b], w.x, acc[b][0]); acc[b][1] = fmaf(h[b], w.y, acc[b][1]);
+      acc[b][2] = fmaf(h[b], w.z, acc[b][2]); acc[b][3] = fmaf(h[b], w.w, acc[b][3]);
+    }
+  } else if constexpr (FAM == FAM_F16) {
+    float w[8];
+    widen8(lds128(a), w);
 #pragma unroll
-        for (int i = 0; i < MQ; ++i)
-          if (need >> i & 1u) {
-            const int q = base + t + i * kConsumerThreads;
-            const uint64_t* src = (q < G) ? p.cx + q : p.lx + (size_t)((q - G) / kBalK) * kMaxOwn + (q - G) % kBalK;
-            w[i] = ld_tag(src);
-          }
+    for (int b = 0; b < NB; ++b)
 #pragma unroll
-        for (int i = 0; i < MQ; ++i)
-          if ((need >> i & 1u) && tag_ok(w[i], tag_c)) need &= ~(1u << i);
-        if (!need || aborted(sm)) break;
-        if (!started) { tp = wait_start(); started = true; }
-        else if (timed_out(tp, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
-        if (p.poll_ns) __nanosleep(p.poll_ns);
-      }
+      for (int e = 0; e < 8; ++e) acc[b][e] = fmaf(h[b], w[e], acc[b][e]);
+  } else {
+    // byte j of the block: element j in its low nibble, element j + 16 in its high one
+    const uint4 nb = lds128(a);
+    const uint32_t wv[4] = {nb.x, nb.y, nb.z, nb.w};
+    float hs[NB];
 #pragma unroll
-      for (int i = 0; i < MQ; ++i) {
-        const int q = base + t + i * kConsumerThreads;
-        if (q < G) sm.cnt[q] = __float_as_int(tag_val(w[i]));
-        else if (q < nq) sm.bsnap[q - G] = (uint32_t)w[i];
+    for (int b = 0; b < NB; ++b) hs[b] = h[b] * sc;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const uint32_t lo = wv[m] & 0x0F0F0F0Fu, hi = (wv[m] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float cl = q4_val(lo, k), ch = q4_val(hi, k);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          acc[b][4 * m + k] = fmaf(hs[b], cl, acc[b][4 * m + k]);
+          acc[b][16 + 4 * m + k] = fmaf(hs[b], ch, acc[b][16 + 4 * m + k]);
+        }
       }
     }
   }
-  stamp(p, l, 23);
-  named_bar_sync(kRedBar, kConsumerThreads);
-  stamp(p, l, 24);
-  // block-wide: N = sum of the counts, T, the exclusive prefix of the excess over T, and
-  // this block's deficit start (the deficits of the blocks before it), in fixed orders
-  const int cv = (t < G) ? sm.cnt[t] : 0;
-  {
-    int v = cv;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) sm.wsum[0][warp] = v;
-  }
-  named_bar_sync(kRedBar, kConsumerThreads);
-  int n = 0;
-#pragma unroll
-  for (int w = 0; w < kConsumerWarps; ++w) n += sm.wsum[0][w];
-  const int Tb = max((n + G - 1) / G, floor);
-  const int ex = (t < G) ? max(0, cv - Tb) : 0;
-  const int de = (t < c) ? max(0, Tb - cv) : 0;
-  int incl = ex, dsum = de;
-#pragma unroll
-  for (int k = 1; k < 32; k <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, k);
-    if (lane >= k) incl += v;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
-  if (lane == 31) sm.wsum[1][warp] = incl;
-  if (lane == 0) sm.wsum[2][warp] = dsum;
-  named_bar_sync(kRedBar, kConsumerThreads);
-  {
-    int off = 0, total = 0, dstart_all = 0;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      if (w < warp) off += sm.wsum[1][w];
-      total += sm.wsum[1][w];
-      dstart_all += sm.wsum[2][w];
-    }
-    if (t < G) sm.xpre[t] = off + incl - ex;
-    if (t == 0) {
-      sm.xpre[G] = total;
-      sm.bal[0] = Tb;
-      sm.bal[1] = dstart_all;
-      sm.bal[2] = total;
-    }
-  }
-  named_bar_sync(kRedBar, kConsumerThreads);
-  const int T = sm.bal[0], dstart = sm.bal[1], xtotal = sm.bal[2];
-  const int keep = min(n_own, T);
-  const int deficit = max(0, T - n_own);
-  const int ntake = max(0, min(dstart + deficit, xtotal) - dstart);
-  stamp(p, l, 25);
-  if (t < ntake) {
-    const int x = dstart + t;
-    int lo = 0, hi = G;   // owner o: xpre[o] <= x < xpre[o + 1]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (sm.xpre[mid] <= x) lo = mid;
-      else hi = mid;
-    }
-    const int k = T + (x - sm.xpre[lo]);
-    uint32_t v;
-    if (k < kBalK) {
-      v = sm.bsnap[lo * kBalK + k];
-    } else {   // past the snapshot (a block far above the target): read it now
-      uint64_t w[1];
-      poll_words<1>(p.lx + (size_t)lo * kMaxOwn + k, 0, 1, 1, tag_c, w, sm, p);
-      v = (uint32_t)w[0];
-    }
-    sm.list[keep + t] = (int32_t)(v & 0xFFFFFFu);
-    sm.list_bits[keep + t] = (uint8_t)(v >> 24);
-  }
-  named_bar_sync(kRedBar, kConsumerThreads);
-  return keep + ntake;
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -439,22 +429,40 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
   constexpr int UE = Fam<FAM>::UE;
   constexpr int XW = Fam<FAM>::XW;
   constexpr int PB = Fam<FAM>::PB;
+  constexpr int PE = down_unit_elems(FAM);
   using XT = typename Fam<FAM>::X;
   extern __shared__ __align__(128) uint8_t dsmem[];
   Smem& sm = *reinterpret_cast<Smem*>(dsmem);
-  uint8_t* ring_base = dsmem + ((sizeof(Smem) + 127) / 128) * 128;
-  XT* xs = reinterpret_cast<XT*>(ring_base + p.ring_bytes);            // [NB][d] current input
-  float* u_s = reinterpret_cast<float*>(xs + (size_t)NB * p.d);        // [NB][r]
-  float* red2 = u_s + (size_t)NB * p.r;                                // [8][NB][4][32]
+  uint8_t* ring_base = dsmem + p.off_ring;
+  XT* xs = reinterpret_cast<XT*>(dsmem + p.off_xs);                  // [NB][d] current input
+  float* u_s = reinterpret_cast<float*>(dsmem + p.off_us);           // [NB][r]
+  uint32_t* ob = reinterpret_cast<uint32_t*>(dsmem + p.off_ob);      // [G][NB][nw] every block's own bits
+  int32_t* dlist = reinterpret_cast<int32_t*>(dsmem + p.off_dlist);  // [2][dch] neuron of each chunk entry
+  float* dred = reinterpret_cast<float*>(dsmem + p.off_dred);        // down reduction / v slice / moments
+  const uint32_t dbuf_u = smem_u32(dsmem + p.off_dbuf);              // [2][dch][pmax] 16-byte down units
+  const uint32_t dsc_u = smem_u32(dsmem + p.off_dsc);                // Q4_0: [2][dch][pmax] scale words
 
   const int c = blockIdx.x, G = gridDim.x;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const bool do_pred = p.mode & MODE_PREDICT, do_ffn = p.mode & MODE_FFN, do_glue = p.mode & MODE_GLUE;
-  const int d = p.d, f = p.f, r = p.r, B = p.B;
-  const int k0 = (int)((long long)c * r / G), k1 = (int)((long long)(c + 1) * r / G);
+  const int d = p.d, f = p.f, B = p.B;
   const int nown = (c < f) ? (f - c + G - 1) / G : 0;
   const int nunits = d / UE;
   const int words = f / 32;
+  const int nw = p.nw;
+  const int dch = p.dch, pmax = p.pmax;
+  // the block's down slice: 16-byte units [cu0, cu1) of every down row.  In the down
+  // phase lpe consecutive lanes take one entry (lane % lpe is the unit, so the lanes of an
+  // entry read one contiguous piece of its row) and a warp takes epw entries per pass:
+  // this lane handles unit dw of the entries de0, de0 + dstep, ... of every chunk
+  const int cu0 = (int)((long long)c * p.dunits / G), cu1 = (int)((long long)(c + 1) * p.dunits / G);
+  const int npc = cu1 - cu0;
+  const int lpe = npc <= 1 ? 1 : npc <= 2 ? 2 : npc <= 4 ? 4 : npc <= 8 ? 8 : 16;
+  const int epw = 32 / lpe;
+  const int dw = (lane % lpe) < npc ? lane % lpe : -1;
+  const int de0 = warp * epw + lane / lpe;
+  const int dstep = kConsumerWarps * epw;
+  const int col0 = cu0 * PE, ncol = npc * PE;
   const uint32_t epoch = *reinterpret_cast<volatile const uint32_t*>(p.bar + 2);
 
   if (t == 0) {
@@ -464,8 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     }
     mbar_init(&sm.list_ready, 1);
     mbar_init(&sm.list2_ready, 1);
-    mbar_init(&sm.f_done, 1);
-    for (int s = 0; s < kHr; ++s) mbar_init(&sm.hready[s], f_group_warps(FAM, ACT, NB));
+    for (int s = 0; s < kHr; ++s) sm.hcnt[s] = 0;
     sm.abort_flag = 0;
     sm.nlist = 0;
     mbar_fence_init();
@@ -476,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
   if (warp == kConsumerWarps) {
     if (lane == 0) {
       uint32_t head = 0, issued = 0, oldest = 0;
+      uint32_t landed = 0, inflight = 0;   // items known to have landed; bytes issued beyond them
       // Reserve ring space for the next item: wait (in order) for the release of every
       // older item that overlaps it, and of the item that last used its barrier pair.
       auto reserve = [&](uint32_t size, uint32_t& pos) -> bool {
@@ -502,9 +510,35 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         }
         return !aborted(sm);
       };
+      // Keep at most inflight_budget bytes of this block's copies in flight (one item at
+      // least): more would not raise the block's share of HBM bandwidth, only the queueing
+      // delay every latency-critical exchange word waits behind.
+      auto throttle = [&](uint32_t size) -> bool {
+        while (landed < issued && inflight + size > (uint32_t)p.inflight_budget) {
+          uint64_t* fb = &sm.full[landed % kItems];
+          const uint32_t par = (landed / kItems) & 1u;
+          if (!mbar_try_wait(fb, par)) {
+            const uint64_t t0 = wait_start();
+            while (!mbar_try_wait_sleep(fb, par, kSleepNs)) {
+              if (aborted(sm)) return false;
+              if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); return false; }
+            }
+          }
+          inflight -= sm.item_size[landed % kItems];
+          ++landed;
+        }
+        return !aborted(sm);
+      };
       auto begin_item = [&](uint32_t size, uint8_t*& dst, uint64_t*& fb) -> bool {
         uint32_t pos;
+        if (!throttle(size)) return false;
         if (!reserve(size, pos)) return false;
+        // released items have landed: account for them before their slot is reused
+        while (landed < oldest) {
+          inflight -= sm.item_size[landed % kItems];
+          ++landed;
+        }
+        inflight += size;
         sm.item_pos[issued % kItems] = pos;
         sm.item_size[issued % kItems] = size;
         dst = ring_base + pos;
@@ -513,22 +547,23 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         ++issued;
         return true;
       };
+      auto wait_list = [&](uint64_t* bar, uint32_t par) -> bool {
+        const uint64_t t0 = wait_start();
+        while (!mbar_try_wait_sleep(bar, par, kSleepNs)) {
+          if (aborted(sm)) return false;
+          if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); return false; }
+        }
+        return true;
+      };
       bool ok = true;
       for (int l = 0; l < p.L && ok; ++l) {
         const LayerDev Ld = p.layers[l];
+        const int r = Ld.r;
+        const int k0 = (int)((long long)c * r / G), k1 = (int)((long long)(c + 1) * r / G);
+        const int p2_stride = p2_stride_of(r, PB);
+        const int p2_rows = max(1, min(p.nown_max, p.p2_item_bytes / p2_stride));
         uint8_t* dst;
         uint64_t* fb;
-        if (do_pred && do_ffn && l > 0) {
-          // the predictor rows of this layer are not needed before the glue of the last
-          // one ends: start their copies once this block has taken its last F record, so
-          // that they do not compete with the F records other blocks still wait for
-          const uint64_t t0 = wait_start();
-          while (!mbar_try_wait_sleep(&sm.f_done, (uint32_t)((l - 1) & 1), kSleepNs)) {
-            if (aborted(sm)) { ok = false; break; }
-            if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
-          }
-          if (!ok) break;
-        }
         if (do_pred) {
           for (int k = k0; k < k1 && ok; k += p.p1_rows_per_item) {
             const int n = min(p.p1_rows_per_item, k1 - k);
@@ -536,48 +571,33 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
             if (!(ok = begin_item(bytes, dst, fb))) break;
             bulk_g2s(dst, Ld.p1t + (size_t)k * p.p1_row, bytes, fb);
           }
-          const uint8_t* own = Ld.p2o + (size_t)c * p.nown_max * p.p2_stride;
-          for (int m = 0; m < nown && ok; m += p.p2_rows_per_item) {
-            const int n = min(p.p2_rows_per_item, nown - m);
-            const uint32_t bytes = (uint32_t)n * p.p2_stride;
+          const uint8_t* own = Ld.p2o + (size_t)c * p.nown_max * p2_stride;
+          for (int m = 0; m < nown && ok; m += p2_rows) {
+            const int n = min(p2_rows, nown - m);
+            const uint32_t bytes = (uint32_t)n * p2_stride;
             if (!(ok = begin_item(bytes, dst, fb))) break;
-            bulk_g2s(dst, own + (size_t)m * p.p2_stride, bytes, fb);
+            bulk_g2s(dst, own + (size_t)m * p2_stride, bytes, fb);
           }
         }
         if (do_ffn && ok) {
-          pstamp(p, l, 9);
-          const uint64_t t0 = wait_start();
-          while (!mbar_try_wait_sleep(&sm.list_ready, (uint32_t)(l & 1), kSleepNs)) {
-            if (aborted(sm)) { ok = false; break; }
-            if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
-          }
-          pstamp(p, l, 10);
-          // Ask HBM for every record at once (L2 prefetch needs no shared memory); the
-          // ring copies then find them in L2 as space frees up.  The first part of the
-          // list is known before the balancing exchange ends, the rest after it.
+          pstamp(p, l, 20);
+          ok = wait_list(&sm.list_ready, (uint32_t)(l & 1));
+          pstamp(p, l, 21);
+          // The kept part of the list is known before the mask exchange ends, the rest
+          // after it.
           const int na = ok ? sm.nlist_a : 0;
-          for (int e = 0; e < na && ok; ++e)
-            prefetch_l2_bulk(Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride);
           int e = 0;
           for (; e < na && ok; ++e) {
             if (!(ok = begin_item((uint32_t)p.rec_stride, dst, fb))) break;
             bulk_g2s(dst, Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride, fb);
           }
-          if (ok) {
-            const uint64_t t0 = wait_start();
-            while (!mbar_try_wait_sleep(&sm.list2_ready, (uint32_t)(l & 1), kSleepNs)) {
-              if (aborted(sm)) { ok = false; break; }
-              if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
-            }
-          }
+          if (ok) ok = wait_list(&sm.list2_ready, (uint32_t)(l & 1));
           const int n = ok ? sm.nlist : 0;
-          for (int q = na; q < n && ok; ++q)
-            prefetch_l2_bulk(Ld.rec + (size_t)sm.list[q] * p.rec_stride, (uint32_t)p.rec_stride);
           for (; e < n && ok; ++e) {
             if (!(ok = begin_item((uint32_t)p.rec_stride, dst, fb))) break;
             bulk_g2s(dst, Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride, fb);
           }
-          pstamp(p, l, 11);
+          pstamp(p, l, 22);
         }
       }
       // drain: never leave the block while a bulk copy may still write shared memory
@@ -600,38 +620,29 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
   // the input x of the first layer into shared memory
   for (int idx = t; idx < B * d; idx += kConsumerThreads) xs[idx] = reinterpret_cast<const XT*>(p.x_in)[idx];
   for (int idx = B * d + t; idx < NB * d; idx += kConsumerThreads) xs[idx] = XT(0.f);
-
-  const int ngroups = d / 32;
-  const int nslices = p.nslices;
-  const bool slice_owner = c < nslices;
-  const int col0 = slice_owner ? slice_begin(c, nslices, ngroups) : 0;
-  const int col1 = slice_owner ? slice_begin(c + 1, nslices, ngroups) : 0;
-  const int ng = (col1 - col0) / 32;
-  // slice owners keep their slice of the current layer input (fp32) for the residual:
-  // warp b holds token b, lane = column within a 32-column group
-  float xsl[kMaxColGroups];
-#pragma unroll
-  for (int gq = 0; gq < kMaxColGroups; ++gq) xsl[gq] = 0.f;
-  if (do_glue && slice_owner && warp < B) {
-#pragma unroll
-    for (int gq = 0; gq < kMaxColGroups; ++gq)
-      if (gq < ng) {
-        const size_t idx = (size_t)warp * d + col0 + 32 * gq + lane;
-        xsl[gq] = load_act<FAM>(p.x_in, idx);
-        if (p.trace.x) store_act<FAM>(p.trace.x, idx, xsl[gq]);
-      }
-  }
+  // the trace's layer-0 input: every block writes its own columns
+  if (do_glue && p.trace.x)
+    for (int q = t; q < B * ncol; q += kConsumerThreads) {
+      const size_t idx = (size_t)(q / ncol) * d + col0 + q % ncol;
+      store_act<FAM>(p.trace.x, idx, load_act<FAM>(p.x_in, idx));
+    }
   named_bar_sync(kRedBar, kConsumerThreads);
 
-  int redbuf = 0;   // which half of sm.red the next block reduction uses
+  int redbuf = 0;     // which half of sm.red the next block reduction uses
   uint32_t fseq = 0;  // F records of earlier layers (h slot of record e: (fseq + e) % kHr)
   for (int l = 0; l < p.L; ++l) {
-    const uint32_t tag_u = tag_of(epoch, l, 0), tag_p = tag_of(epoch, l, 1), tag_v = tag_of(epoch, l, 2),
-                   tag_c = tag_of(epoch, l, 3);
-    int nlist = 0;
-    bool signaled_a = false;   // the first part of the list was handed over already
+    const LayerDev Ld = p.layers[l];
+    const int r = Ld.r;
+    const int k0 = (int)((long long)c * r / G), k1 = (int)((long long)(c + 1) * r / G);
+    const int p2_stride = p2_stride_of(r, PB);
+    const int p2_rows = max(1, min(p.nown_max, p.p2_item_bytes / p2_stride));
+    const uint32_t tag_u = tag_of(epoch, l, EX_U), tag_m = tag_of(epoch, l, EX_M), tag_h = tag_of(epoch, l, EX_H),
+                   tag_v = tag_of(epoch, l, EX_V);
+    int nlist = 0;      // records this block dots
+    int ntotal = 0;     // active entries of the layer (the down list)
+    bool signaled_a = false;
     stamp(p, l, 0);
-    // this layer's x units, fp32, in registers for P-a and F
+    // this layer's x units, fp32, in registers for P-a
     uint32_t xr[NU][NB][XW];
 #pragma unroll
     for (int j = 0; j < NU; ++j) {
@@ -655,7 +666,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         const int n = min(p.p1_rows_per_item, k1 - k);
         const uint8_t* item = ring_next(ring, (uint32_t)n * p.p1_row);
         ring_wait_item_warp(ring.item, sm, p);
-        if (k == k0) stamp(p, l, 13);
         for (int i0 = 0; i0 < n; i0 += RP) {
           float v[16];
 #pragma unroll
@@ -711,17 +721,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       uint32_t* mask_dst = do_glue ? (p.trace.mask ? p.trace.mask + (size_t)l * B * words : nullptr) : p.mask_out;
       const int rchunks = r * PB / 16;
       long long pb_wait = 0;   // diagnostics: cycles spent waiting for P2 items
-      for (int m0 = 0; m0 < nown; m0 += p.p2_rows_per_item) {
-        const int n = min(p.p2_rows_per_item, nown - m0);
-        const uint8_t* item = ring_next(ring, (uint32_t)n * p.p2_stride);
+      for (int m0 = 0; m0 < nown; m0 += p2_rows) {
+        const int n = min(p2_rows, nown - m0);
+        const uint8_t* item = ring_next(ring, (uint32_t)n * p2_stride);
         const long long wt0 = diag_clock(p);
         ring_wait_item_warp(ring.item, sm, p);
         pb_wait += diag_clock(p) - wt0;
-        if (m0 == 0) stamp(p, l, 12);
         for (int mb = warp * 8; mb < n; mb += kConsumerWarps * 8) {
           uint32_t rows[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) rows[i] = smem_u32(item) + (uint32_t)(min(mb + i, n - 1) * p.p2_stride);   // past n: repeats, unused
+          for (int i = 0; i < 8; ++i) rows[i] = smem_u32(item) + (uint32_t)(min(mb + i, n - 1) * p2_stride);   // past n: repeats, unused
           float acc[8][NB];
 #pragma unroll
           for (int i = 0; i < 8; ++i)
@@ -789,12 +798,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         ring_release_item(ring.item++, sm);
       }
       named_bar_sync(kRedBar, kConsumerThreads);
-      stamp(p, l, 7);
+      stamp(p, l, 3);
       stamp_val(p, l, 18, pb_wait);
+      if (!do_ffn) break;   // predictor only
 
-      // ---------------------------------------------------------- own active list
-      // Block c processes the active neurons it owns, i = c + m*G in ascending m: the
-      // list needs nothing from other blocks.
+      // ---------------------------------------------------------- own active list + bits
+      // Block c's own neurons are i = c + m*G in ascending m.  Warp w < nw also publishes
+      // word w of the block's own bits for every token (the mask exchange).
       if (warp == 0) {
         int base = 0;
         for (int mm = 0; mm < nown; mm += 32) {
@@ -810,24 +820,137 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         }
         if (lane == 0) sm.count = base;
       }
+      for (int w = warp; w < nw; w += kConsumerWarps) {
+        const int m = 32 * w + lane;
+        const uint32_t tb = (m < nown) ? sm.own_bits[m] : 0u;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const uint32_t word = __ballot_sync(0xffffffffu, (tb >> b) & 1u);
+          if (lane == 0 && b < B) st_tag_u(p.mx + ((size_t)c * 4 + b) * kMaxOwnWords + w, word, tag_m);
+        }
+      }
       named_bar_sync(kRedBar, kConsumerThreads);
-      nlist = sm.count;
-      if (t == 0 && do_ffn && nlist > 0) {
+      const int n_own = sm.count;
+      const int floor = Ld.keep_floor;
+      // the kept part (own records every block keeps whatever the counts) goes to the
+      // producer now, so its copies run during the mask exchange
+      if (t == 0) {
+        sm.nlist_a = min(n_own, floor);
+        mbar_arrive(&sm.list_ready);
+      }
+      signaled_a = true;
+      stamp(p, l, 4);
+
+      // ---------------------------------------------------------- mask exchange
+      {
+        const int per = B * nw;
+        const int nq = G * per;
+        constexpr int MQ = 16;
+        if (NB > B)
+          for (int q = t; q < G * NB * nw; q += kConsumerThreads)
+            if ((q / nw) % NB >= B) ob[q] = 0u;
+        for (int base = 0; base < nq; base += MQ * kConsumerThreads) {
+          uint64_t w[MQ];
+          uint32_t need = 0;
+#pragma unroll
+          for (int i = 0; i < MQ; ++i) {
+            w[i] = 0;
+            if (base + t + i * kConsumerThreads < nq) need |= 1u << i;
+          }
+          bool started = false;
+          uint64_t tp0 = 0;
+          while (need) {
+#pragma unroll
+            for (int i = 0; i < MQ; ++i)
+              if (need >> i & 1u) {
+                const int q = base + t + i * kConsumerThreads;
+                const int o = q / per, rem = q % per;
+                w[i] = ld_tag(p.mx + ((size_t)o * 4 + rem / nw) * kMaxOwnWords + rem % nw);
+              }
+#pragma unroll
+            for (int i = 0; i < MQ; ++i)
+              if ((need >> i & 1u) && tag_ok(w[i], tag_m)) need &= ~(1u << i);
+            if (!need || aborted(sm)) break;
+            if (!started) { tp0 = wait_start(); started = true; }
+            else if (timed_out(tp0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+            if (p.poll_ns) __nanosleep(p.poll_ns);
+          }
+#pragma unroll
+          for (int i = 0; i < MQ; ++i) {
+            const int q = base + t + i * kConsumerThreads;
+            if (q < nq) {
+              // only bits of neurons the owner has can be set (a word of an aborted
+              // exchange may hold anything)
+              const int o = q / per, rem = q % per, ww = rem % nw;
+              const int nown_o = (o < f) ? (f - o + G - 1) / G : 0;
+              const int nv = min(32, max(0, nown_o - 32 * ww));
+              const uint32_t valid = nv >= 32 ? 0xFFFFFFFFu : ((1u << nv) - 1u);
+              ob[((size_t)o * NB + rem / nw) * nw + ww] = (uint32_t)w[i] & valid;
+            }
+          }
+        }
+      }
+      named_bar_sync(kRedBar, kConsumerThreads);
+      stamp(p, l, 5);
+      if (t < G) {
+        int n = 0;
+        for (int w = 0; w < nw; ++w) n += __popc(union_word<NB>(ob, t, w, nw));
+        sm.cnt[t] = n;
+      }
+      named_bar_sync(kRedBar, kConsumerThreads);
+
+      // ---------------------------------------------------------- balanced assignment
+      // N = the sum of the counts; target T = max(ceil(N / G), floor).  Block c keeps its
+      // first min(n_c, T) own entries; the entries past T of the blocks above the target,
+      // in (block, position) order, fill the blocks below it in block order.  Every block
+      // derives the same assignment from the counts alone.
+      {
+        const int cv = (t < G) ? sm.cnt[t] : 0;
+        int v1[1] = {cv}, e1[1], s1[1];
+        block_excl_scan<1>(v1, e1, s1, sm, warp, lane);
+        const int N = s1[0];
+        const int T = max((N + G - 1) / G, floor);
+        int v2[2] = {(t < G) ? max(0, cv - T) : 0, (t < G) ? max(0, T - cv) : 0}, e2[2], s2[2];
+        block_excl_scan<2>(v2, e2, s2, sm, warp, lane);
+        if (t < G) {
+          sm.pre[t] = e1[0];
+          sm.xpre[t] = e2[0];
+        }
+        if (t == c) sm.bal[1] = e2[1];
+        if (t == 0) {
+          sm.pre[G] = N;
+          sm.xpre[G] = s2[0];
+          sm.bal[0] = T;
+          sm.bal[2] = s2[0];
+        }
+        named_bar_sync(kRedBar, kConsumerThreads);
+        const int dstart = sm.bal[1], xtotal = sm.bal[2];
+        const int keep = min(n_own, T);
+        const int deficit = max(0, T - n_own);
+        const int ntake = max(0, min(dstart + deficit, xtotal) - dstart);
+        for (int q = t; q < keep; q += kConsumerThreads) sm.list_ent[q] = sm.pre[c] + q;
+        for (int q = t; q < ntake; q += kConsumerThreads) {
+          const int x = dstart + q;
+          int lo = 0, hi = G;   // owner o: xpre[o] <= x < xpre[o + 1]
+          while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (sm.xpre[mid] <= x) lo = mid;
+            else hi = mid;
+          }
+          const int k = T + (x - sm.xpre[lo]);
+          const int m = owner_select<NB>(ob, lo, k, nw);
+          const int i = lo + max(m, 0) * G;
+          sm.list[keep + q] = i < f ? i : 0;
+          sm.list_ent[keep + q] = sm.pre[lo] + k;
+          sm.list_bits[keep + q] = (uint8_t)owner_token_bits<NB>(ob, lo, max(m, 0), nw);
+        }
+        nlist = keep + ntake;
+        ntotal = N;
+      }
+      if (t == 0) {
         atomicAdd(p.active_total, (unsigned long long)nlist);
         if (p.layer_count) atomicAdd(p.layer_count + l, nlist);
       }
-      stamp(p, l, 15);
-      if (do_ffn && p.cx) {
-        // the first part (own records every block keeps) goes to the producer now
-        const int floor = p.layers[l].keep_floor;
-        if (t == 0) {
-          sm.nlist_a = min(nlist, floor);
-          mbar_arrive(&sm.list_ready);
-        }
-        signaled_a = true;
-        nlist = balance_list(nlist, floor, tag_c, sm, p, c, G, t, warp, lane, l);
-      }
-      stamp_val(p, l, 14, nlist);
     } else if (do_ffn) {
       // ---------------------------------------------------------- list from the caller
       int cnt = __ldg(p.count_in);
@@ -847,12 +970,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         uint32_t bits = 0;
         for (int b = 0; b < B; ++b) bits |= ((__ldg(p.mask_in + (size_t)b * words + (i >> 5)) >> (i & 31)) & 1u) << b;
         sm.list[e] = i;
+        sm.list_ent[e] = a0 + e;
         sm.list_bits[e] = (uint8_t)bits;
       }
       if (t == 0) atomicAdd(p.active_total, (unsigned long long)nlist);
+      ntotal = cnt;
     }
 
-    if (!do_ffn) break;   // predictor only
     named_bar_sync(kRedBar, kConsumerThreads);
     if (t == 0) {
       if (!signaled_a) {
@@ -862,26 +986,73 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       sm.nlist = nlist;
       mbar_arrive(&sm.list2_ready);
     }
-    stamp(p, l, 3);
+    stamp(p, l, 6);
+    stamp_val(p, l, 14, nlist);
+    stamp_val(p, l, 15, ntotal);
 
-    // ------------------------------------------------------------ F: records
-    // The 16 consumer warps form groups of KG; group g takes the gate/up dots of records
-    // g, g + 16/KG, ... with no block barrier: each warp of the group waits for the record
-    // to land, dots its slice of the units with x from shared memory, reduces across its
-    // lanes, posts its partial sums in the record's h slot and arrives on the slot's
-    // barrier.  Every thread then adds h * (its units of each down row) into its y units
-    // in list order: it waits on each record's slot, sums the KG partials in a fixed order,
-    // forms h and releases the record.  A warp dots a record only while it is fewer than R
-    // records ahead of its own down-row cursor, so the records a warp waits for always
-    // fit in the ring beside the ones not yet released.  Sums run in a fixed order
-    // whatever the timing.
-    float y[NU][NB][UE];
-#pragma unroll
-    for (int j = 0; j < NU; ++j)
-#pragma unroll
-      for (int b = 0; b < NB; ++b)
-#pragma unroll
-        for (int e = 0; e < UE; ++e) y[j][b][e] = 0.f;
+    // ------------------------------------------------------------ down list and copies
+    // Chunk k holds the active entries [k*dch, (k+1)*dch) of the layer in owner-major
+    // order (the caller's order for a given list); dlist half k%2 holds their neuron ids
+    // and dbuf half k%2 their units [cu0, cu1).  Each thread copies, and later reads,
+    // only its own slots, so its cp.async groups alone order the copies and the reads.
+    const int nchunks = (ntotal + dch - 1) / dch;
+    const uint8_t* dn = Ld.rec + p.dn_off;
+    auto build_dlist = [&](int k) {
+      const int lo = k * dch, hi = min(ntotal, lo + dch);
+      int32_t* dl = dlist + (k & 1) * dch;
+      if (do_pred) {
+        for (int o = t; o < G; o += kConsumerThreads) {
+          const int e0 = sm.pre[o], e1 = e0 + sm.cnt[o];
+          if (e1 <= lo || e0 >= hi) continue;
+          int e = e0;
+          for (int w = 0; w < nw && e < hi; ++w) {
+            uint32_t u = union_word<NB>(ob, o, w, nw);
+            const int n = __popc(u);
+            if (e + n <= lo) { e += n; continue; }
+            while (u && e < hi) {
+              const int bit = __ffs(u) - 1;
+              u &= u - 1;
+              if (e >= lo) dl[e - lo] = o + (32 * w + bit) * G;
+              ++e;
+            }
+          }
+        }
+      } else {
+        for (int e = lo + t; e < hi; e += kConsumerThreads) {
+          int i = __ldg(p.idx_in + e);
+          if (i < 0 || i >= f) i = 0;   // reported above
+          dl[e - lo] = i;
+        }
+      }
+    };
+    auto issue_down = [&](int k) {
+      if (dw < 0) return;
+      const int lo = k * dch, hi = min(ntotal, lo + dch);
+      const int32_t* dl = dlist + (k & 1) * dch;
+      const int half = (k & 1) * dch;
+      for (int e = lo + de0; e < hi; e += dstep) {
+        const int i = dl[e - lo];
+        const uint8_t* row = dn + (size_t)i * p.dn_stride;
+        const uint32_t slot = (uint32_t)((half + e - lo) * pmax + dw);
+        cpa16(dbuf_u + slot * 16u, row + (size_t)(cu0 + dw) * 16);
+        if constexpr (FAM == FAM_Q4) cpa4(dsc_u + slot * 4u, row + (size_t)(d >> 1) + (size_t)((cu0 + dw) >> 1) * 4);
+      }
+    };
+    build_dlist(0);
+    if (nchunks > 1) build_dlist(1);
+    named_bar_sync(kRedBar, kConsumerThreads);
+    issue_down(0);
+    cpa_commit();
+    if (nchunks > 1) issue_down(1);
+    cpa_commit();
+    stamp(p, l, 7);
+
+    // ------------------------------------------------------------ F: records -> h
+    // The 16 consumer warps form groups of KG; group g dots records g, g + 16/KG, ...
+    // with no block barrier: each warp of the group waits for the record to land, dots
+    // its slice of the units with x from shared memory, reduces across its lanes and
+    // posts its partial sums in the record's h slot.  The last warp of the group to post
+    // sums the group's partials in a fixed order, forms h and publishes it.
     {
       constexpr int NV = (ACT == PI_REGLU) ? 2 : 1;
       constexpr int NVAL = NB * NV;                 // partial sums per warp and record
@@ -890,194 +1061,208 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       constexpr int KG = f_group_warps(FAM, ACT, NB);
       constexpr int NG = kConsumerWarps / KG;       // records dotted at once
       static_assert(KG * NVAL <= 16 && kConsumerWarps % KG == 0, "h slot layout");
-      // records E .. E + R - 1 fit in the ring together (at most one record's worth of
-      // space is lost where the placement wraps)
-      const int R = max(1, min((int)(ring.cap / (uint32_t)p.rec_stride) - 1, kConsumerWarps));
       const uint32_t base = smem_u32(ring.base), xsa = smem_u32(xs);
       const uint32_t item0 = ring.item;
       const int kq = warp % KG;
-      long long f_wait = 0, d_wait = 0;   // diagnostics: cycles thread 0 waits for h / for records
-      int ed = warp / KG;                  // next record this warp's group dots
-      uint32_t hd = ring.head;             // ring head before record id (dot cursor)
+      long long f_wait = 0;   // diagnostics: cycles warp 0 waits for records
+      uint32_t hd = ring.head;   // ring head before record id (dot cursor)
       int id = 0;
-      for (int ea = 0; ea < nlist; ++ea) {
-        while (ed < nlist && ed < ea + R) {
-          uint32_t pos = 0;
-          for (; id <= ed; ++id) pos = ring_place(hd, (uint32_t)p.rec_stride, ring.cap);
-          const long long wt0 = diag_clock(p);
-          ring_wait_item_warp(item0 + ed, sm, p);
-          d_wait += diag_clock(p) - wt0;
-          if (ed == 0) stamp(p, l, 5);
-          float au[NB], ag[NB];
-          record_dot<FAM, ACT, NB>(base + pos, xsa, p, nunits, 32 * kq + lane, 32 * KG, au, ag);
-          float v[V];
-#pragma unroll
-          for (int i = 0; i < V; ++i) v[i] = 0.f;
-#pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            v[b * NV] = au[b];
-            if constexpr (ACT == PI_REGLU) v[b * NV + 1] = ag[b];
-          }
-          const float sw = reduce_scatter<V>(v, lane);   // lane k: value k >> (5 - LG)
-          const uint32_t s = (fseq + (uint32_t)ed) % kHr;
-          if ((lane & ((32 >> LG) - 1)) == 0 && (lane >> (5 - LG)) < NVAL) sm.hpart[s][kq * NVAL + (lane >> (5 - LG))] = sw;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.hready[s]);
-          ed += NG;
-        }
-        const uint32_t pa = ring_place(ring.head, (uint32_t)p.rec_stride, ring.cap);
-        const uint32_t sq = fseq + (uint32_t)ea;
+      for (int e = warp / KG; e < nlist; e += NG) {
+        uint32_t pos = 0;
+        for (; id <= e; ++id) pos = ring_place(hd, (uint32_t)p.rec_stride, ring.cap);
         const long long wt0 = diag_clock(p);
-        if (lane == 0) bar_wait(&sm.hready[sq % kHr], (sq / kHr) & 1u, sm, p);
-        __syncwarp();
+        ring_wait_item_warp(item0 + e, sm, p);
         f_wait += diag_clock(p) - wt0;
-        const float* hp = sm.hpart[sq % kHr];
-        float sv[NVAL];
+        if (e == 0) stamp(p, l, 8);
+        float au[NB], ag[NB];
+        record_dot<FAM, ACT, NB>(base + pos, xsa, p, nunits, 32 * kq + lane, 32 * KG, au, ag);
+        float v[V];
 #pragma unroll
-        for (int i = 0; i < NVAL; ++i) {
-          float a = hp[i];
-#pragma unroll
-          for (int k = 1; k < KG; ++k) a += hp[k * NVAL + i];
-          sv[i] = a;
-        }
-        const float bi = lds_f32(base + pa + (uint32_t)p.bias_off);
-        const uint32_t bits = sm.list_bits[ea];
-        float h[NB];
+        for (int i = 0; i < V; ++i) v[i] = 0.f;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          float a;
-          if constexpr (ACT == PI_REGLU) a = fmaxf(sv[b * NV + 1] + bi, 0.f) * sv[b * NV];
-          else a = fmaxf(sv[b * NV] + bi, 0.f);
-          h[b] = (b < B && ((bits >> b) & 1u)) ? a : 0.f;
+          v[b * NV] = au[b];
+          if constexpr (ACT == PI_REGLU) v[b * NV + 1] = ag[b];
         }
-        const uint32_t drow = base + pa + (uint32_t)p.down_off;
-#pragma unroll
-        for (int j = 0; j < NU; ++j)
-          if (t + kConsumerThreads * j < nunits) unit_axpy<FAM, NB>(drow, d, t + kConsumerThreads * j, h, y[j]);
-        ring_release_item(item0 + ea, sm);
-      }
-      ring.item = item0 + (uint32_t)nlist;
-      fseq += (uint32_t)nlist;
-      if (t == 0) mbar_arrive(&sm.f_done);
-      stamp(p, l, 20);
-      stamp_val(p, l, 19, f_wait);
-      stamp_val(p, l, 21, d_wait);
-    }
-    // publish the partial y of this block as tagged words
-    {
-      uint64_t* part = p.px + (size_t)c * B * d;
-#pragma unroll
-      for (int b = 0; b < NB; ++b)
-#pragma unroll
-        for (int j = 0; j < NU; ++j) {
-          const int q = t + kConsumerThreads * j;
-          if (b < B && q < nunits) {
-            uint64_t* dst = part + (size_t)b * d + (size_t)q * UE;
-#pragma unroll
-            for (int e = 0; e < UE; e += 2) st_tag2(dst + e, y[j][b][e], y[j][b][e + 1], tag_p);
-          }
-        }
-    }
-    stamp(p, l, 4);
-
-    // ------------------------------------------------------------ R: slice reduce
-    if (slice_owner) {
-      // warp w sums partial rows cc = w, w+8, ...; KU rows' words are read together so
-      // the L2 round trips overlap; sums run in ascending cc (fixed order)
-      constexpr int KU = 10 / NB;   // 16 warps x 10 rows: all 148 partials in one round at one token
-      float acc[NB][kMaxColGroups];
-#pragma unroll
-      for (int b = 0; b < NB; ++b)
-#pragma unroll
-        for (int gq = 0; gq < kMaxColGroups; ++gq) acc[b][gq] = 0.f;
-      const uint64_t t0 = wait_start();
-      for (int gq = 0; gq < ng; ++gq) {
-        for (int cc0 = warp; cc0 < G; cc0 += kConsumerWarps * KU) {
-          float tmp[KU][NB];
-          uint32_t need = 0;
-#pragma unroll
-          for (int k = 0; k < KU; ++k)
+        const float sw = reduce_scatter<V>(v, lane);   // lane k: value k >> (5 - LG)
+        const uint32_t s = (fseq + (uint32_t)e) % kHr;
+        if ((lane & ((32 >> LG) - 1)) == 0 && (lane >> (5 - LG)) < NVAL) sm.hpart[s][kq * NVAL + (lane >> (5 - LG))] = sw;
+        const float bi = lds_f32(base + pos + (uint32_t)p.bias_off);
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence_block();
+          if (atomicAdd(&sm.hcnt[s], 1) == KG - 1) {
+            __threadfence_block();
+            const volatile float* hp = sm.hpart[s];
+            const int ent = sm.list_ent[e];
+            const uint32_t bits = sm.list_bits[e];
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
-              tmp[k][b] = 0.f;
-              if (cc0 + kConsumerWarps * k < G && b < B) need |= 1u << (k * NB + b);
-            }
-          while (need) {
-            uint64_t wk[KU][NB];
+              if (b < B) {
+                float su = hp[b * NV], sg = 0.f;
 #pragma unroll
-            for (int k = 0; k < KU; ++k)
+                for (int k = 1; k < KG; ++k) su += hp[k * NVAL + b * NV];
+                if constexpr (ACT == PI_REGLU) {
+                  sg = hp[b * NV + 1];
 #pragma unroll
-              for (int b = 0; b < NB; ++b) {
-                wk[k][b] = 0;
-                if (need >> (k * NB + b) & 1u)
-                  wk[k][b] = ld_tag(p.px + ((size_t)(cc0 + kConsumerWarps * k) * B + b) * d + col0 + 32 * gq + lane);
+                  for (int k = 1; k < KG; ++k) sg += hp[k * NVAL + b * NV + 1];
+                }
+                float a;
+                if constexpr (ACT == PI_REGLU) {
+                  a = fmaxf(sg + bi, 0.f) * su;
+                } else {
+                  a = fmaxf(su + bi, 0.f);
+                  if (p.act_square) a *= a;
+                }
+                st_tag(p.hx + (size_t)ent * B + b, ((bits >> b) & 1u) ? a : 0.f, tag_h);
               }
+            }
+            sm.hcnt[s] = 0;
+          }
+        }
+        ring_release_item(item0 + e, sm, (uint32_t)(kConsumerWarps / KG));
+      }
+      for (int q = 0; q < nlist; ++q) ring_place(ring.head, (uint32_t)p.rec_stride, ring.cap);
+      ring.item = item0 + (uint32_t)nlist;
+      fseq += (uint32_t)nlist;
+      stamp_val(p, l, 19, f_wait);
+    }
+    stamp(p, l, 9);
+
+    // ------------------------------------------------------------ down: y of the slice
+    float acc[NB][PE];
 #pragma unroll
-            for (int k = 0; k < KU; ++k)
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int e = 0; e < PE; ++e) acc[b][e] = 0.f;
+    long long h_wait = 0;   // diagnostics: cycles thread 0 polls for h
+    for (int k = 0; k < nchunks; ++k) {
+      cpa_wait_but_newest();   // this thread's copies of chunk k have landed
+      if (dw >= 0) {
+        const int lo = k * dch, hi = min(ntotal, lo + dch);
+        const int32_t* dl = dlist + (k & 1) * dch;
+        const int half = (k & 1) * dch;
+        constexpr int HB = NB == 1 ? 8 : NB == 2 ? 4 : 2;   // entries whose h words one polling round reads
+        for (int eb = lo + de0; eb < hi; eb += HB * dstep) {
+          uint64_t hw[HB][NB];
+          uint32_t need = 0;
+#pragma unroll
+          for (int q = 0; q < HB; ++q)
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+              hw[q][b] = 0;
+              if (eb + q * dstep < hi && b < B) need |= 1u << (q * NB + b);
+            }
+          const long long wt0 = diag_clock(p);
+          bool started = false;
+          uint64_t tp0 = 0;
+          while (need) {
+#pragma unroll
+            for (int q = 0; q < HB; ++q)
 #pragma unroll
               for (int b = 0; b < NB; ++b)
-                if ((need >> (k * NB + b) & 1u) && tag_ok(wk[k][b], tag_p)) {
-                  tmp[k][b] = tag_val(wk[k][b]);
-                  need &= ~(1u << (k * NB + b));
-                }
-            if (need && aborted(sm)) break;
-            if (need && timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
-            if (need && p.poll_ns) __nanosleep(p.poll_ns);
+                if (need >> (q * NB + b) & 1u) hw[q][b] = ld_tag(p.hx + (size_t)(eb + q * dstep) * B + b);
+#pragma unroll
+            for (int q = 0; q < HB; ++q)
+#pragma unroll
+              for (int b = 0; b < NB; ++b)
+                if ((need >> (q * NB + b) & 1u) && tag_ok(hw[q][b], tag_h)) need &= ~(1u << (q * NB + b));
+            if (!need || aborted(sm)) break;
+            if (!started) { tp0 = wait_start(); started = true; }
+            else if (timed_out(tp0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+            if (p.poll_ns) __nanosleep(p.poll_ns);
           }
+          h_wait += diag_clock(p) - wt0;
 #pragma unroll
-          for (int k = 0; k < KU; ++k)
+          for (int q = 0; q < HB; ++q) {
+            const int e = eb + q * dstep;
+            if (e < hi) {
+              float h[NB];
 #pragma unroll
-            for (int b = 0; b < NB; ++b) acc[b][gq] += tmp[k][b];
+              for (int b = 0; b < NB; ++b) h[b] = b < B ? tag_val(hw[q][b]) : 0.f;
+              const uint32_t slot = (uint32_t)((half + e - lo) * pmax + dw);
+              float sc = 0.f;
+              if constexpr (FAM == FAM_Q4) {
+                const uint32_t sw = lds_u32(dsc_u + slot * 4u);
+                sc = __half2float(__ushort_as_half((unsigned short)(((cu0 + dw) & 1) ? (sw >> 16) : (sw & 0xFFFFu))));
+              }
+              down_unit_fma<FAM, NB>(dbuf_u + slot * 16u, sc, h, acc);
+            }
+          }
         }
       }
+      if (k + 2 < nchunks) {
+        named_bar_sync(kRedBar, kConsumerThreads);   // every thread is done with dlist half k%2
+        build_dlist(k + 2);
+        named_bar_sync(kRedBar, kConsumerThreads);
+        issue_down(k + 2);
+      }
+      cpa_commit();
+    }
+    cpa_wait_all();
+    stamp_val(p, l, 17, h_wait);
+    stamp(p, l, 10);
+
+    // ------------------------------------------------------------ slice reduction
+    // The lanes of a warp that hold the same unit are summed by a butterfly over the lane
+    // bits above the unit bits; then the warps are summed in ascending order.
+    {
+      constexpr int V = NB * PE;
 #pragma unroll
       for (int b = 0; b < NB; ++b)
 #pragma unroll
-        for (int gq = 0; gq < kMaxColGroups; ++gq)
-          red2[((warp * NB + b) * kMaxColGroups + gq) * 32 + lane] = acc[b][gq];
-      named_bar_sync(kRedBar, kConsumerThreads);
-      // warp b finishes token b's columns, summing the warps' parts in a fixed order
-      if (warp < NB && warp < B) {
-        const int b = warp;
-        float sq = 0.f, sv = 0.f;
-#pragma unroll
-        for (int gq = 0; gq < kMaxColGroups; ++gq) {
-          if (gq < ng) {
-            float yv = 0.f;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) yv += red2[((w * NB + b) * kMaxColGroups + gq) * 32 + lane];
-            const int j = col0 + 32 * gq + lane;
-            if (do_glue) {
-              const float vv = xsl[gq] + yv;
-              xsl[gq] = vv;   // holds v until the glue turns it into the next input
-              sq += vv * vv;
-              sv += vv;
-              st_tag(p.vx + (size_t)b * d + j, vv, tag_v);
-              if (p.trace.y) p.trace.y[((size_t)l * B + b) * d + j] = yv;
-            } else {
-              p.y_out[(size_t)b * d + j] = yv;
-            }
-          }
+        for (int e = 0; e < PE; ++e) {
+          float v = acc[b][e];
+          for (int o = lpe; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          acc[b][e] = v;
         }
+      if (lane < lpe && dw >= 0) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int e = 0; e < PE; ++e) dred[(warp * pmax + dw) * V + b * PE + e] = acc[b][e];
+      }
+      named_bar_sync(kRedBar, kConsumerThreads);
+      float* vsl = dred + kConsumerWarps * pmax * V;   // [NB][ncol] v of the slice
+      if (t < B * ncol) {
+        const int b = t / ncol, q = t % ncol, w = q / PE, e = q % PE;
+        float y = 0.f;
+        for (int k = 0; k < kConsumerWarps; ++k) y += dred[(k * pmax + w) * V + b * PE + e];
+        const int col = col0 + q;
         if (do_glue) {
-          sq = warp_sum(sq);
-          sv = warp_sum(sv);
-          if (lane == 0) {
-            st_tag(p.sx + ((size_t)b * G + c) * 2, sv, tag_v);
-            st_tag(p.sx + ((size_t)b * G + c) * 2 + 1, sq, tag_v);
+          const float v = xs_val<FAM>(xs, b * d + col) + y;
+          vsl[b * ncol + q] = v;
+          st_tag(p.vx + (size_t)b * d + col, v, tag_v);
+          if (p.trace.y) p.trace.y[((size_t)l * B + b) * d + col] = y;
+        } else {
+          p.y_out[(size_t)b * d + col] = y;
+        }
+      }
+      if (!do_glue) break;
+      named_bar_sync(kRedBar, kConsumerThreads);
+      if (warp < NB) {
+        float s = 0.f, s2 = 0.f;
+        if (warp < B)
+          for (int q = lane; q < ncol; q += 32) {
+            const float v = vsl[warp * ncol + q];
+            s += v;
+            s2 += v * v;
           }
+        s = warp_sum(s);
+        s2 = warp_sum(s2);
+        if (lane == 0 && warp < B) {
+          st_tag(p.sx + ((size_t)warp * G + c) * 2, s, tag_v);
+          st_tag(p.sx + ((size_t)warp * G + c) * 2 + 1, s2, tag_v);
         }
       }
     }
-    if (!do_glue) break;
-    stamp(p, l, 6);
+    stamp(p, l, 11);
 
     // ------------------------------------------------------------ glue: x' = (v - mean) / sd
-    // One polling round reads both what the slice owners published: every thread polls its
-    // v pairs of the first chunk and a few of the slices' (sum, sum of squares) words.
+    // One polling round reads every v and every slice's (sum, sum of squares).
     {
       const int npairs = B * d / 2;
-      const int nmom = 2 * nslices * B;
+      const int nmom = 2 * G * B;
       constexpr int MQ = (2 * kMaxGrid * 4 + kConsumerThreads - 1) / kConsumerThreads;
       uint64_t w0[8], w1[8], wm[MQ];
       uint32_t need = 0, needm = 0;
@@ -1093,18 +1278,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       }
       {
         bool started = false;
-        uint64_t tp = 0;
+        uint64_t tp0 = 0;
         while (need | needm) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             if (need >> k & 1u) ld_tag2(p.vx + 2 * (size_t)(t + k * kConsumerThreads), w0[k], w1[k]);
 #pragma unroll
           for (int i = 0; i < MQ; ++i)
-            if (needm >> i & 1u) {
-              const int q = t + i * kConsumerThreads;
-              const int bq = q / (2 * nslices), cq = (q >> 1) % nslices;
-              wm[i] = ld_tag(p.sx + ((size_t)bq * G + cq) * 2 + (q & 1));
-            }
+            if (needm >> i & 1u) wm[i] = ld_tag(p.sx + t + i * kConsumerThreads);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             if ((need >> k & 1u) && tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
@@ -1112,14 +1293,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           for (int i = 0; i < MQ; ++i)
             if ((needm >> i & 1u) && tag_ok(wm[i], tag_v)) needm &= ~(1u << i);
           if (!(need | needm) || aborted(sm)) break;
-          if (!started) { tp = wait_start(); started = true; }
-          else if (timed_out(tp, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+          if (!started) { tp0 = wait_start(); started = true; }
+          else if (timed_out(tp0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
           if (p.poll_ns) __nanosleep(p.poll_ns);
         }
       }
-      named_bar_sync(kRedBar, kConsumerThreads);   // the slice reduce is done with red2; nobody reads xs
-      stamp(p, l, 16);
-      float* mom = red2;                            // [B][nslices][2]
+      named_bar_sync(kRedBar, kConsumerThreads);   // nobody reads vsl or xs any more
+      stamp(p, l, 12);
+      float* mom = dred;                            // [B][G][2]
 #pragma unroll
       for (int i = 0; i < MQ; ++i)
         if (t + i * kConsumerThreads < nmom) mom[t + i * kConsumerThreads] = tag_val(wm[i]);
@@ -1127,9 +1308,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       if (warp < NB) {
         float s = 0.f, s2 = 0.f;
         if (warp < B)
-          for (int cq = lane; cq < nslices; cq += 32) {
-            s += mom[(warp * nslices + cq) * 2];
-            s2 += mom[(warp * nslices + cq) * 2 + 1];
+          for (int cq = lane; cq < G; cq += 32) {
+            s += mom[(warp * G + cq) * 2];
+            s2 += mom[(warp * G + cq) * 2 + 1];
           }
         const float sum = warp_sum(s);
         s2 = warp_sum(s2);
@@ -1137,7 +1318,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           const float mean = sum / (float)d;
           const float var = fmaxf(s2 / (float)d - mean * mean, 0.f);
           sm.gmean[warp] = mean;
-          sm.gsd[warp] = sqrtf(var + kRmsEps);
+          sm.gsd[warp] = sqrtf(var + kNormEps);
         }
       }
       named_bar_sync(kRedBar, kConsumerThreads);
@@ -1160,7 +1341,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         for (int k = 0; k < 8; ++k)
           if (base + t + k * kConsumerThreads < npairs) need |= 1u << k;
         bool started = false;
-        uint64_t tp = 0;
+        uint64_t tp0 = 0;
         while (need) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
@@ -1169,8 +1350,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           for (int k = 0; k < 8; ++k)
             if ((need >> k & 1u) && tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
           if (!need || aborted(sm)) break;
-          if (!started) { tp = wait_start(); started = true; }
-          else if (timed_out(tp, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+          if (!started) { tp0 = wait_start(); started = true; }
+          else if (timed_out(tp0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
           if (p.poll_ns) __nanosleep(p.poll_ns);
         }
 #pragma unroll
@@ -1184,23 +1365,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           }
         }
       }
-      stamp(p, l, 17);
-      // slice owners: the new input of their slice, the trace, and the output
-      if (slice_owner && warp < NB && warp < B) {
-        const int b = warp;
-        const float mean = sm.gmean[b], sd = sm.gsd[b];
-#pragma unroll
-        for (int gq = 0; gq < kMaxColGroups; ++gq)
-          if (gq < ng) {
-            const size_t j = (size_t)b * d + col0 + 32 * gq + lane;
-            xsl[gq] = round_act<FAM>((xsl[gq] - mean) / sd);
-            if (p.trace.x) store_act<FAM>(p.trace.x, (size_t)(l + 1) * B * d + j, xsl[gq]);
-            if (l == p.L - 1) store_act<FAM>(p.x_out, j, xsl[gq]);
-          }
-      }
       named_bar_sync(kRedBar, kConsumerThreads);
+      // every block writes its own columns of the trace and of the output
+      if (p.trace.x || l == p.L - 1)
+        for (int q = t; q < B * ncol; q += kConsumerThreads) {
+          const int b = q / ncol;
+          const size_t j = (size_t)b * d + col0 + q % ncol;
+          const float xv = xs_val<FAM>(xs, (int)j);
+          if (p.trace.x) store_act<FAM>(p.trace.x, (size_t)(l + 1) * B * d + j, xv);
+          if (l == p.L - 1) store_act<FAM>(p.x_out, j, xv);
+        }
     }
-    stamp(p, l, 8);
+    stamp(p, l, 13);
   }
 
   // last block out: advance the epoch (new tags for the next launch) and reset the count
@@ -1209,7 +1385,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     __threadfence();
     const uint32_t prev = atomicAdd(p.bar + 1, 1u);
     if (prev == (uint32_t)G - 1) {
-      atomicExch(p.bar + 2, epoch + 1u);
+      atomicExch(p.bar + 2, next_launch_epoch(epoch));
       atomicExch(p.bar + 1, 0u);
     }
   }
@@ -1255,8 +1431,8 @@ __global__ void __launch_bounds__(kThreads, 1) barrier_probe_kernel(const FusedP
 constexpr int ue_of(int fam) { return fam == FAM_F32 ? 4 : fam == FAM_F16 ? 8 : 16; }
 
 // Largest d_model each (family, tokens) pair serves, and the unit count per consumer
-// thread that covers it; a launch takes the smallest count that covers its d, so x and y
-// in registers stay small.
+// thread that covers it; a launch takes the smallest count that covers its d, so x in
+// registers stays small.
 constexpr int d_max_of(int fam, int nb) {
   return fam == FAM_F32 ? (nb == 4 ? 2048 : 4096)
                         : fam == FAM_F16 ? (nb == 1 ? 12288 : nb == 2 ? 8192 : 4096) : (nb <= 2 ? 8192 : 0);
@@ -1307,6 +1483,8 @@ cudaError_t launch_nb(int B, const FusedParams& p, size_t smem, cudaStream_t str
   return cudaErrorNotSupported;
 }
 
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
 }  // namespace
 
 bool fused_supported(int family, int B, int d) {
@@ -1315,13 +1493,59 @@ bool fused_supported(int family, int B, int d) {
   return d <= d_max_of(family, nb);
 }
 
-size_t fused_fixed_smem(int B, int d, int r, int grid, int nown_max, int family) {
-  const int nb = nb_of(B) ? nb_of(B) : 4;
+bool fused_plan_smem(FusedParams& p, int family, size_t budget, size_t& smem_bytes) {
+  const int nb = nb_of(p.B);
+  if (nb == 0) return false;
+  const int G = p.grid;
   const size_t xbytes = family == FAM_F32 ? 4 : 2;
-  return ((sizeof(Smem) + 127) / 128) * 128 + (size_t)nb * d * xbytes + (size_t)nb * r * sizeof(float) +
-         (size_t)kConsumerWarps * nb * kMaxColGroups * 32 * sizeof(float) + 128;
+  const int pe = down_unit_elems(family);
+  p.nw = (p.nown_max + 31) / 32;
+  p.dunits = p.d / pe;
+  p.pmax = (p.dunits + G - 1) / G;
+  if (p.nw > kMaxOwnWords || p.pmax > kMaxPieces || p.pmax < 1) return false;
+  // ring items: whole neuron records; P1^T rows grouped into ~32 KB copies; the block's own
+  // P2 rows in copies of up to 48 KB
+  const int cap = std::max(p.rec_stride, 32 * 1024);
+  p.p1_rows_per_item = std::max(1, cap / p.p1_row);
+  p.p2_item_bytes = std::max(cap, 48 * 1024);
+  // the largest copy of predictor rows any layer makes: its rows per copy times its stride,
+  // at most max(p2_item_bytes, one row of the largest rank)
+  const long long max_p2_item = std::max((long long)p.p2_item_bytes, (long long)p.p2_stride);
+  const long long max_item = std::max({(long long)p.rec_stride, (long long)p.p1_rows_per_item * p.p1_row,
+                                       max_p2_item});
+  const size_t dred_floats = std::max((size_t)(kConsumerWarps + 1) * p.pmax * nb * pe, (size_t)nb * G * 2);
+  size_t off = round_up(sizeof(Smem), 128);
+  const size_t fixed_tail = round_up((size_t)nb * p.d * xbytes, 16) + round_up((size_t)nb * p.r * 4, 16) +
+                            round_up((size_t)G * nb * p.nw * 4, 16) + round_up(dred_floats * 4, 16);
+  // per chunk entry: its dlist slot and its units (plus a scale word per Q4_0 unit), twice
+  const size_t entry_bytes = 2 * (4 + (size_t)p.pmax * 16 + (family == FAM_Q4 ? (size_t)p.pmax * 4 : 0));
+  const size_t ring_min = std::max((size_t)112 * 1024, (size_t)(2 * max_item));
+  if (budget < off + fixed_tail + ring_min + 64 * entry_bytes + 256) return false;
+  size_t dch = (budget - off - fixed_tail - ring_min - 256) / entry_bytes;
+  dch = std::min(dch, (size_t)kMaxDch);
+  p.dch = (int)dch;
+  const size_t down_bytes = round_up(dch * entry_bytes, 128);
+  p.ring_bytes = (int)((budget - off - fixed_tail - down_bytes - 256) / 128 * 128);
+  if (p.ring_bytes < 2 * max_item || max_item >= (1 << 20)) return false;
+  p.off_ring = (int)off;
+  off += (size_t)p.ring_bytes;
+  p.off_xs = (int)off;
+  off += round_up((size_t)nb * p.d * xbytes, 16);
+  p.off_us = (int)off;
+  off += round_up((size_t)nb * p.r * 4, 16);
+  p.off_ob = (int)off;
+  off += round_up((size_t)G * nb * p.nw * 4, 16);
+  p.off_dred = (int)off;
+  off += round_up(dred_floats * 4, 16);
+  p.off_dlist = (int)off;
+  off += round_up((size_t)2 * dch * 4, 16);
+  p.off_dbuf = (int)off;
+  off += (size_t)2 * dch * p.pmax * 16;
+  p.off_dsc = (int)off;
+  off += family == FAM_Q4 ? (size_t)2 * dch * p.pmax * 4 : 0;
+  smem_bytes = round_up(off, 128);
+  return smem_bytes <= budget;
 }
-
 
 cudaError_t launch_fused(int family, int act, int B, const FusedParams& p, size_t smem, cudaStream_t stream) {
   if (family == FAM_F32)

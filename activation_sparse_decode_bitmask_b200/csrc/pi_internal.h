@@ -19,6 +19,16 @@ enum DevErr : int {
   DEV_ERR_BAD_FREQ = 5,       // a non-finite firing frequency
 };
 
+// Launch epochs tag the cross-block exchange words (tag = epoch * 1024 + layer * 8 +
+// exchange, 32 bits).  An epoch that is a multiple of 2^22 would give layer 0's first
+// exchange the tag 0, the tag of a cleared word, so such epochs are skipped.
+constexpr uint32_t kEpochWrap = 1u << 22;
+__host__ __device__ inline uint32_t next_launch_epoch(uint32_t e) {
+  ++e;
+  if (e % kEpochWrap == 0) ++e;
+  return e;
+}
+
 // dtype families (w, x, p)
 enum Family : int { FAM_F32 = 0, FAM_F16 = 1, FAM_Q4 = 2 };
 
@@ -27,19 +37,26 @@ constexpr int kConsumerWarps = 16;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;
 constexpr int kMaxOwn = 512;          // owned neurons per block (d_ff <= 512 * grid)
+constexpr int kMaxOwnWords = kMaxOwn / 32;
+constexpr int kMaxPieces = 16;        // 16-byte down units one block owns
 constexpr int kMaxList = 512;         // active neurons a block may process in one layer
 constexpr int kMaxLayers = 100;       // layers of one pi_decode_stack call
 constexpr int kMaxGrid = 256;         // blocks of the fused kernel (SMs)
 constexpr int kDiagSlots = 64;        // diagnostic stamps per block and layer
 
-// Library-owned, re-laid-out layer.
+// Library-owned, re-laid-out layer, as the fused kernel sees it.
 struct LayerDev {
-  const uint8_t* rec;     // [f][rec_stride]   per-neuron record [gate][up][down]
+  const uint8_t* rec;     // [f][rec_stride] per-neuron record [gate row][up row][16-byte header: bias],
+                          // followed by the down rows [f][dn_stride] (neuron-major)
   const uint8_t* p1t;     // [r][p1_row]       P1 transposed, p_dtype
-  const uint8_t* p2o;     // [G][nown_max][p2_stride] predictor row + (t, b) of neuron c + m*G
-  int hot;                // hot-prefix length at this call's batch, 0 = none
-  int keep_floor;         // records every block keeps of its own before balancing (0 = none)
+  const uint8_t* p2o;     // [G][nown_max][p2_stride(r)] predictor row + (t, b) of neuron c + m*G
+  int keep_floor;         // own records every block keeps before the mask exchange (0 = none)
+  int r;                  // this layer's predictor rank (layers of one stack may differ)
 };
+
+// Bytes of one owner-major predictor row of rank r: r values of p_bytes, then (t, b),
+// rounded to 16.
+__host__ __device__ inline int p2_stride_of(int r, int p_bytes) { return (r * p_bytes + 8 + 15) / 16 * 16; }
 
 }  // namespace pi
 
@@ -47,14 +64,16 @@ struct pi_layer {
   pi_layer_desc desc;
   int family;
   int row_bytes;    // one weight row (d elements) in the record
-  int rec_stride;   // bytes per neuron record (gate? + up + down), multiple of 16
-  int gate_off, up_off, down_off;   // byte offsets of the rows in a record (gate_off -1 for ReLU)
+  int rec_stride;   // bytes per neuron record (gate? + up + bias header), multiple of 16
+  int gate_off, up_off;   // byte offsets of the rows in a record (gate_off -1 for ReLU)
   int bias_off;     // byte offset of the record's 16-byte header holding the bias (f32)
+  int dn_stride;    // bytes per down row (multiple of 16)
+  size_t dn_off;    // byte offset of the down rows in the record allocation (f * rec_stride)
   int p1_row;       // bytes of one P1^T row (d * p_bytes)
   int p2_stride;    // bytes per neuron predictor row (r * p_bytes + 8, rounded to 16)
   int G;            // blocks the owner-major predictor layout was built for (the SM count)
   int nown_max;     // ceil(f / G): predictor rows per block, padded
-  uint8_t* rec;
+  uint8_t* rec;     // records, then the down rows
   uint8_t* p1t;
   uint8_t* p2o;
   float* bias;      // [f] stored order
@@ -64,7 +83,6 @@ struct pi_layer {
   float* freq_host;    // host copy of freq_sorted (descending), or null
   int keep_floor[4];   // per batch 1..4: own records every block keeps before balancing
   int hot_count;    // -1: derived per batch from freq_sorted
-  int hot_len_b[33];   // per batch 1..32: hot-prefix length (set with freq_host)
   int device;
 };
 
@@ -73,11 +91,10 @@ struct pi_workspace {
   int grid;          // blocks of the fused kernel (one per SM)
   int device;
   uint64_t* ux;      // [B_max][r_max]          tagged u
-  uint64_t* px;      // [grid][B_max][d_max]    tagged y partials
+  uint64_t* mx;      // [grid][4][kMaxOwnWords] tagged own mask words
+  uint64_t* hx;      // [f_max][B_max]          tagged h of the active neurons
   uint64_t* vx;      // [B_max][d_max]          tagged x + y
-  uint64_t* sx;      // [B_max][grid][2]        tagged slice sums and sums of squares
-  uint64_t* cx;      // [grid]                  tagged own active counts (balance)
-  uint64_t* lx;      // [grid][kMaxOwn]         tagged own active list entries (balance)
+  uint64_t* sx;      // [B_max][grid][2]        tagged column-slice sums and sums of squares
   uint32_t* bar;     // [0] probe barrier count, [1] exit count, [2] launch epoch (tags)
   int* err;          // device error word
   unsigned long long* active_total;  // running sum of active-list lengths (all calls)
@@ -107,12 +124,22 @@ void note_launch();
 // Parameters of one launch of the fused kernel.
 struct FusedParams {
   int mode;            // bit 1: predictor, bit 2: FFN, bit 4: stack glue (layer loop)
-  int L, B, d, f, r;
+  int L, B, d, f;
+  int r;               // the largest predictor rank of the launch's layers (u buffer size)
   int grid;
-  int row_bytes, rec_stride, gate_off, up_off, down_off, bias_off, p1_row, p2_stride;
-  int ring_bytes, p1_rows_per_item, p2_rows_per_item, nown_max;
-  int rec_window;      // ring_bytes / rec_stride - 2: at least 1, so three records fit in the ring
-  int nslices;
+  int row_bytes, rec_stride, gate_off, up_off, bias_off, p1_row, p2_stride;
+  int dn_stride;       // bytes per down row
+  int act_square;      // squared ReLU: h = max(0, up + b)^2 (the ReLU instantiation squares)
+  long long dn_off;    // byte offset of the down rows behind a layer's records
+  int ring_bytes, p1_rows_per_item, nown_max;
+  int inflight_budget; // bytes of bulk copies one block keeps in flight at most (one item at least)
+  int p2_item_bytes;   // target bytes of one copy of predictor rows (a layer's rows per copy follow)
+  int nw;              // 32-bit words of one block's own bits per token: ceil(nown_max / 32)
+  int dunits;          // 16-byte down units of a row: d/4 (fp32), d/8 (fp16), d/32 (Q4_0 blocks)
+  int pmax;            // most down units one block owns: ceil(dunits / grid), <= kMaxPieces
+  int dch;             // active entries per down chunk (each chunk's rows fit one half of dbuf)
+  // dynamic shared-memory layout (byte offsets)
+  int off_ring, off_xs, off_us, off_ob, off_dlist, off_dbuf, off_dsc, off_dred;
   LayerDev layers[kMaxLayers];
   // inputs / outputs
   const void* x_in;          // [B][d] activation dtype
@@ -126,11 +153,10 @@ struct FusedParams {
   pi_trace trace;            // (stack)
   // workspace
   uint64_t* ux;
-  uint64_t* px;
+  uint64_t* mx;
+  uint64_t* hx;
   uint64_t* vx;
   uint64_t* sx;
-  uint64_t* cx;        // tagged own active counts [grid]; null: no balancing (each block keeps its own)
-  uint64_t* lx;        // tagged own active list entries [grid][kMaxOwn]
   uint32_t* bar;
   int* err;
   unsigned long long* active_total;
@@ -147,7 +173,9 @@ enum : int { MODE_PREDICT = 1, MODE_FFN = 2, MODE_GLUE = 4 };
 
 cudaError_t launch_fused(int family, int act, int B, const FusedParams& p, size_t smem_bytes,
                          cudaStream_t stream);
-size_t fused_fixed_smem(int B, int d, int r, int grid, int nown_max, int family);
+// Fills the shared-memory layout, item sizes and down-chunk geometry of `p` (whose shape,
+// record and grid fields are set) within `budget` bytes; false if the shape does not fit.
+bool fused_plan_smem(FusedParams& p, int family, size_t budget, size_t& smem_bytes);
 bool fused_supported(int family, int B, int d);
 cudaError_t launch_barrier_probe(const FusedParams& p, int rounds, cudaStream_t stream);
 
@@ -155,13 +183,16 @@ cudaError_t launch_barrier_probe(const FusedParams& p, int rounds, cudaStream_t 
 struct BatchedLayer {
   int d, f, r, G, nown_max;
   const uint8_t* rec;
-  int rec_stride, up_off, gate_off, down_off;
+  int rec_stride, up_off, gate_off;
+  const uint8_t* dn;     // down rows [f][dn_stride]
+  int dn_stride;
   const uint8_t* p1t;
   int p1_row;
   const uint8_t* p2o;
   int p2_stride;
   const float* thresh;
   const float* bias;
+  int act_square;        // squared ReLU
 };
 bool batched_supported(int family, int B, int d, int r);
 cudaError_t batched_predict(const BatchedLayer& L, const void* x, int B, uint32_t* mask, float* logits,

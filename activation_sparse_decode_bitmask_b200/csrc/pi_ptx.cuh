@@ -108,3 +108,19 @@ __device__ __forceinline__ float2 h2f2(uint32_t v) {
 }
 
 }  // namespace pi
+
+namespace pi {
+// ---------------------------------------------------------------- per-thread async copies
+// cp.async (global -> shared, completion tracked per thread by commit groups): 16 bytes
+// through L2 only, or 4 bytes.  Both addresses aligned to the copy size.
+__device__ __forceinline__ void cpa16(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa4(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// every group but the newest one has landed
+__device__ __forceinline__ void cpa_wait_but_newest() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cpa_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+}  // namespace pi

@@ -1,16 +1,22 @@
 // Row arithmetic of the fused kernel.
 //
-// Consumer thread t owns the units q = t + kConsumerThreads * j (j < NU) of every d-long
-// row: 4 elements for fp32, 8 for fp16 and 16 (half a Q4_0 block) for Q4_0.  It keeps
-// its units of every token's x and y in registers as fp32 for a whole layer, so a row's
-// dot product is a per-thread partial sum over the thread's units (the caller reduces
-// the partials across the block) and the down projection y += h * row needs no
-// cross-thread step at all.
+// Consumer thread t owns the units q = t + kConsumerThreads * j (j < NU) of a d-long
+// row: 4 elements for fp32, 8 for fp16 and 16 (half a Q4_0 block) for Q4_0.  It keeps its
+// units of every token's x in registers for the predictor's first stage, and a row's dot
+// product is a per-thread partial sum over the thread's units (the caller reduces the
+// partials across the warp and the block).
+//
+// x units are kept as they are stored: fp32 values for the fp32 family, fp16 pairs for the
+// fp16 and Q4_0 families.  fp16 weights meet fp16 x through fma.rn.f32.f16: the product of
+// two fp16 values is exact in fp32, so only the fp32 sums round.
 //
 // Q4_0 rows: 32-weight blocks; the row holds the 16 nibble bytes of every block (byte j
 // has element j in its low four bits and element j + 16 in its high four bits), then the
 // fp16 scales of all its blocks.  Value = (code - 8) * scale.  A unit is the low or the
-// high nibbles of one block.  Products and sums are formed in fp32.
+// high nibbles of one block.  Two codes become one fp16 pair exactly: a code q under the
+// exponent pattern of 1024 is the fp16 value 1024 + q, and one packed subtraction of 1032
+// leaves q - 8 (integers below 2048 are exact in fp16).  The pair then meets x like an
+// fp16 weight pair, and the block's scale multiplies the unit's sum once.
 #pragma once
 #include <cuda_fp16.h>
 #include <cstdint>
@@ -22,11 +28,11 @@ namespace pi {
 
 template <int FAM> struct Fam;
 // UE: elements per unit; PB: bytes per predictor element; XW: 32-bit registers that hold
-// one token's unit of x (fp32 values, or fp16 pairs for the fp16 family, whose dots use
-// fp16 x fp16 products accumulated in fp32)
+// one token's unit of x (fp32 values, or fp16 pairs for the fp16 and Q4_0 families, whose
+// dots use fp16 x fp16 products accumulated in fp32)
 template <> struct Fam<FAM_F32> { static constexpr int UE = 4;  static constexpr int PB = 4; static constexpr int XW = 4;  using X = float; };
 template <> struct Fam<FAM_F16> { static constexpr int UE = 8;  static constexpr int PB = 2; static constexpr int XW = 4;  using X = __half; };
-template <> struct Fam<FAM_Q4>  { static constexpr int UE = 16; static constexpr int PB = 2; static constexpr int XW = 16; using X = __half; };
+template <> struct Fam<FAM_Q4>  { static constexpr int UE = 16; static constexpr int PB = 2; static constexpr int XW = 8;  using X = __half; };
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -78,23 +84,14 @@ __device__ __forceinline__ void fma2_h(uint32_t w2, uint32_t x2, float& acc, flo
 template <int FAM, int NB>
 __device__ __forceinline__ void load_x_unit(const void* xs, int d, int q, uint32_t (&xu)[NB][Fam<FAM>::XW]) {
   constexpr int UE = Fam<FAM>::UE;
+  constexpr int XB = FAM == FAM_F32 ? 4 : 2;
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
-    if constexpr (FAM == FAM_F32) {
-      const uint4 v = reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(xs) + (size_t)b * d)[q];
-      xu[b][0] = v.x; xu[b][1] = v.y; xu[b][2] = v.z; xu[b][3] = v.w;
-    } else if constexpr (FAM == FAM_F16) {
-      const uint4 v = reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(xs) + (size_t)b * d)[q];
-      xu[b][0] = v.x; xu[b][1] = v.y; xu[b][2] = v.z; xu[b][3] = v.w;
-    } else {
-      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(xs) + (size_t)b * d + UE * q);
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(xs) + (size_t)XB * (b * d + UE * q));
 #pragma unroll
-      for (int c = 0; c < UE / 8; ++c) {
-        float w[8];
-        widen8(src[c], w);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xu[b][8 * c + e] = __float_as_uint(w[e]);
-      }
+    for (int c = 0; c < Fam<FAM>::XW / 4; ++c) {
+      const uint4 v = src[c];
+      xu[b][4 * c] = v.x; xu[b][4 * c + 1] = v.y; xu[b][4 * c + 2] = v.z; xu[b][4 * c + 3] = v.w;
     }
   }
 }
@@ -107,19 +104,21 @@ __device__ __forceinline__ void lds_x_unit(uint32_t xs, int d, int q, uint32_t (
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
     const uint32_t a = xs + XB * (uint32_t)(b * d + UE * q);
-    if constexpr (FAM == FAM_F32 || FAM == FAM_F16) {
-      const uint4 v = lds128(a);
-      xu[b][0] = v.x; xu[b][1] = v.y; xu[b][2] = v.z; xu[b][3] = v.w;
-    } else {
 #pragma unroll
-      for (int c = 0; c < UE / 8; ++c) {
-        float w[8];
-        widen8(lds128(a + 16u * c), w);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xu[b][8 * c + e] = __float_as_uint(w[e]);
-      }
+    for (int c = 0; c < Fam<FAM>::XW / 4; ++c) {
+      const uint4 v = lds128(a + 16u * c);
+      xu[b][4 * c] = v.x; xu[b][4 * c + 1] = v.y; xu[b][4 * c + 2] = v.z; xu[b][4 * c + 3] = v.w;
     }
   }
+}
+
+// Two Q4_0 codes (bytes k and k + 1 of `codes`, each 0..15) as the fp16 pair
+// (code_k - 8, code_{k+1} - 8), exactly: 0x64cc is the fp16 value 1024 + cc.
+template <int K>
+__device__ __forceinline__ uint32_t q4_pair(uint32_t codes) {
+  const uint32_t biased = __byte_perm(codes, 0x00006464u, K == 0 ? 0x5140u : 0x5342u);
+  const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&biased), __floats2half2_rn(1032.f, 1032.f));
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 // acc[b] += (unit q of a weight row) . xu[b]
@@ -151,16 +150,17 @@ __device__ __forceinline__ void unit_dot(uint32_t row, int d, int q, const uint3
     const int sh = (q & 1) * 4;
     const uint32_t wv[4] = {(nb.x >> sh) & 0x0F0F0F0Fu, (nb.y >> sh) & 0x0F0F0F0Fu, (nb.z >> sh) & 0x0F0F0F0Fu,
                             (nb.w >> sh) & 0x0F0F0F0Fu};
+    uint32_t wp[8];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      wp[2 * m] = q4_pair<0>(wv[m]);       // elements 4m, 4m + 1 of the unit
+      wp[2 * m + 1] = q4_pair<1>(wv[m]);   // elements 4m + 2, 4m + 3
+    }
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       float s = 0.f, s2 = 0.f;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        s = fmaf(q4_val(wv[m], 0), __uint_as_float(xu[b][4 * m]), s);
-        s2 = fmaf(q4_val(wv[m], 1), __uint_as_float(xu[b][4 * m + 1]), s2);
-        s = fmaf(q4_val(wv[m], 2), __uint_as_float(xu[b][4 * m + 2]), s);
-        s2 = fmaf(q4_val(wv[m], 3), __uint_as_float(xu[b][4 * m + 3]), s2);
-      }
+      for (int k = 0; k < 8; ++k) fma2_h(wp[k], xu[b][k], s, s2);
       acc[b] = fmaf(sc, s + s2, acc[b]);
     }
   }
@@ -175,60 +175,18 @@ __device__ __forceinline__ void unit_dot_p(uint32_t row, int q, const uint32_t (
   if constexpr (FAM == FAM_F32 || FAM == FAM_F16) {
     unit_dot<FAM, NB>(row, 0, q, xu, acc);
   } else {
+    // fp16 predictor row: 16 elements per unit, two 16-byte chunks
     const uint32_t src = row + (uint32_t)q * UE * 2;
-#pragma unroll
-    for (int c = 0; c < UE / 8; ++c) {
-      float w[8];
-      widen8(lds128(src + 16u * c), w);
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        float s = acc[b], s2 = w[4] * __uint_as_float(xu[b][8 * c + 4]);
-        s = fmaf(w[0], __uint_as_float(xu[b][8 * c + 0]), s); s2 = fmaf(w[5], __uint_as_float(xu[b][8 * c + 5]), s2);
-        s = fmaf(w[1], __uint_as_float(xu[b][8 * c + 1]), s); s2 = fmaf(w[6], __uint_as_float(xu[b][8 * c + 6]), s2);
-        s = fmaf(w[2], __uint_as_float(xu[b][8 * c + 2]), s); s2 = fmaf(w[7], __uint_as_float(xu[b][8 * c + 7]), s2);
-        s = fmaf(w[3], __uint_as_float(xu[b][8 * c + 3]), s);
-        acc[b] = s + s2;
-      }
-    }
-  }
-}
-
-// yu[b] += h[b] * (unit q of a weight row)
-template <int FAM, int NB>
-__device__ __forceinline__ void unit_axpy(uint32_t row, int d, int q, const float (&h)[NB],
-                                          float (&yu)[NB][Fam<FAM>::UE]) {
-  if constexpr (FAM == FAM_F32) {
-    const float4 w = u4f(lds128(row + 16u * q));
+    const uint4 w0 = lds128(src), w1 = lds128(src + 16u);
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      yu[b][0] = fmaf(h[b], w.x, yu[b][0]); yu[b][1] = fmaf(h[b], w.y, yu[b][1]);
-      yu[b][2] = fmaf(h[b], w.z, yu[b][2]); yu[b][3] = fmaf(h[b], w.w, yu[b][3]);
+      float s = acc[b], s2 = 0.f;
+      fma2_h(w0.x, xu[b][0], s, s2); fma2_h(w0.y, xu[b][1], s, s2);
+      fma2_h(w0.z, xu[b][2], s, s2); fma2_h(w0.w, xu[b][3], s, s2);
+      fma2_h(w1.x, xu[b][4], s, s2); fma2_h(w1.y, xu[b][5], s, s2);
+      fma2_h(w1.z, xu[b][6], s, s2); fma2_h(w1.w, xu[b][7], s, s2);
+      acc[b] = s + s2;
     }
-  } else if constexpr (FAM == FAM_F16) {
-    float w[8];
-    widen8(lds128(row + 16u * q), w);
-#pragma unroll
-    for (int b = 0; b < NB; ++b)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) yu[b][e] = fmaf(h[b], w[e], yu[b][e]);
-  } else {
-    const int blk = q >> 1;
-    const uint4 nb = lds128(row + 16u * blk);
-    const float sc = lds_h2f(row + (uint32_t)(d >> 1) + 2u * blk);
-    const int sh = (q & 1) * 4;
-    const uint32_t wv[4] = {(nb.x >> sh) & 0x0F0F0F0Fu, (nb.y >> sh) & 0x0F0F0F0Fu, (nb.z >> sh) & 0x0F0F0F0Fu,
-                            (nb.w >> sh) & 0x0F0F0F0Fu};
-    float hs[NB];
-#pragma unroll
-    for (int b = 0; b < NB; ++b) hs[b] = h[b] * sc;
-#pragma unroll
-    for (int m = 0; m < 4; ++m)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float cv = q4_val(wv[m], k);
-#pragma unroll
-        for (int b = 0; b < NB; ++b) yu[b][4 * m + k] = fmaf(hs[b], cv, yu[b][4 * m + k]);
-      }
   }
 }
 

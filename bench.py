@@ -35,7 +35,8 @@ import pi_synth as S  # noqa: E402
 
 METRIC = "decode tokens/s of sparse FFN stack at batch 1; active-bytes HBM GB/s vs peak"
 WORKLOADS = {"llama2_7b": S.LLAMA2_7B, "falcon40b": S.FALCON_40B, "llama2_70b_q4": S.LLAMA2_70B_Q4,
-             "opt175b": S.OPT_175B, "ffn512_cal": S.FFN512_CAL, "ffn512_lit": S.FFN512_LIT}
+             "opt175b": S.OPT_175B, "ffn512_cal": S.FFN512_CAL, "ffn512_lit": S.FFN512_LIT,
+             "llama2_7b_adaptive": S.LLAMA2_7B_ADAPTIVE}
 CSRC = os.path.join(ROOT, "activation_sparse_decode_bitmask_b200", "csrc")
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 
@@ -54,6 +55,11 @@ def bytes_per_neuron(wl):
 def predictor_bytes(wl):
     """P1 + P2 + thresholds per layer (read densely every step)."""
     return wl.d_model * wl.rank * p_bytes(wl) + wl.rank * wl.d_ff * p_bytes(wl) + 4 * wl.d_ff
+
+
+def stack_predictor_bytes(wl):
+    """Predictor bytes of one step through the whole stack (layers may differ in rank)."""
+    return sum(predictor_bytes(wl.at_layer(l)) for l in range(wl.n_layers))
 
 
 FUSED_SOURCES = ("pi_fused.cu", "pi_rowmath.cuh", "pi_ptx.cuh")
@@ -181,41 +187,64 @@ def dist_barrier(world):
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_tokens_per_s(wl, budget_s=15.0, batch=1, device="cuda"):
-    """Time the oracle's decode of one token layer by layer on the host cores; a bounded
-    sample (a few layer-steps, cycling through the first layers), scaled to the stack."""
-    from oracle import ffn as O
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
-    n_layers_sample = min(2, wl.n_layers)
-    hl = [O.layer_weights_f64(S.make_layer(wl, l, device).to_numpy(), wl.act) for l in range(n_layers_sample)]
-    xs = S.make_inputs(wl.with_(x_dtype="f32"), 64 * batch, "cpu", stream_id=99).double().numpy()
+def _oracle_layers(wl, n, device):
+    from oracle import cpp as OC
+    return [OC.Layer(S.make_layer(wl, l, device).to_numpy(), wl.act) for l in range(n)]
+
+
+def _time_layer_steps(fn, budget_s, min_steps=2):
+    """Mean seconds of fn(k) over as many calls as fit the budget (at least min_steps)."""
     times, k = [], 0
     t_start = time.perf_counter()
     while True:
-        x = xs[(k % 64) * batch:(k % 64 + 1) * batch]
-        w = hl[k % n_layers_sample]
         t0 = time.perf_counter()
-        O.layer_step(x, w, wl.act, wl.x_dtype)
+        fn(k)
         times.append(time.perf_counter() - t0)
         k += 1
-        if time.perf_counter() - t_start > budget_s and k >= 2:
+        if time.perf_counter() - t_start > budget_s and k >= min_steps:
             break
-    per_layer = float(np.mean(times))
-    tok_s = batch / (per_layer * wl.n_layers)
-    sample = (f"{k} oracle layer-steps (batch {batch}) over layers 0..{n_layers_sample - 1} of {wl.name}, "
-              f"{per_layer * 1e3:.1f} ms each, scaled to {wl.n_layers} layers; fp64 numpy")
-    return tok_s, cores, sample
+    return float(np.mean(times)), k
+
+
+def oracle_tokens_per_s(wl, budget_s=15.0, batch=1, device="cuda"):
+    """Time the C++ oracle's decode of one token, layer by layer, on the host cores: a
+    bounded sample of layer-steps cycling through the first layers, scaled to the stack.
+    Three legs share the budget: the sparse oracle on every core (the reported value), the
+    sparse oracle on one core, and the dense FFN (every neuron, no predictor) on every core."""
+    from oracle import cpp as OC
+    OC.build()
+    n_layers_sample = min(2, wl.n_layers)
+    layers = _oracle_layers(wl, n_layers_sample, device)
+    xs = S.make_inputs(wl.with_(x_dtype="f32"), 64 * batch, "cpu", stream_id=99).double().numpy()
+    xb = lambda k: xs[(k % 64) * batch:(k % 64 + 1) * batch]
+    all_cores = OC.max_threads()
+    try:
+        OC.set_threads(all_cores)
+        sparse, k_sp = _time_layer_steps(lambda k: layers[k % n_layers_sample].layer_step(xb(k), wl.x_dtype),
+                                         0.45 * budget_s)
+        dense, k_de = _time_layer_steps(lambda k: layers[k % n_layers_sample].dense_ffn(xb(k)), 0.25 * budget_s, 1)
+        OC.set_threads(1)
+        single, k_1 = _time_layer_steps(lambda k: layers[k % n_layers_sample].layer_step(xb(k), wl.x_dtype),
+                                        0.3 * budget_s, 1)
+    finally:
+        OC.set_threads(all_cores)
+    L = wl.n_layers
+    out = {"value": batch / (sparse * L), "cores": all_cores,
+           "single_core_value": round(batch / (single * L), 6),
+           "dense_value": round(batch / (dense * L), 6),
+           "sample": (f"C++ oracle (fp64 loops), batch {batch}, layers 0..{n_layers_sample - 1} of {wl.name}, "
+                      f"scaled to {L} layers: sparse layer-step {sparse * 1e3:.1f} ms on {all_cores} cores "
+                      f"({k_sp} steps), {single * 1e3:.1f} ms on 1 core ({k_1} steps); dense FFN "
+                      f"{dense * 1e3:.1f} ms on {all_cores} cores ({k_de} steps)")}
+    return out
 
 
 # ------------------------------------------------------------------ our arm
 def build_stack(pi, wl, reorder=True):
     layers = []
-    desc = pi.make_desc(wl.d_model, wl.d_ff, wl.rank, wl.act, wl.w_dtype, wl.x_dtype, wl.p_dtype)
     for l in range(wl.n_layers):
+        wll = wl.at_layer(l)
+        desc = pi.make_desc(wll.d_model, wll.d_ff, wll.rank, wll.act, wll.w_dtype, wll.x_dtype, wll.p_dtype)
         L = S.make_layer(wl, l, "cuda")
         g = pi.load_layer(desc, L.tensors())
         if reorder:
@@ -237,7 +266,8 @@ def run_ours(args, world, rank, local):
     layers = build_stack(pi, wl, reorder=not args.no_reorder)
     torch.cuda.synchronize()
     t_gen = time.perf_counter() - t_gen
-    ws = pi.Workspace(wl.d_model, wl.d_ff, wl.rank, max(B, 1), wl.n_layers)
+    r_max = max(wl.at_layer(l).rank for l in range(wl.n_layers))
+    ws = pi.Workspace(wl.d_model, wl.d_ff, r_max, max(B, 1), wl.n_layers)
     K, W = args.steps, args.warmup
     xs = S.make_inputs(wl, (W + K + wl.prompt_len) * B, "cuda", stream_id=1000 + rank)
     xs = xs.view(W + K + wl.prompt_len, B, wl.d_model)
@@ -279,24 +309,25 @@ def run_ours(args, world, rank, local):
     ms_step = ms / K
     value = whole_job_rate(world, K, B, ms)
     active_per_step = (act1 - act0) / K                     # summed over layers
-    algo_bytes = wl.n_layers * predictor_bytes(wl) + active_per_step * bytes_per_neuron(wl)
+    pred_bytes = stack_predictor_bytes(wl)
+    algo_bytes = pred_bytes + active_per_step * bytes_per_neuron(wl)
     achieved = algo_bytes / (ms_local / K / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
     traffic = profiled_traffic(wl.name, wl.n_layers, B)
 
-    # end to end through the host-buffer entry point: H2D x, the stack, D2H x, sync
+    # end to end through the host-buffer entry point: H2D x, the stack, D2H x, sync.  The
+    # call returns only after the stream is synchronised, so a host clock brackets it.
     xo = torch.empty_like(xh[0]).pin_memory()
     for k in range(min(3, Ke)):
         pi.decode_stack_host(layers, xh[k], xo, B, ws)
     dist_barrier(world)
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
     with ClockSampler(local) as clk_e2e:
-        f0.record(stream)
+        h0 = time.perf_counter()
         for k in range(Ke):
             pi.decode_stack_host(layers, xh[k], xo, B, ws)
-        f1.record(stream)
-        torch.cuda.synchronize()
-    e2e_ms = dist_max(f0.elapsed_time(f1), world)
+        h1 = time.perf_counter()
+    e2e_ms = dist_max((h1 - h0) * 1e3, world)
     xbytes = B * wl.d_model * (4 if wl.x_dtype == "f32" else 2)
 
     out = {
@@ -309,6 +340,9 @@ def run_ours(args, world, rank, local):
                    "avg_active_per_layer": round(active_per_step / wl.n_layers, 1),
                    "us_per_layer": round(ms_step * 1e3 / wl.n_layers, 3),
                    "algorithmic_bytes_per_step": int(algo_bytes),
+                   "predictor_bytes_per_step": int(pred_bytes),
+                   "predictor_bytes_per_step_at_uniform_rank": int(wl.n_layers * predictor_bytes(wl)),
+                   "layer_ranks": sorted({wl.at_layer(l).rank for l in range(wl.n_layers)}),
                    "l2": f"no flush: per-step working set {algo_bytes / 1e9:.2f} GB > 126 MB L2",
                    "parallelism": f"replicas x{world}", "setup_s": round(t_gen, 1)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -318,59 +352,64 @@ def run_ours(args, world, rank, local):
                      "peak_source": peak_kind},
         "e2e": {"value": round(world * Ke * B / (e2e_ms / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": xbytes, "steps": Ke,
+                "timing": "host wall clock around the calls (each call synchronises)",
                 "clocks": clk_e2e.summary()},
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok_s, cores, sample = oracle_tokens_per_s(wl, budget_s=args.cpu_budget, batch=B)
-        out["cpu_baseline"] = {"value": round(tok_s, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                               "sample": sample}
+        cb = oracle_tokens_per_s(wl, budget_s=args.cpu_budget, batch=B)
+        out["cpu_baseline"] = {"value": round(cb["value"], 6), "unit": "tokens/s", "cores": cb["cores"],
+                               "kind": "oracle", "sample": cb["sample"],
+                               "single_core_value": cb["single_core_value"], "dense_value": cb["dense_value"]}
     if rank == 0:
         print(json.dumps(out), flush=True)
 
 
 # ------------------------------------------------------------------ reference arm
 def run_reference(args, world, rank):
+    """The oracle arm: the C++ oracle decodes K tokens through the whole stack on the host
+    cores (every layer: predictor, compaction, sparse FFN, glue), timed on the host clock.
+    K is capped so that the timed steps fit the CPU budget."""
     if rank != 0:
         return
     wl = WORKLOADS[args.workload]
+    if args.layers:
+        wl = wl.with_(n_layers=args.layers)
     B = args.batch
-    budget = args.cpu_budget
-    from oracle import ffn as O
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
+    from oracle import cpp as OC
+    OC.build()
+    cores = OC.max_threads()
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    hl = O.layer_weights_f64(S.make_layer(wl, 0, dev).to_numpy(), wl.act)
+    layers = _oracle_layers(wl, wl.n_layers, dev)
     xs = S.make_inputs(wl.with_(x_dtype="f32"), 64 * B, "cpu", stream_id=99).double().numpy()
-    # one step = the oracle's decode of one token through a sample of one layer, scaled to
-    # the stack; the number of timed steps is capped so the run stays within the budget
+    xb = lambda k: xs[(k % 64) * B:(k % 64 + 1) * B]
+
+    def step(k):
+        OC.decode_stack(xb(k), layers, wl.x_dtype)
+
     t0 = time.perf_counter()
-    O.layer_step(xs[:B], hl, wl.act, wl.x_dtype)
+    step(0)
     est = time.perf_counter() - t0
     W = min(args.warmup, 3)
-    K = max(1, min(args.steps, int(budget / max(est, 1e-6))))
-    for k in range(W):
-        O.layer_step(xs[(k % 64) * B:(k % 64 + 1) * B], hl, wl.act, wl.x_dtype)
+    K = max(1, min(args.steps, int(args.cpu_budget / max(est, 1e-6))))
+    for k in range(1, W):
+        step(k)
     t0 = time.perf_counter()
     for k in range(K):
-        O.layer_step(xs[(k % 64) * B:(k % 64 + 1) * B], hl, wl.act, wl.x_dtype)
+        step(W + k)
     el = time.perf_counter() - t0
-    per_layer = el / K
-    tok_s = B / (per_layer * wl.n_layers)
-    sample = (f"{K} oracle layer-steps of layer 0 of {wl.name} (batch {B}), {per_layer * 1e3:.1f} ms each, "
-              f"scaled to {wl.n_layers} layers; fp64 numpy on the host")
-    out = {"impl": "reference", "metric": METRIC, "value": round(tok_s, 4), "unit": "tokens/s", "n_gpus": world,
-           "steps": K, "warmup": W, "ms_per_step": round(per_layer * wl.n_layers * 1e3, 3),
+    tok_s = K * B / el
+    sample = (f"{K} decode steps of the C++ oracle through all {wl.n_layers} layers of {wl.name} "
+              f"(batch {B}) on {cores} cores, {el:.2f} s on the host clock")
+    out = {"impl": "reference", "metric": METRIC, "value": round(tok_s, 6), "unit": "tokens/s", "n_gpus": world,
+           "steps": K, "warmup": W, "ms_per_step": round(el / K * 1e3, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": wl.name, "layers": wl.n_layers, "d_model": wl.d_model, "d_ff": wl.d_ff,
                       "rank": wl.rank, "act": wl.act, "batch": B, "weights": wl.w_dtype},
-           "cpu_baseline": {"value": round(tok_s, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "cpu_baseline": {"value": round(tok_s, 6), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                             "sample": sample},
-           "e2e": {"value": round(tok_s, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+           "e2e": {"value": round(tok_s, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
 

@@ -14,8 +14,9 @@
  *     maps every placed neuron back to its original position (same page,
  *     §"Penempatan dan Pengelolaan Neuron"; KPD "PowerInfer: Fast Large Language Model
  *     Serving with a Consumer-grade GPU", §"Метод").
- *   - Activations: ReLU and ReGLU (GeekNews "Tüketici sınıfı GPU takılı PC'lerde yüksek hızlı büyük dil modeli serving",
- *     §"Kısıtlar ve SSS").
+ *   - Activations: ReLU, ReGLU and squared ReLU (GeekNews "Tüketici sınıfı GPU takılı
+ *     PC'lerde yüksek hızlı büyük dil modeli serving", §"Kısıtlar ve SSS": the method
+ *     serves the ReLU family, whose exact zeros can be skipped).
  *     Weights: fp32, fp16 or Q4_0 (same page, §"Kuantizasyon ve uyumluluk").
  *
  * Per layer and token x (d = d_model, f = d_ff, r = rank):
@@ -25,6 +26,7 @@
  *   idx     = ascending ids of the neurons whose bit is set for any token of the batch
  *   ReLU :  a_i = max(0, w_up_i . x + b_i)
  *   ReGLU:  a_i = max(0, w_gate_i . x + b_i) * (w_up_i . x)
+ *   ReLU^2: a_i = max(0, w_up_i . x + b_i)^2
  *   a[b,i] = 0 where token b's own bit is 0
  *   y_j     = sum over active i of W_down[j,i] * a_i          (fp32 accumulation)
  *   stack:  v = x + y;  x' = (v - mean(v)) / sqrt(var(v) + 1e-6), in fp32, stored in
@@ -78,14 +80,14 @@ typedef enum {
 } pi_status;
 
 typedef enum { PI_F32 = 0, PI_F16 = 1, PI_Q4_0 = 2 } pi_dtype;
-typedef enum { PI_RELU = 0, PI_REGLU = 1 } pi_act;
+typedef enum { PI_RELU = 0, PI_REGLU = 1, PI_RELU2 = 2 } pi_act;
 
 /* Shape and types of one FFN layer. */
 typedef struct {
   int d_model;       /* d */
   int d_ff;          /* f, a multiple of 32 */
   int rank;          /* r, predictor rank */
-  pi_act act;        /* PI_RELU: bias on up; PI_REGLU: bias on gate */
+  pi_act act;        /* PI_RELU, PI_RELU2 (squared ReLU): bias on up; PI_REGLU: bias on gate */
   pi_dtype w_dtype;  /* up/gate/down weights */
   pi_dtype x_dtype;  /* activations x (F32 or F16) */
   pi_dtype p_dtype;  /* predictor P1/P2 (F32 or F16) */
@@ -100,7 +102,7 @@ typedef struct {
  *            high four bits. s_up / s_gate / s_down are fp16 scale planes [f][d/32].
  *            The value is (q - 8) * scale. The down weights are given neuron-major
  *            ([f] rows of d), the axis the blocks run along.
- *   w_gate / s_gate are NULL for ReLU. s_* are NULL unless w_dtype is Q4_0.
+ *   w_gate / s_gate are NULL for ReLU and squared ReLU. s_* are NULL unless w_dtype is Q4_0.
  *   bias [f] f32, thresh [f] f32; p1 [d x r] and p2 [r x f] row-major in p_dtype. */
 typedef struct {
   const void* w_up;
@@ -140,7 +142,10 @@ typedef struct {
 /* ---------------------------------------------------------------- layers */
 
 /* Copy one layer into library-owned device memory, in the library's own layout.
- *   - One contiguous record per neuron: [gate row | up row | down row].
+ *   - One contiguous record per neuron: [gate row | up row | 16-byte bias header], so
+ *     one copy brings everything a neuron's gate/up dot products need.
+ *   - The down weights neuron-major, one row of d_model per neuron, so a block can read
+ *     its own column slice of each active neuron's row.
  *   - P1 is stored transposed and P2 neuron-major.
  * desc and w are host structs holding device pointers. Synchronises `stream` before it
  * returns. On success *out holds the layer. */
@@ -153,9 +158,10 @@ pi_status pi_load_layer(const pi_layer_desc* desc, const pi_layer_weights* w,
  * (pi_get_perm) is updated to match.
  *   freq:      device f32[d_ff], the measured firing frequency of each neuron in the
  *              layer's current stored order.
- *   hot_count: the length of the dense hot prefix used at batch >= 8. -1 means derive
- *              it per batch B: the neurons whose union firing probability
- *              1 - (1 - freq)^B is >= 1/2.
+ *   hot_count: -1, or the length of the hot prefix in [0, d_ff]. It is validated and
+ *              kept; the kernels do not read it (the hot order itself is what they use:
+ *              it places the always-firing neurons first, and its frequencies set how
+ *              many own records every block keeps before the mask exchange).
  * Synchronises `stream` before it returns. Calling it again composes the orders. */
 pi_status pi_reorder_hot_prefix(pi_layer* layer, const float* freq, int hot_count,
                                 cudaStream_t stream);
@@ -170,9 +176,10 @@ void pi_free_layer(pi_layer* layer);
 
 /* ---------------------------------------------------------------- workspace */
 
-/* Scratch for the kernels: the predictor vector u, per-block partial outputs, the
- * grid-barrier words, the device error word, and the stack's internal mask and index
- * buffers. It is sized for the largest shapes it will serve: calls with larger d_model,
+/* Scratch for the kernels: the cross-block exchange words (the predictor vector u,
+ * every block's mask words, h of the active neurons, the stack's x + y and its
+ * moments), the launch words, the device error word, and the multi-launch path's mask,
+ * index and partial-sum buffers. It is sized for the largest shapes it will serve: calls with larger d_model,
  * d_ff, rank, B or L return PI_ERR_ARG. A workspace serves one stream at a time. Calls
  * that overlap on the device and share a workspace race. */
 pi_status pi_workspace_create(int d_model_max, int d_ff_max, int rank_max, int B_max,
@@ -201,17 +208,16 @@ pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaSt
 
 /* Diagnostic: with `on`, every later pi_decode_stack on this workspace records each
  * block's SM cycle counter at up to 64 points of every layer. Consumer warps: 0 layer
- * start, 1 u rows published, 2 u received, 7 logits done, 15 own active list formed,
- * 3 list handed to the producer, 5 first record landed, 4 FFN partials published,
- * 6 slice reduce done, 16 moments read, 17 v read, 8 glue done. Producer warp: 9 waits
- * for the list, 10 list received, 11 all records issued; 12 and 13 mark the first
- * predictor item landing (P2, P1), 20 F loop done, 22-25 the balancing steps (list
- * published, thread 0's words read, every thread's words read, targets computed).
- * Slot 14 holds the block's record count, 18 the cycles spent waiting for P2 rows, 19
- * the cycles thread 0 waits for the h of records and 21 those warp 0 waits for records
- * to land. With `on` = 2
- * the stamps come from the GPU's global nanosecond timer instead, so blocks can be
- * compared with one another. With `on` = 0 recording stops and the buffer is freed. */
+ * start, 1 u rows published, 2 u received, 3 logits done, 4 own list and mask words
+ * published, 5 every block's mask words received, 6 assignment done (list handed to the
+ * producer), 7 down-row copies issued, 8 first record landed, 9 gate/up dots done,
+ * 10 down slice summed, 11 v and moments published, 12 every v and moment received,
+ * 13 glue done. Producer warp: 20 waits for the list, 21 list received, 22 all records
+ * issued. Slot 14 holds the block's record count, 15 the layer's active count, 17 the
+ * cycles thread 0 polls for h, 18 the cycles spent waiting for P2 rows and 19 those
+ * warp 0 waits for records to land. With `on` = 2 the stamps come from the GPU's global
+ * nanosecond timer instead, so blocks can be compared with one another. With `on` = 0
+ * recording stops and the buffer is freed. */
 pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on);
 
 /* Copy the first n stamps ([grid][L_max][64], int64) to host memory (synchronous). */
@@ -231,23 +237,32 @@ pi_status pi_predict(const pi_layer* layer, const void* x, int B, uint32_t* mask
 /* Bytes of the static device scratch behind pi_predict_noalloc (256 KiB). */
 #define PI_NOALLOC_SCRATCH_BYTES (256u * 1024u)
 
-/* pi_predict without a workspace: the same predictor launch, with the same outputs and
- * the same bits as pi_predict. It allocates no memory: its cross-block scratch is
- * one static device array of PI_NOALLOC_SCRATCH_BYTES per device. The pages have no
- * counterpart; this entry point is this library's own. It is for callers that cannot
- * allocate device memory when they call it, such as a serving loop that has already
- * handed all free HBM to its weights and KV cache, or a plug-in that sees only a
- * stream and plain pointers and has nowhere to keep a workspace between calls.
+/* pi_predict without a workspace: the predictor launch of pi_predict, with the same
+ * outputs and the same bits wherever both serve the shape. It allocates no memory: its
+ * cross-block scratch is one static device array of PI_NOALLOC_SCRATCH_BYTES per device.
+ * The pages have no counterpart; this entry point is this library's own. It is for
+ * callers that cannot allocate device memory when they call it, such as a serving loop
+ * that has already handed all free HBM to its weights and KV cache, or a plug-in that
+ * sees only a stream and plain pointers and has nowhere to keep a workspace between
+ * calls.
  *
+ * Shapes served: only those the single persistent launch serves, that is 1 to 4 tokens
+ *   (1 to 2 for Q4_0) with d_model up to 12288 (fp16, 1 token), 8192 (fp16 2 tokens,
+ *   Q4_0), 4096 (fp16 4 tokens, fp32 1-2 tokens) or 2048 (fp32 4 tokens). Other shapes,
+ *   which pi_predict runs on its multi-launch path, return PI_ERR_UNSUPPORTED before
+ *   anything is enqueued, the first call's set-up included.
  * status: device i32, owned by the caller (required). After the launch it receives
  *   PI_OK, PI_ERR_TIMEOUT (a bounded device-side wait gave up) or PI_ERR_DEVICE (a
  *   device-side check failed). After an error the scratch is reset on the device for
- *   the next call.
+ *   the next call. The word is written only when the call returns PI_OK; after any
+ *   other return it keeps what it held.
  * Scratch needed: 256 + round256(B * rank * 8) bytes. A shape that needs more than
  *   PI_NOALLOC_SCRATCH_BYTES returns PI_ERR_UNSUPPORTED and enqueues nothing.
  * Set-up: the first call on each device takes the array's address, clears it and
  *   synchronises `stream` before it returns. Make that first call before any stream
- *   capture begins.
+ *   capture begins. The set-up is kept for the life of the process: after
+ *   cudaDeviceReset (or anything else that destroys the device's primary context) this
+ *   entry point must not be called again on that device.
  * Calls share the one array per device. Two calls that may run at the same time (on
  *   different streams, or from different threads without ordering) race on it and
  *   give undefined results. Order them on one stream or with events. */
@@ -276,7 +291,11 @@ pi_status pi_sparse_ffn(const pi_layer* layer, const void* x, int B, const uint3
  * layer runs a fixed sequence of kernels: tensor-core row tiles for the predictor and
  * gate/up, compaction, the down columns and the glue. The host does not synchronise
  * inside either way. x_inout: device [B][d] in the activation dtype. It holds x_0 on
- * entry and x_L on return. All layers must share one descriptor. trace may be NULL. */
+ * entry and x_L on return. All layers must share one descriptor except for the
+ * predictor rank, which may differ from layer to layer (the pages size each layer's
+ * predictor by its own sparsity: unite.ai "PowerInfer: Mesin Inferensi LLM Cepat dengan
+ * GPU Konsumen", §"Prediktor Kepadatan Adaptif"); the workspace's rank_max must cover the
+ * largest. trace may be NULL. */
 pi_status pi_decode_stack(pi_layer* const* layers, int L, void* x_inout, int B,
                           const pi_trace* trace, pi_workspace* ws, cudaStream_t stream);
 

@@ -212,6 +212,7 @@ def _fit_sketch(w: Workload, layer: int, fire_rows32: torch.Tensor,
 
 
 def make_layer(w: Workload, layer: int, device="cpu") -> SynthLayer:
+    w = w.at_layer(layer)
     d, f = w.d_model, w.d_ff
     if f % 32 or d % 32:
         raise ValueError("d_model and d_ff must be multiples of 32")

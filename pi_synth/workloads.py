@@ -38,9 +38,21 @@ class Workload:
     steps: int = 1           # decode steps
     batches: Tuple[int, ...] = (1,)
     w_std_q4: float = 0.02   # std of the |N(0, s)| Q4_0 block scales
+    layer_mean_p: Optional[Tuple[float, ...]] = None   # per-layer mean firing probability (cycled)
+    layer_rank: Optional[Tuple[int, ...]] = None       # per-layer predictor rank (cycled)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
+
+    def at_layer(self, layer: int) -> "Workload":
+        """The workload as layer `layer` sees it: its own density and predictor rank when
+        the workload gives them per layer."""
+        kw = {}
+        if self.layer_mean_p:
+            kw.update(mean_p=self.layer_mean_p[layer % len(self.layer_mean_p)], c=None)
+        if self.layer_rank:
+            kw.update(rank=self.layer_rank[layer % len(self.layer_rank)])
+        return replace(self, **kw) if kw else self
 
 
 # Single ReLU layer, fp32, d_model 512, d_ff 2048, rank-64 least-squares predictor.
@@ -87,3 +99,32 @@ def scaled(base: Workload, name: str, n_layers: int, d_model: int, d_ff: int,
     """A smaller workload with the same law, dtypes and predictor fit as `base`."""
     return base.with_(name=name, n_layers=n_layers, d_model=d_model, d_ff=d_ff,
                       rank=rank, **kw)
+
+
+def adaptive_ranks(base_rank: int, layer_mean_p: Tuple[float, ...], d_model: int,
+                   floor: int = 64) -> Tuple[int, ...]:
+    """Per-layer predictor ranks from per-layer densities.  The pages size each layer's
+    predictor by the layer's own sparsity (a sparser layer gets a smaller predictor;
+    unite.ai "PowerInfer: Mesin Inferensi LLM Cepat dengan GPU Konsumen", §"Prediktor
+    Kepadatan Adaptif") but give no formula.  The reading here is the plainest one: the
+    densest layer keeps the base rank, and every other layer gets the base rank in
+    proportion to its mean firing probability, rounded to a multiple of 8 and kept within
+    [floor, d_model]."""
+    top = max(layer_mean_p)
+    out = []
+    for p in layer_mean_p:
+        r = int(round(base_rank * p / top / 8.0)) * 8
+        out.append(max(floor, min(d_model, r)))
+    return tuple(out)
+
+
+def _linear_profile(n: int, lo: float, hi: float) -> Tuple[float, ...]:
+    return tuple(hi + (lo - hi) * l / (n - 1) for l in range(n))
+
+
+# Llama-2-7B-shaped stack whose layers differ in density (a synthetic profile from 14 %
+# active in the first layer down to 6 % in the last, 10 % on average, the base workload's
+# mean), each with the adaptive predictor rank of its density.
+_ADAPTIVE_P = _linear_profile(32, 0.06, 0.14)
+LLAMA2_7B_ADAPTIVE = LLAMA2_7B.with_(name="llama2_7b_reglu_f16_adaptive_rank", layer_mean_p=_ADAPTIVE_P,
+                                     layer_rank=adaptive_ranks(512, _ADAPTIVE_P, 4096))

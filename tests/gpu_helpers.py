@@ -9,6 +9,9 @@ Parity rules (the pages' tolerances for this path):
     and Q4_0 (fp32 accumulation on the device, fp64 in the oracle).
 Every oracle input comes from the seeded generator or from the oracle itself; GPU
 results are only ever compared, never fed to the oracle.
+
+The oracle used here is the C++ one (oracle/pi_oracle.cpp through oracle/cpp.py): it
+reads the generator's stored tensors directly and accumulates in double.
 """
 from __future__ import annotations
 
@@ -18,6 +21,7 @@ import numpy as np
 import torch
 
 import pi_synth as S
+from oracle import cpp as OC
 from oracle import ffn as O
 
 BAND = 1e-3
@@ -37,23 +41,25 @@ def build_layers(pi, wl: S.Workload, n_layers: int | None = None, keep_host: boo
     gl, sl = [], []
     for l in range(n):
         L = S.make_layer(wl, l, "cuda")
-        gl.append(pi.load_layer(desc_of(pi, wl), L.tensors()))
+        gl.append(pi.load_layer(desc_of(pi, wl.at_layer(l)), L.tensors()))
         sl.append(L if keep_host else None)
     torch.cuda.synchronize()
     return gl, sl
 
 
-def host_layer(L: S.SynthLayer) -> Dict[str, np.ndarray]:
-    return O.layer_weights_f64(L.to_numpy(), L.workload.act)
+def cpp_layer(L: S.SynthLayer) -> OC.Layer:
+    """The whole layer, stored values, for the C++ oracle."""
+    return OC.Layer(L.to_numpy(), L.workload.act)
 
 
-def host_predictor(L: S.SynthLayer) -> Dict[str, np.ndarray]:
-    return {"p1": L.p1.cpu().double().numpy(), "p2": L.p2.cpu().double().numpy(),
-            "thresh": L.thresh.cpu().double().numpy()}
+def oracle_logits(L: S.SynthLayer, x: np.ndarray) -> np.ndarray:
+    """The C++ oracle's fp64 logits, from the layer's stored predictor only."""
+    t = {"p1": L.p1.cpu().numpy(), "p2": L.p2.cpu().numpy(), "thresh": L.thresh.cpu().numpy()}
+    return OC.Layer(t, L.workload.act).predictor_logits(x)
 
 
-def host_rows(L: S.SynthLayer, rows: np.ndarray) -> Dict[str, np.ndarray]:
-    """Oracle weights of the given neuron rows only (subset k = neuron rows[k])."""
+def stored_rows(L: S.SynthLayer, rows: np.ndarray) -> Dict[str, np.ndarray]:
+    """Stored tensors of the given neuron rows only (subset k = neuron rows[k])."""
     act = L.workload.act
     ri = torch.as_tensor(np.asarray(rows, np.int64), device=L.bias.device)
     t = {"bias": L.bias[ri], "p1": L.p1, "p2": L.p2[:, ri], "thresh": L.thresh[ri]}
@@ -62,18 +68,18 @@ def host_rows(L: S.SynthLayer, rows: np.ndarray) -> Dict[str, np.ndarray]:
         if act == "reglu":
             t.update(q_gate=L.q_gate[ri], s_gate=L.s_gate[ri])
     else:
-        t.update(w_up=L.w_up[ri], w_down=L.w_down[:, ri])
+        t.update(w_up=L.w_up[ri], w_down=L.w_down[:, ri].contiguous())
         if act == "reglu":
             t["w_gate"] = L.w_gate[ri]
-    return O.layer_weights_f64({k: v.cpu().numpy() for k, v in t.items()}, act)
+    return {k: v.cpu().numpy() for k, v in t.items()}
 
 
 def oracle_ffn_rows(x: np.ndarray, L: S.SynthLayer, bits: np.ndarray, idx: np.ndarray) -> np.ndarray:
-    """Oracle sparse FFN over `idx` (ascending), computed from those rows only."""
+    """The C++ oracle's sparse FFN over `idx` (ascending), computed from those rows only."""
     if len(idx) == 0:
         return np.zeros((np.atleast_2d(x).shape[0], L.workload.d_model))
-    sub = host_rows(L, idx)
-    return O.sparse_ffn(x, sub, L.workload.act, np.atleast_2d(bits)[:, idx], np.arange(len(idx)))
+    sub = OC.Layer(stored_rows(L, idx), L.workload.act)
+    return sub.sparse_ffn(x, np.atleast_2d(bits)[:, idx], np.arange(len(idx)))
 
 
 def mask_parity(logits_ref: np.ndarray, bits_gpu: np.ndarray):
@@ -98,3 +104,8 @@ def unpack_words(words: torch.Tensor, f: int) -> np.ndarray:
 
 def x_to_np(x: torch.Tensor) -> np.ndarray:
     return x.detach().cpu().double().numpy()
+
+
+def cpp_layer_as(L: S.SynthLayer, act: str) -> OC.Layer:
+    """The layer's stored tensors under another activation family (same weights)."""
+    return OC.Layer(L.to_numpy(), act)

@@ -39,8 +39,7 @@ def _predict_check(gl, L, wl, B, ws, stream_id):
     logits = torch.empty(B, wl.d_ff, device="cuda")
     pi.predict(gl, x, B, mask, logits, ws)
     assert ws.status() == 0
-    hp = H.host_predictor(L)
-    lref = O.predictor_logits(H.x_to_np(x), hp["p1"], hp["p2"], hp["thresh"])
+    lref = H.oracle_logits(L, H.x_to_np(x))
     lg = logits.cpu().double().numpy()
     scale = max(1.0, float(np.max(np.abs(lref))))
     assert np.max(np.abs(lg - lref)) <= 1e-4 * scale, np.max(np.abs(lg - lref))
@@ -66,8 +65,7 @@ def test_batched_ffn_parity(wl, B):
     ws = _ws(wl, B)
     x = S.make_inputs(wl, B, "cuda", stream_id=120 + B)
     xn = H.x_to_np(x)
-    hp = H.host_predictor(sl[0])
-    bits = O.fire_bits(O.predictor_logits(xn, hp["p1"], hp["p2"], hp["thresh"]))
+    bits = O.fire_bits(H.oracle_logits(sl[0], xn))
     words = O.pack_mask(bits)
     idx, cnt = O.compact(words, wl.d_ff)
     y_ref = H.oracle_ffn_rows(xn, sl[0], bits, idx)

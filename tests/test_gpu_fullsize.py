@@ -43,8 +43,7 @@ def test_fullsize_layer_parity(wl):
     logits = torch.empty(1, wl.d_ff, device="cuda")
     pi.predict(gl[0], x, 1, mask, logits, ws)
     assert ws.status() == 0
-    hp = H.host_predictor(L)
-    lref = O.predictor_logits(xn, hp["p1"], hp["p2"], hp["thresh"])
+    lref = H.oracle_logits(L, xn)
     bits = H.unpack_words(mask, wl.d_ff)
     bad, flips, band = H.mask_parity(lref, bits)
     assert bad == 0, (bad, flips, band)
@@ -105,8 +104,7 @@ def test_fullsize_stack(wl):
     # layer 0 against the oracle, from the generator's x0 (in original neuron order)
     L0 = sl[0]
     xn = H.x_to_np(x0)
-    hp = H.host_predictor(L0)
-    lref = O.predictor_logits(xn, hp["p1"], hp["p2"], hp["thresh"])          # original order
+    lref = H.oracle_logits(L0, xn)          # original order
     lg0 = tr["logits"][0].cpu().double().numpy()                             # stored order
     bits0 = H.unpack_words(tr["mask"][0], wl.d_ff)
     bad, flips, _ = H.mask_parity(lref[:, perm0], bits0)

@@ -7,6 +7,7 @@ import pytest
 import torch
 
 import pi_synth as S
+from oracle import cpp as OC
 from oracle import ffn as O
 import gpu_helpers as H
 
@@ -50,8 +51,7 @@ def test_predict_parity(wl, B):
     logits = torch.empty(B, wl.d_ff, device="cuda")
     pi.predict(gl[0], x, B, mask, logits, ws)
     assert ws.status() == 0
-    hp = H.host_predictor(sl[0])
-    lref = O.predictor_logits(H.x_to_np(x), hp["p1"], hp["p2"], hp["thresh"])
+    lref = H.oracle_logits(sl[0], H.x_to_np(x))
     lg = logits.cpu().double().numpy()
     scale = max(1.0, float(np.max(np.abs(lref))))
     assert np.max(np.abs(lg - lref)) <= 1e-4 * scale, np.max(np.abs(lg - lref))
@@ -92,8 +92,7 @@ def test_sparse_ffn_parity(wl, B):
     ws = _ws(wl)
     x = S.make_inputs(wl, B, "cuda", stream_id=10 + B)
     xn = H.x_to_np(x)
-    hp = H.host_predictor(sl[0])
-    bits = O.fire_bits(O.predictor_logits(xn, hp["p1"], hp["p2"], hp["thresh"]))
+    bits = O.fire_bits(H.oracle_logits(sl[0], xn))
     words = O.pack_mask(bits)
     idx, cnt = O.compact(words, wl.d_ff)
     y_ref = H.oracle_ffn_rows(xn, sl[0], bits, idx)
@@ -116,11 +115,11 @@ def test_sparse_equals_dense_on_gpu(wl):
     ws = _ws(wl)
     x = S.make_inputs(wl, 1, "cuda", stream_id=21)
     xn = H.x_to_np(x)
-    hw = H.host_layer(sl[0])
-    m = O.true_mask(xn, hw, wl.act)
+    cl = H.cpp_layer(sl[0])
+    m = cl.true_mask(xn)
     words = O.pack_mask(m)
     idx, cnt = O.compact(words, wl.d_ff)
-    y_dense = O.dense_ffn(xn, hw, wl.act)
+    y_dense = cl.dense_ffn(xn)
     y = torch.empty(1, wl.d_model, device="cuda")
     pi.sparse_ffn(gl[0], x, 1, torch.from_numpy(words.view(np.int32)).cuda(),
                   torch.from_numpy(idx).cuda(), torch.tensor([cnt], dtype=torch.int32, device="cuda"), y, ws)
@@ -162,11 +161,11 @@ def _stack_check(wl, B, n_layers, stream_id=0):
     trajectory.  When a mask bit flips inside the band (both results are correct), the
     GPU's segment from that layer on is re-run from the oracle's next input."""
     gl, sl = H.build_layers(pi, wl, n_layers)
-    hls = [H.host_layer(L) for L in sl]
+    cls = [H.cpp_layer(L) for L in sl]
     ws = _ws(wl, B=B, L=n_layers)
     xdt = torch.float32 if wl.x_dtype == "f32" else torch.float16
     x0 = S.make_inputs(wl, B, "cuda", stream_id=stream_id)
-    ref = O.decode_stack(H.x_to_np(x0), hls, wl.act, wl.x_dtype)
+    ref = OC.decode_stack(H.x_to_np(x0), cls, wl.x_dtype)
     total_flips, l0, x_start, resyncs = 0, 0, x0, 0
     tol = H.y_tol(wl.w_dtype)
     words = wl.d_ff // 32
@@ -205,7 +204,7 @@ def _stack_check(wl, B, n_layers, stream_id=0):
                 in_band = np.abs(r["logits"]) < H.BAND
                 alt = np.where(in_band, bits, r["logits"] > 0)
                 alt_idx, _ = O.compact(O.pack_mask(alt), wl.d_ff)
-                y_alt = O.sparse_ffn(r["x_in"], hls[l], wl.act, alt, alt_idx)
+                y_alt = cls[l].sparse_ffn(r["x_in"], alt, alt_idx)
                 assert H.rel_err(y, y_alt) <= tol
                 total_flips += flips
                 flipped_at = l
@@ -276,8 +275,7 @@ def test_reorder_hot_prefix(wl):
     mask = torch.empty(1, wl.d_ff // 32, dtype=torch.int32, device="cuda")
     logits = torch.empty(1, wl.d_ff, device="cuda")
     pi.predict(gl[0], x, 1, mask, logits, ws)
-    hp = H.host_predictor(L)
-    lref = O.predictor_logits(H.x_to_np(x), hp["p1"], hp["p2"], hp["thresh"])
+    lref = H.oracle_logits(L, H.x_to_np(x))
     lg = logits.cpu().double().numpy()
     assert np.max(np.abs(lg[:, :] - lref[:, perm])) <= 1e-4 * max(1.0, np.max(np.abs(lref)))
     bits = H.unpack_words(mask, wl.d_ff)
@@ -333,3 +331,48 @@ def test_argument_errors():
     small = pi.Workspace(256, 1024, 64, 1, 1)
     with pytest.raises(pi.PiError):
         pi.predict(gl[0], x, 1, mask, None, small)
+
+
+def test_allocation_failure_is_reported():
+    """A workspace larger than the device can hold returns PI_ERR_OOM from the allocation
+    (no fault, nothing left allocated), and the device goes on working."""
+    free0, _ = torch.cuda.mem_get_info()
+    with pytest.raises(pi.PiError) as e:
+        pi.Workspace(4096, 1 << 30, 512, pi.PI_MAX_BATCH, 1)   # h words alone: 2^30 x 32 x 8 bytes
+    assert e.value.status == 3                                # PI_ERR_OOM
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert abs(free1 - free0) < (64 << 20), (free0, free1)
+    wl = W_F16_REGLU
+    gl, _ = H.build_layers(pi, wl, 1, keep_host=False)
+    ws = _ws(wl)
+    x = S.make_inputs(wl, 1, "cuda")
+    pi.decode_stack(gl, x, 1, ws)
+    assert ws.status() == 0
+
+
+# ----------------------------------------------------------------- per-layer predictor rank
+W_MIXED_RANK = S.scaled(S.LLAMA2_7B, "reglu_f16_mixed_rank", 3, 1024, 4192, 192, layer_rank=(128, 64, 192))
+
+
+@pytest.mark.parametrize("B", [1, 2, 8])
+def test_decode_stack_mixed_rank(B):
+    """Layers of one stack with different predictor ranks (unite.ai "PowerInfer: Mesin
+    Inferensi LLM Cepat dengan GPU Konsumen", §"Prediktor Kepadatan Adaptif": each layer's
+    predictor is sized on its own) run in one call and match the oracle layer by layer."""
+    assert [W_MIXED_RANK.at_layer(l).rank for l in range(3)] == [128, 64, 192]
+    flips, resyncs = _stack_check(W_MIXED_RANK, B, 3, stream_id=600 + B)
+    print(f"mixed-rank stack B={B}: in-band flips {flips}, re-syncs {resyncs}")
+
+
+def test_decode_stack_rejects_other_shapes():
+    """Only the rank may differ between the layers of a stack."""
+    a = S.scaled(S.LLAMA2_7B, "reglu_f16_d1024_a", 1, 1024, 4192, 128)
+    b = S.scaled(S.LLAMA2_7B, "reglu_f16_d1024_b", 1, 1024, 4096, 128)
+    ga, _ = H.build_layers(pi, a, 1, keep_host=False)
+    gb, _ = H.build_layers(pi, b, 1, keep_host=False)
+    ws = _ws(a, B=1, L=2)
+    x = S.make_inputs(a, 1, "cuda")
+    with pytest.raises(pi.PiError) as e:
+        pi.decode_stack([ga[0], gb[0]], x, 1, ws)
+    assert e.value.status == 1
