@@ -83,12 +83,12 @@ void free_layer_buffers(pi_layer* L) {
 // Bytes of bulk copies each block of the fused kernel keeps in flight: enough to keep its
 // share of HBM busy (about the SM's share of bandwidth times the unloaded latency), and no
 // more, since every byte beyond that only lengthens the queue the exchange words wait in.
-// PI_FUSED_INFLIGHT_KB in the environment (read once) overrides the default of 64 KB.
+// PI_FUSED_INFLIGHT_KB in the environment (read once) overrides the default of 128 KB.
 int inflight_budget_bytes() {
   static const int v = [] {
     const char* e = std::getenv("PI_FUSED_INFLIGHT_KB");
     const int kb = e ? std::atoi(e) : 0;
-    return (kb > 0 && kb <= 4096 ? kb : 64) * 1024;
+    return (kb > 0 && kb <= 4096 ? kb : 128) * 1024;
   }();
   return v;
 }
@@ -112,13 +112,13 @@ pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedPara
   if (!fused_supported(L->family, B, d.d_model)) return PI_ERR_UNSUPPORTED;
   if (!fused_plan_smem(p, L->family, (size_t)smem_optin(ws->device), smem)) return PI_ERR_UNSUPPORTED;
   // ws fields
-  p.ux = ws->ux; p.mx = ws->mx; p.hx = ws->hx; p.vx = ws->vx; p.sx = ws->sx;
+  p.ux = ws->ux; p.mx = ws->mx; p.hx = ws->hx; p.vx = ws->vx;
   p.bar = ws->bar; p.err = ws->err; p.active_total = ws->active_total;
   p.layer_count = nullptr;
   p.barrier_timeout_ns = kDefaultWaitNs;
   p.wait_cycles = kDefaultWaitNs * 3;   // cycles at up to 3 GHz: at least the nominal budget
   p.barrier_extra = 0;
-  p.poll_ns = 64;          // back-off between exchange polling rounds
+  p.poll_ns = 256;         // back-off between exchange polling rounds (a round costs ~1 us anyway)
   p.inflight_budget = inflight_budget_bytes();
   return PI_OK;
 }
@@ -408,12 +408,11 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
   if (ws->grid <= 0) { delete ws; return PI_ERR_CUDA; }
   if (ws->grid > kMaxGrid) { delete ws; return PI_ERR_UNSUPPORTED; }
   const size_t G = ws->grid, Bm = B_max;
-  const size_t mx_bytes = G * 4 * kMaxOwnWords * 8, hx_bytes = (size_t)f_max * Bm * 8;
+  const size_t mx_bytes = G * 4 * kMaxOwnWords * 8, hx_bytes = ((size_t)f_max + G) * Bm * 8;
   bool ok = dmalloc(&ws->ux, Bm * r_max * 8) == cudaSuccess &&
             dmalloc(&ws->mx, mx_bytes) == cudaSuccess &&
             dmalloc(&ws->hx, hx_bytes) == cudaSuccess &&
-            dmalloc(&ws->vx, Bm * d_max * 8) == cudaSuccess &&
-            dmalloc(&ws->sx, Bm * G * 16) == cudaSuccess &&
+            dmalloc(&ws->vx, (Bm * d_max + 2 * Bm * G) * 8) == cudaSuccess &&
             dmalloc(&ws->bar, 64) == cudaSuccess &&
             dmalloc(&ws->err, 16) == cudaSuccess &&
             dmalloc(&ws->active_total, 16) == cudaSuccess &&
@@ -433,7 +432,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
     const uint32_t bar0[4] = {0u, 0u, 1u, 0u};
     ok = cudaMemset(ws->ux, 0, Bm * r_max * 8) == cudaSuccess && cudaMemset(ws->mx, 0, mx_bytes) == cudaSuccess &&
          cudaMemset(ws->hx, 0, hx_bytes) == cudaSuccess &&
-         cudaMemset(ws->vx, 0, Bm * d_max * 8) == cudaSuccess && cudaMemset(ws->sx, 0, Bm * G * 16) == cudaSuccess &&
+         cudaMemset(ws->vx, 0, (Bm * d_max + 2 * Bm * G) * 8) == cudaSuccess &&
          cudaMemset(ws->bar, 0, 64) == cudaSuccess &&
          cudaMemcpy(ws->bar, bar0, sizeof(bar0), cudaMemcpyHostToDevice) == cudaSuccess &&
          cudaMemset(ws->err, 0, 16) == cudaSuccess && cudaMemset(ws->active_total, 0, 16) == cudaSuccess &&
@@ -450,7 +449,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
 
 void pi_workspace_free(pi_workspace* ws) {
   if (!ws) return;
-  cudaFree(ws->ux); cudaFree(ws->mx); cudaFree(ws->hx); cudaFree(ws->vx); cudaFree(ws->sx);
+  cudaFree(ws->ux); cudaFree(ws->mx); cudaFree(ws->hx); cudaFree(ws->vx);
   cudaFree(ws->bar); cudaFree(ws->err); cudaFree(ws->active_total);
   cudaFree(ws->layer_count); cudaFree(ws->x_dev); cudaFree(ws->phase_clk);
   cudaFree(ws->u_hi); cudaFree(ws->u_lo); cudaFree(ws->bmask); cudaFree(ws->bidx); cudaFree(ws->bcount);

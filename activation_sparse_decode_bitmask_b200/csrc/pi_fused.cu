@@ -1,35 +1,39 @@
 // The fused persistent kernel of the activation-sparse FFN decode path.
 //
 // One block per SM: 16 consumer warps and 1 producer warp.  The producer streams the
-// block's predictor rows and the [gate | up | bias] record of every active neuron the
-// block dots from HBM into a byte ring in shared memory, as bulk copies completing on
-// mbarriers.  It runs ahead of the consumers as far as the ring allows, so the next
-// layer's predictor is in flight while the consumers finish the current one.
+// block's predictor rows and the [gate | up | bias] record of every neuron the block dots
+// from HBM into a byte ring in shared memory, as bulk copies completing on mbarriers.
+// A layer's predictor rows wait until the previous layer's records are dotted, so the
+// records have HBM to themselves and the predictor copies fill the exchanges after them.
 //
 // Per layer, for block c of G (stack mode):
 //   P-a   u_k = P1^T[k] . x for the block's rank rows k -> u exchange
 //   P-b   logit_i = P2^T[i] . u - t_i for the block's own neurons i = c, c+G, c+2G, ...;
-//         bit = logit > 0.  The block lists its own active neurons and hands the first
-//         of them (a floor set from the firing frequencies) to the producer at once.
-//   mask  every block publishes its own bit words; one polling round gives every block
-//         every bit.  From the union counts each block derives the same balanced
-//         assignment: it keeps up to T of its own active neurons and takes the excess of
-//         the blocks above T, so every block dots at most T = max(ceil(N/G), floor).
-//   F     gate/up dot products of the assigned records (a group of warps per record):
+//         bit = logit > 0.  The block lists its own active neurons, publishes its bit
+//         words and hands the first na of the list (a floor set from the firing
+//         frequencies) to the producer at once.
+//   F     warps 0..11 dot records as they land (a group of warps per record):
 //           ReLU : h = max(0, w_up_i . x + b_i)    ReGLU: max(0, w_gate_i . x + b_i) * (w_up_i . x)
 //           squared ReLU: h = max(0, w_up_i . x + b_i)^2
 //           h[b] = 0 where token b's bit is 0
-//         -> h exchange (one tagged word per neuron and token)
-//   down  block c owns a slice of the d output columns.  While F runs, its threads copy
-//         their slice of every active neuron's down row into shared memory (cp.async);
-//         then y[slice] = sum over the active neurons of h_i * W_down[i][slice], in a fixed
+//         -> h exchange: owner o's k-th active neuron publishes h at word o * nown_max + k
+//   help  meanwhile warps 12..15 poll every block's bit words, count them, and derive the
+//         same balanced assignment in every block: target T = ceil(N / G); a block dots
+//         at most max(T, na) of its own records and takes the excess of the blocks above
+//         T in block order.  They list the rest of the block's records for the producer
+//         and the F warps, build the layer's down list (all N active neurons in owner-major
+//         order with their h words) and copy the block's slice of every listed down row
+//         into shared memory (cp.async, completing on an mbarrier).
+//   down  block c owns a slice of the d output columns: once the h words are in,
+//         y[slice] = sum over the active neurons of h_i * W_down[i][slice], in a fixed
 //         order, and v = x + y with the slice's sum and sum of squares -> v exchange
 //   glue  x' = (v - mean(v)) / sqrt(var(v) + 1e-6) from every slice's v and moments,
 //         rounded to the activation dtype
 // The down projection is column-owned: a block reads only its slice of each active down
 // row, so nothing like a d-long partial sum per block is ever exchanged; the exchanges
 // carry r values (u), f/32 bit words (mask), one value per active neuron (h) and d
-// values (v) per token.
+// values (v) per token.  An own record that its owner dots although a taker dots it too
+// publishes the same value twice (both blocks hold the same x and sum in the same order).
 // Mask words (predict output, trace) are OR-ed in by the owner blocks of their bits.
 // Cross-block exchanges use 64-bit words {tag, value}: a reader polls the words
 // themselves until every tag matches, so data and completion arrive together and no grid
@@ -51,37 +55,42 @@ namespace {
 constexpr float kNormEps = 1e-6f;
 constexpr int kRedBar = 1;          // named barrier id among consumers
 constexpr int kItems = 32;          // ring items in flight (mbarrier pairs)
-constexpr uint32_t kSleepNs = 20000;  // suspend hint of blocking mbarrier waits (wakes on completion)
 constexpr int kHr = 48;             // F h slots: more than kItems, so a slot is free before its reuse
+constexpr uint32_t kSleepNs = 20000;  // suspend hint of blocking mbarrier waits (wakes on completion)
 constexpr int kMaxDch = 1024;       // entries per down chunk
+constexpr int kFWarps = 12;         // consumer warps that dot records; the others help
+constexpr int kHelperThreads = (kConsumerWarps - kFWarps) * 32;
+constexpr int kAssignBar = 2;       // F warps + helpers: the taken records are listed
+constexpr int kHelpBar = 3;         // helpers only
 
 enum Exchange : int { EX_U = 0, EX_M = 1, EX_H = 2, EX_V = 3 };
 
 struct Smem {
   uint64_t full[kItems];
   uint64_t empty[kItems];
-  uint64_t list_ready;          // the kept part of the block's list is in place
-  uint64_t list2_ready;         // the whole list is in place
   int abort_flag;
-  int nlist_a;                  // records of the kept part of the list
-  int nlist;
   int count;                    // own active neurons of the layer (union over tokens)
-  uint32_t item_pos[kItems];    // producer bookkeeping of items in flight
+  uint64_t item_at[kItems];     // producer bookkeeping: unwrapped ring offset of items in flight
   uint32_t item_size[kItems];
-  float gmean[4];               // glue: mean and standard deviation of v per token
+  float gmean[4];               // glue: mean and 1 / standard deviation of v per token
   float gsd[4];
   float red[2][kConsumerWarps][16];   // block reductions: warp partials (double-buffered)
   int hcnt[kHr];                // F: warps of the record's group that posted partials
-  float hpart[kHr][16];         // [warp of the record's group][token][gate/up]
-  int32_t list[kMaxList];       // the neurons this block dots, kept ones first
-  int32_t list_ent[kMaxList];   // their positions in the layer's entry order (h word index)
+  float hpart[kHr][16];         // F: [warp of the record's group][token][gate/up]
+  int32_t list[kMaxList];       // the neurons this block dots: its own active ones, then taken ones
+  int32_t list_hid[kMaxList];   // h word of each taken entry
   uint8_t list_bits[kMaxList];
   uint8_t own_bits[kMaxOwn];
-  int32_t cnt[kMaxGrid];        // union active count of every block's own neurons
   int32_t pre[kMaxGrid + 1];    // exclusive prefix of cnt: entries in owner-major order
-  int32_t xpre[kMaxGrid + 1];   // exclusive prefix of the blocks' excess over the target
-  int32_t bal[4];               // target, this block's deficit start, total excess
-  int32_t wsum[3][kConsumerWarps];   // per-warp partials of block scans
+  int32_t xpre[kMaxGrid + 1];   // exclusive prefix of the owners' excess over the target
+  int32_t wsum[2][kConsumerWarps];   // block scans: the warps' totals
+  uint64_t list_ready;          // the first na records of the list are in place
+  uint64_t list2_ready;         // all nrec records of the list are in place
+  int na;                       // records handed to the producer before the mask exchange
+  int own_cnt;                  // own records this block dots (list entries [0, own_cnt))
+  int nrec;                     // records this block dots: own_cnt own ones, then taken ones
+  uint64_t dfull[2];            // down chunk copies of each half landed
+  uint64_t fdone;               // the layer's neuron records are dotted (the producer's gate)
 };
 
 // Diagnostics: SM cycle (or global ns) stamps at phase boundaries, [block][layer][slot].
@@ -93,13 +102,15 @@ __device__ __forceinline__ void stamp(const FusedParams& p, int l, int ph) {
   if (p.phase_clk && threadIdx.x == 0)
     p.phase_clk[((size_t)blockIdx.x * p.L + l) * kPhases + ph] = stamp_now(p);
 }
+// the same stamp from the first helper thread
+__device__ __forceinline__ void hstamp(const FusedParams& p, int l, int ph) {
+  if (p.phase_clk && threadIdx.x == kFWarps * 32)
+    p.phase_clk[((size_t)blockIdx.x * p.L + l) * kPhases + ph] = stamp_now(p);
+}
 __device__ __forceinline__ void stamp_val(const FusedParams& p, int l, int ph, long long v) {
   if (p.phase_clk && threadIdx.x == 0) p.phase_clk[((size_t)blockIdx.x * p.L + l) * kPhases + ph] = v;
 }
 __device__ __forceinline__ long long diag_clock(const FusedParams& p) { return p.phase_clk ? clock64() : 0; }
-__device__ __forceinline__ void pstamp(const FusedParams& p, int l, int ph) {
-  if (p.phase_clk) p.phase_clk[((size_t)blockIdx.x * p.L + l) * kPhases + ph] = stamp_now(p);
-}
 
 // Bounded waits count SM cycles (clock64 is cheap to read; the global timer is not):
 // `limit` is the wait budget converted to cycles at an upper bound of the SM clock.
@@ -126,11 +137,7 @@ __device__ __forceinline__ uint64_t ld_tag(const uint64_t* p) {
   asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
   return w;
 }
-__device__ __forceinline__ void ld_tag2(const uint64_t* p, uint64_t& a, uint64_t& b) {
-  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
-}
 __device__ __forceinline__ bool tag_ok(uint64_t w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
-__device__ __forceinline__ float tag_val(uint64_t w) { return __uint_as_float((uint32_t)w); }
 
 __device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
   uint32_t v;
@@ -197,6 +204,53 @@ __device__ __forceinline__ void poll_words(const uint64_t* base, int first, int 
     }
     if (p.poll_ns) __nanosleep(p.poll_ns);   // back off: many blocks poll the same lines
   }
+}
+
+// Poll the n tagged words src + at(q), q in [0, n), with the npw consumer warps from
+// thread tbase on only (the other warps go on to the caller's named barrier and issue
+// nothing meanwhile): MQ
+// words per lane and round, all loads of a round issued before any tag is checked.  The
+// 32-bit payload of word q goes to dst[q].
+template <int MQ, typename At>
+__device__ __forceinline__ void poll_words(const uint64_t* src, At at, int n, int npw, uint32_t tag, uint32_t* dst,
+                                           Smem& sm, const FusedParams& p, int tbase = 0) {
+  const int t = (int)threadIdx.x - tbase;
+  if (t < 0) return;
+  if (t >= npw * 32) return;
+  const int nthr = npw * 32;
+  for (int b0 = 0; b0 < n; b0 += MQ * nthr) {
+    uint64_t w[MQ];
+    uint32_t need = 0;
+#pragma unroll
+    for (int i = 0; i < MQ; ++i) {
+      w[i] = 0;
+      if (b0 + t + i * nthr < n) need |= 1u << i;
+    }
+    bool started = false;
+    uint64_t t0 = 0;
+    while (need) {
+#pragma unroll
+      for (int i = 0; i < MQ; ++i)
+        if (need >> i & 1u) w[i] = ld_tag(src + at(b0 + t + i * nthr));
+#pragma unroll
+      for (int i = 0; i < MQ; ++i)
+        if ((need >> i & 1u) && tag_ok(w[i], tag)) need &= ~(1u << i);
+      if (!need || aborted(sm)) break;
+      if (!started) { t0 = wait_start(); started = true; }
+      else if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
+      if (p.poll_ns) __nanosleep(p.poll_ns);
+    }
+#pragma unroll
+    for (int i = 0; i < MQ; ++i)
+      if (b0 + t + i * nthr < n) dst[b0 + t + i * nthr] = (uint32_t)w[i];
+  }
+}
+
+// The same over the consecutive words src[0..n).
+template <int MQ>
+__device__ __forceinline__ void poll_linear(const uint64_t* src, int n, int npw, uint32_t tag, uint32_t* dst, Smem& sm,
+                                         const FusedParams& p) {
+  poll_words<MQ>(src, [](int q) { return (size_t)q; }, n, npw, tag, dst, sm, p);
 }
 
 // ------------------------------------------------------------------ ring (shared by both sides)
@@ -275,11 +329,10 @@ __device__ __forceinline__ uint32_t tag_of(uint32_t epoch, int l, int e) {
 __host__ __device__ constexpr int pow2_ceil(int v) { return v <= 1 ? 1 : 2 * pow2_ceil((v + 1) / 2); }
 __host__ __device__ constexpr int log2_exact(int v) { return v <= 1 ? 0 : 1 + log2_exact(v / 2); }
 
-// Warps that share the gate/up dots of one F record: 4 (8 for Q4_0, whose units cost
-// more arithmetic), fewer where the partials of the group would not fit a 16-float slot.
-__host__ __device__ constexpr int f_group_warps(int fam, int act, int nb) {
-  return (fam == FAM_Q4 ? 8 : 4) * nb * (act == PI_REGLU ? 2 : 1) <= 16 ? (fam == FAM_Q4 ? 8 : 4)
-                                                                        : 16 / (nb * (act == PI_REGLU ? 2 : 1));
+// Warps that share the gate/up dots of one F record: 4, or 2 where the partials of a
+// group of 4 would not fit a 16-float slot; either divides the kFWarps F warps.
+__host__ __device__ constexpr int f_group_warps(int act, int nb) {
+  return 4 * nb * (act == PI_REGLU ? 2 : 1) <= 16 ? 4 : 2;
 }
 
 // Elements of one 16-byte down unit: 4 fp32, 8 fp16, or the 32 weights of a Q4_0 block.
@@ -299,52 +352,17 @@ __device__ __forceinline__ int select_bit(uint32_t u, int k) {
   return pos;
 }
 
-// Exclusive prefix sums over the consumer threads of K values per thread (thread order),
-// with the totals.  Integer sums: the result is exact.
-template <int K>
-__device__ __forceinline__ void block_excl_scan(const int (&v)[K], int (&excl)[K], int (&tot)[K], Smem& sm, int warp,
-                                                int lane) {
-  int incl[K];
-#pragma unroll
-  for (int k = 0; k < K; ++k) {
-    incl[k] = v[k];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int x = __shfl_up_sync(0xffffffffu, incl[k], o);
-      if (lane >= o) incl[k] += x;
-    }
-    if (lane == 31) sm.wsum[k][warp] = incl[k];
-  }
-  named_bar_sync(kRedBar, kConsumerThreads);
-#pragma unroll
-  for (int k = 0; k < K; ++k) {
-    int off = 0, total = 0;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      const int s = sm.wsum[k][w];
-      if (w < warp) off += s;
-      total += s;
-    }
-    excl[k] = off + incl[k] - v[k];
-    tot[k] = total;
-  }
-  named_bar_sync(kRedBar, kConsumerThreads);   // sm.wsum is free again
-}
-
-// Union over the tokens of block o's own bit word w (ob: [G][NB][nw]).
-template <int NB>
-__device__ __forceinline__ uint32_t union_word(const uint32_t* ob, int o, int w, int nw) {
+// Union over the B tokens of block o's own bit word w (ob: [G][B][nw]).
+__device__ __forceinline__ uint32_t union_word(const uint32_t* ob, int o, int w, int nw, int B) {
   uint32_t u = 0;
-#pragma unroll
-  for (int b = 0; b < NB; ++b) u |= ob[((size_t)o * NB + b) * nw + w];
+  for (int b = 0; b < B; ++b) u |= ob[((size_t)o * B + b) * nw + w];
   return u;
 }
 
 // Own index m of the k-th active neuron of block o, from the union of its bit words.
-template <int NB>
-__device__ __forceinline__ int owner_select(const uint32_t* ob, int o, int k, int nw) {
+__device__ __forceinline__ int owner_select(const uint32_t* ob, int o, int k, int nw, int B) {
   for (int w = 0; w < nw; ++w) {
-    const uint32_t u = union_word<NB>(ob, o, w, nw);
+    const uint32_t u = union_word(ob, o, w, nw, B);
     const int n = __popc(u);
     if (k < n) return 32 * w + select_bit(u, k);
     k -= n;
@@ -352,18 +370,16 @@ __device__ __forceinline__ int owner_select(const uint32_t* ob, int o, int k, in
   return -1;   // unreachable with consistent counts
 }
 
-template <int NB>
-__device__ __forceinline__ uint32_t owner_token_bits(const uint32_t* ob, int o, int m, int nw) {
+__device__ __forceinline__ uint32_t owner_token_bits(const uint32_t* ob, int o, int m, int nw, int B) {
   uint32_t bits = 0;
-#pragma unroll
-  for (int b = 0; b < NB; ++b) bits |= ((ob[((size_t)o * NB + b) * nw + (m >> 5)] >> (m & 31)) & 1u) << b;
+  for (int b = 0; b < B; ++b) bits |= ((ob[((size_t)o * B + b) * nw + (m >> 5)] >> (m & 31)) & 1u) << b;
   return bits;
 }
 
 // ------------------------------------------------------------------ gate/up dots
-// This lane's partial gate/up dot products of one F record (at shared address rec) with
-// every token's x (xs: [NB][d] at shared address xs) over the units q0, q0 + qs, ... in
-// ascending order.
+// This lane's partial gate/up dot products of one neuron record (at shared address rec)
+// with every token's x (xs: [NB][d] at shared address xs) over the units q0, q0 + qs, ...
+// in ascending order.
 template <int FAM, int ACT, int NB>
 __device__ __forceinline__ void record_dot(uint32_t rec, uint32_t xs, const FusedParams& p, int nunits, int q0,
                                            int qs, float (&au)[NB], float (&ag)[NB]) {
@@ -425,7 +441,7 @@ __device__ __forceinline__ void down_unit_fma(uint32_t a, float sc, const float 
 
 // ------------------------------------------------------------------ the kernel
 template <int FAM, int ACT, int NB, int NU>
-__global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p) {
+__global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constant__ FusedParams p) {
   constexpr int UE = Fam<FAM>::UE;
   constexpr int XW = Fam<FAM>::XW;
   constexpr int PB = Fam<FAM>::PB;
@@ -436,26 +452,36 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
   uint8_t* ring_base = dsmem + p.off_ring;
   XT* xs = reinterpret_cast<XT*>(dsmem + p.off_xs);                  // [NB][d] current input
   float* u_s = reinterpret_cast<float*>(dsmem + p.off_us);           // [NB][r]
-  uint32_t* ob = reinterpret_cast<uint32_t*>(dsmem + p.off_ob);      // [G][NB][nw] every block's own bits
+  uint32_t* ob = reinterpret_cast<uint32_t*>(dsmem + p.off_ob);      // [G][B][nw] every block's own bits
   int32_t* dlist = reinterpret_cast<int32_t*>(dsmem + p.off_dlist);  // [2][dch] neuron of each chunk entry
+  int32_t* dhid = dlist + 2 * p.dch;                                  // [2][dch] its h word (per token)
   float* dred = reinterpret_cast<float*>(dsmem + p.off_dred);        // down reduction / v slice / moments
   const uint32_t dbuf_u = smem_u32(dsmem + p.off_dbuf);              // [2][dch][pmax] 16-byte down units
   const uint32_t dsc_u = smem_u32(dsmem + p.off_dsc);                // Q4_0: [2][dch][pmax] scale words
+  float* hs = reinterpret_cast<float*>(dsmem + p.off_hs);            // [2 * dch][B] h of the resident entries
 
   const int c = blockIdx.x, G = gridDim.x;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const bool do_pred = p.mode & MODE_PREDICT, do_ffn = p.mode & MODE_FFN, do_glue = p.mode & MODE_GLUE;
   const int d = p.d, f = p.f, B = p.B;
   const int nown = (c < f) ? (f - c + G - 1) / G : 0;
+  // blocks o < own_rem own nown_max neurons, the others nown_max - 1
+  const int nown_max = p.nown_max;
+  const int own_rem = f - (nown_max - 1) * G;
   const int nunits = d / UE;
   const int words = f / 32;
   const int nw = p.nw;
+  // helpers: this thread's run of the G * nw mask words
+  const int wpt = (G * nw + kHelperThreads - 1) / kHelperThreads;
+  const int wj0 = min(G * nw, max(0, (int)threadIdx.x - kFWarps * 32) * wpt);
+  const int wj1 = min(G * nw, wj0 + wpt);
   const int dch = p.dch, pmax = p.pmax;
   // the block's down slice: 16-byte units [cu0, cu1) of every down row.  In the down
   // phase lpe consecutive lanes take one entry (lane % lpe is the unit, so the lanes of an
   // entry read one contiguous piece of its row) and a warp takes epw entries per pass:
   // this lane handles unit dw of the entries de0, de0 + dstep, ... of every chunk
-  const int cu0 = (int)((long long)c * p.dunits / G), cu1 = (int)((long long)(c + 1) * p.dunits / G);
+  const int cu0 = (int)((unsigned)c * (unsigned)p.dunits / (unsigned)G);
+  const int cu1 = (int)((unsigned)(c + 1) * (unsigned)p.dunits / (unsigned)G);
   const int npc = cu1 - cu0;
   const int lpe = npc <= 1 ? 1 : npc <= 2 ? 2 : npc <= 4 ? 4 : npc <= 8 ? 8 : 16;
   const int epw = 32 / lpe;
@@ -470,11 +496,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], kConsumerWarps);
     }
+    for (int s = 0; s < kHr; ++s) sm.hcnt[s] = 0;
+    mbar_init(&sm.fdone, 1);
     mbar_init(&sm.list_ready, 1);
     mbar_init(&sm.list2_ready, 1);
-    for (int s = 0; s < kHr; ++s) sm.hcnt[s] = 0;
+    mbar_init(&sm.dfull[0], kHelperThreads);
+    mbar_init(&sm.dfull[1], kHelperThreads);
     sm.abort_flag = 0;
-    sm.nlist = 0;
     mbar_fence_init();
   }
   __syncthreads();
@@ -484,19 +512,26 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
     if (lane == 0) {
       uint32_t head = 0, issued = 0, oldest = 0;
       uint32_t landed = 0, inflight = 0;   // items known to have landed; bytes issued beyond them
-      // Reserve ring space for the next item: wait (in order) for the release of every
-      // older item that overlaps it, and of the item that last used its barrier pair.
+      // Reserve ring space for the next item.  Items sit in the ring in issue order, none
+      // across its end; with offsets counted without wrapping (one more lap at each wrap),
+      // an older item can share bytes with the new one only if the new one ends more than
+      // one ring length past the older one's start.  Such items are the oldest ones still
+      // held, so the producer waits for releases in order until the oldest held item is
+      // clear (and no more than kItems - 1 are held).
+      uint32_t lap = 0;
+      uint64_t at_new = 0;
       auto reserve = [&](uint32_t size, uint32_t& pos) -> bool {
-        pos = ring_place(head, size, p.ring_bytes);
+        pos = head;
+        if (pos + size > (uint32_t)p.ring_bytes) {
+          pos = 0;
+          ++lap;
+        }
+        head = pos + size;
+        at_new = (uint64_t)lap * (uint32_t)p.ring_bytes + pos;
         while (oldest < issued) {
-          bool must = issued - oldest >= (uint32_t)kItems;
-          if (!must) {
-            for (uint32_t j = oldest; j < issued; ++j) {
-              const uint32_t a = sm.item_pos[j % kItems], e = a + sm.item_size[j % kItems];
-              if (pos < e && a < pos + size) { must = true; break; }
-            }
-          }
-          if (!must) break;
+          if (issued - oldest < (uint32_t)kItems &&
+              at_new + size <= sm.item_at[oldest % kItems] + (uint32_t)p.ring_bytes)
+            break;
           uint64_t* eb = &sm.empty[oldest % kItems];
           const uint32_t par = (oldest / kItems) & 1u;
           if (!mbar_try_wait(eb, par)) {
@@ -539,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           ++landed;
         }
         inflight += size;
-        sm.item_pos[issued % kItems] = pos;
+        sm.item_at[issued % kItems] = at_new;
         sm.item_size[issued % kItems] = size;
         dst = ring_base + pos;
         fb = &sm.full[issued % kItems];
@@ -548,6 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         return true;
       };
       auto wait_list = [&](uint64_t* bar, uint32_t par) -> bool {
+        if (mbar_try_wait(bar, par)) return true;
         const uint64_t t0 = wait_start();
         while (!mbar_try_wait_sleep(bar, par, kSleepNs)) {
           if (aborted(sm)) return false;
@@ -555,49 +591,66 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         }
         return true;
       };
+      // One issue site for every item: per layer the P1^T rows in copies of
+      // p1_rows_per_item, the own P2 rows in copies of p2_rows, then one record per list
+      // entry: the first na as soon as the block's own list is known, the rest once the
+      // helpers have listed them.
       bool ok = true;
       for (int l = 0; l < p.L && ok; ++l) {
-        const LayerDev Ld = p.layers[l];
-        const int r = Ld.r;
-        const int k0 = (int)((long long)c * r / G), k1 = (int)((long long)(c + 1) * r / G);
-        const int p2_stride = p2_stride_of(r, PB);
-        const int p2_rows = max(1, min(p.nown_max, p.p2_item_bytes / p2_stride));
-        uint8_t* dst;
-        uint64_t* fb;
-        if (do_pred) {
-          for (int k = k0; k < k1 && ok; k += p.p1_rows_per_item) {
-            const int n = min(p.p1_rows_per_item, k1 - k);
-            const uint32_t bytes = (uint32_t)n * p.p1_row;
-            if (!(ok = begin_item(bytes, dst, fb))) break;
-            bulk_g2s(dst, Ld.p1t + (size_t)k * p.p1_row, bytes, fb);
-          }
-          const uint8_t* own = Ld.p2o + (size_t)c * p.nown_max * p2_stride;
-          for (int m = 0; m < nown && ok; m += p2_rows) {
-            const int n = min(p2_rows, nown - m);
-            const uint32_t bytes = (uint32_t)n * p2_stride;
-            if (!(ok = begin_item(bytes, dst, fb))) break;
-            bulk_g2s(dst, own + (size_t)m * p2_stride, bytes, fb);
+        // Layer l's predictor rows wait until layer l - 1's records are dotted: until then
+        // the records' reads have HBM to themselves, and the exchanges after them leave
+        // HBM idle for these copies.
+        if (l > 0 && do_ffn) {
+          const uint32_t par = (uint32_t)((l - 1) & 1);
+          if (!mbar_try_wait(&sm.fdone, par)) {
+            const uint64_t t0 = wait_start();
+            while (!mbar_try_wait_sleep(&sm.fdone, par, kSleepNs)) {
+              if (aborted(sm)) { ok = false; break; }
+              if (timed_out(t0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_RING_TIMEOUT); ok = false; break; }
+            }
+            if (!ok) break;
           }
         }
-        if (do_ffn && ok) {
-          pstamp(p, l, 20);
-          ok = wait_list(&sm.list_ready, (uint32_t)(l & 1));
-          pstamp(p, l, 21);
-          // The kept part of the list is known before the mask exchange ends, the rest
-          // after it.
-          const int na = ok ? sm.nlist_a : 0;
-          int e = 0;
-          for (; e < na && ok; ++e) {
-            if (!(ok = begin_item((uint32_t)p.rec_stride, dst, fb))) break;
-            bulk_g2s(dst, Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride, fb);
+        const LayerDev Ld = p.layers[l];
+        const int r = Ld.r;
+        const int k0 = (int)((unsigned)c * (unsigned)r / (unsigned)G);
+        const int k1 = (int)((unsigned)(c + 1) * (unsigned)r / (unsigned)G);
+        const int p2_stride = p2_stride_of(r, PB);
+        const int p2_rows = max(1, min(p.nown_max, p.p2_item_bytes / p2_stride));
+        const uint8_t* own = Ld.p2o + (size_t)c * p.nown_max * p2_stride;
+        const int n1 = do_pred ? (k1 - k0 + p.p1_rows_per_item - 1) / p.p1_rows_per_item : 0;
+        const int n2 = do_pred ? (nown + p2_rows - 1) / p2_rows : 0;
+        int na = 0, n = 0;   // records: handed over first, in all (known once listed)
+        for (int it = 0; ok; ++it) {
+          const uint8_t* src;
+          uint32_t bytes;
+          if (it < n1) {
+            const int k = k0 + it * p.p1_rows_per_item;
+            src = Ld.p1t + (size_t)k * p.p1_row;
+            bytes = (uint32_t)min(p.p1_rows_per_item, k1 - k) * p.p1_row;
+          } else if (it < n1 + n2) {
+            const int m = (it - n1) * p2_rows;
+            src = own + (size_t)m * p2_stride;
+            bytes = (uint32_t)min(p2_rows, nown - m) * p2_stride;
+          } else {
+            if (!do_ffn) break;
+            const int e = it - n1 - n2;
+            if (e == 0) {
+              if (!(ok = wait_list(&sm.list_ready, (uint32_t)(l & 1)))) break;
+              na = n = sm.na;
+            }
+            if (e == na && n == na) {
+              if (!(ok = wait_list(&sm.list2_ready, (uint32_t)(l & 1)))) break;
+              n = sm.nrec;
+            }
+            if (e >= n) break;
+            src = Ld.rec + (size_t)sm.list[e] * p.rec_stride;
+            bytes = (uint32_t)p.rec_stride;
           }
-          if (ok) ok = wait_list(&sm.list2_ready, (uint32_t)(l & 1));
-          const int n = ok ? sm.nlist : 0;
-          for (; e < n && ok; ++e) {
-            if (!(ok = begin_item((uint32_t)p.rec_stride, dst, fb))) break;
-            bulk_g2s(dst, Ld.rec + (size_t)sm.list[e] * p.rec_stride, (uint32_t)p.rec_stride, fb);
-          }
-          pstamp(p, l, 22);
+          uint8_t* dst;
+          uint64_t* fb;
+          if (!(ok = begin_item(bytes, dst, fb))) break;
+          bulk_g2s(dst, src, bytes, fb);
         }
       }
       // drain: never leave the block while a bulk copy may still write shared memory
@@ -630,17 +683,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
 
   int redbuf = 0;     // which half of sm.red the next block reduction uses
   uint32_t fseq = 0;  // F records of earlier layers (h slot of record e: (fseq + e) % kHr)
+  uint32_t dphase[2] = {0u, 0u};   // completed phases of dfull[0], dfull[1]
   for (int l = 0; l < p.L; ++l) {
     const LayerDev Ld = p.layers[l];
     const int r = Ld.r;
-    const int k0 = (int)((long long)c * r / G), k1 = (int)((long long)(c + 1) * r / G);
+    const int k0 = (int)((unsigned)c * (unsigned)r / (unsigned)G);
+    const int k1 = (int)((unsigned)(c + 1) * (unsigned)r / (unsigned)G);
     const int p2_stride = p2_stride_of(r, PB);
     const int p2_rows = max(1, min(p.nown_max, p.p2_item_bytes / p2_stride));
     const uint32_t tag_u = tag_of(epoch, l, EX_U), tag_m = tag_of(epoch, l, EX_M), tag_h = tag_of(epoch, l, EX_H),
                    tag_v = tag_of(epoch, l, EX_V);
     int nlist = 0;      // records this block dots
     int ntotal = 0;     // active entries of the layer (the down list)
-    bool signaled_a = false;
+    int hid0 = 0;       // h word of the block's first record: records publish h in list order
     stamp(p, l, 0);
     // this layer's x units, fp32, in registers for P-a
     uint32_t xr[NU][NB][XW];
@@ -703,14 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
       }
       stamp(p, l, 1);
       // ---------------------------------------------------------- u exchange
-      {
-        constexpr int KU = 6 * NB;   // r <= 1536
-        uint64_t w[KU];
-        poll_words<KU>(p.ux, t, kConsumerThreads, B * r, tag_u, w, sm, p);
-#pragma unroll
-        for (int k = 0; k < KU; ++k)
-          if (t + k * kConsumerThreads < B * r) u_s[t + k * kConsumerThreads] = tag_val(w[k]);
-      }
+      poll_linear<8>(p.ux, B * r, kConsumerWarps, tag_u, reinterpret_cast<uint32_t*>(u_s), sm, p);
       named_bar_sync(kRedBar, kConsumerThreads);
       stamp(p, l, 2);
 
@@ -826,127 +874,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
           const uint32_t word = __ballot_sync(0xffffffffu, (tb >> b) & 1u);
-          if (lane == 0 && b < B) st_tag_u(p.mx + ((size_t)c * 4 + b) * kMaxOwnWords + w, word, tag_m);
+          if (lane == 0 && b < B) st_tag_u(p.mx + ((size_t)c * B + b) * nw + w, word, tag_m);
         }
       }
-      named_bar_sync(kRedBar, kConsumerThreads);
-      const int n_own = sm.count;
-      const int floor = Ld.keep_floor;
-      // the kept part (own records every block keeps whatever the counts) goes to the
-      // producer now, so its copies run during the mask exchange
       if (t == 0) {
-        sm.nlist_a = min(n_own, floor);
+        // own records handed to the producer now, whatever the exchange says
+        sm.na = min(sm.count, max(Ld.keep_floor, 1));
         mbar_arrive(&sm.list_ready);
       }
-      signaled_a = true;
+      named_bar_sync(kRedBar, kConsumerThreads);
+      nlist = sm.count;
+      hid0 = c * nown_max;
       stamp(p, l, 4);
-
-      // ---------------------------------------------------------- mask exchange
-      {
-        const int per = B * nw;
-        const int nq = G * per;
-        constexpr int MQ = 16;
-        if (NB > B)
-          for (int q = t; q < G * NB * nw; q += kConsumerThreads)
-            if ((q / nw) % NB >= B) ob[q] = 0u;
-        for (int base = 0; base < nq; base += MQ * kConsumerThreads) {
-          uint64_t w[MQ];
-          uint32_t need = 0;
-#pragma unroll
-          for (int i = 0; i < MQ; ++i) {
-            w[i] = 0;
-            if (base + t + i * kConsumerThreads < nq) need |= 1u << i;
-          }
-          bool started = false;
-          uint64_t tp0 = 0;
-          while (need) {
-#pragma unroll
-            for (int i = 0; i < MQ; ++i)
-              if (need >> i & 1u) {
-                const int q = base + t + i * kConsumerThreads;
-                const int o = q / per, rem = q % per;
-                w[i] = ld_tag(p.mx + ((size_t)o * 4 + rem / nw) * kMaxOwnWords + rem % nw);
-              }
-#pragma unroll
-            for (int i = 0; i < MQ; ++i)
-              if ((need >> i & 1u) && tag_ok(w[i], tag_m)) need &= ~(1u << i);
-            if (!need || aborted(sm)) break;
-            if (!started) { tp0 = wait_start(); started = true; }
-            else if (timed_out(tp0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
-            if (p.poll_ns) __nanosleep(p.poll_ns);
-          }
-#pragma unroll
-          for (int i = 0; i < MQ; ++i) {
-            const int q = base + t + i * kConsumerThreads;
-            if (q < nq) {
-              // only bits of neurons the owner has can be set (a word of an aborted
-              // exchange may hold anything)
-              const int o = q / per, rem = q % per, ww = rem % nw;
-              const int nown_o = (o < f) ? (f - o + G - 1) / G : 0;
-              const int nv = min(32, max(0, nown_o - 32 * ww));
-              const uint32_t valid = nv >= 32 ? 0xFFFFFFFFu : ((1u << nv) - 1u);
-              ob[((size_t)o * NB + rem / nw) * nw + ww] = (uint32_t)w[i] & valid;
-            }
-          }
-        }
-      }
-      named_bar_sync(kRedBar, kConsumerThreads);
-      stamp(p, l, 5);
-      if (t < G) {
-        int n = 0;
-        for (int w = 0; w < nw; ++w) n += __popc(union_word<NB>(ob, t, w, nw));
-        sm.cnt[t] = n;
-      }
-      named_bar_sync(kRedBar, kConsumerThreads);
-
-      // ---------------------------------------------------------- balanced assignment
-      // N = the sum of the counts; target T = max(ceil(N / G), floor).  Block c keeps its
-      // first min(n_c, T) own entries; the entries past T of the blocks above the target,
-      // in (block, position) order, fill the blocks below it in block order.  Every block
-      // derives the same assignment from the counts alone.
-      {
-        const int cv = (t < G) ? sm.cnt[t] : 0;
-        int v1[1] = {cv}, e1[1], s1[1];
-        block_excl_scan<1>(v1, e1, s1, sm, warp, lane);
-        const int N = s1[0];
-        const int T = max((N + G - 1) / G, floor);
-        int v2[2] = {(t < G) ? max(0, cv - T) : 0, (t < G) ? max(0, T - cv) : 0}, e2[2], s2[2];
-        block_excl_scan<2>(v2, e2, s2, sm, warp, lane);
-        if (t < G) {
-          sm.pre[t] = e1[0];
-          sm.xpre[t] = e2[0];
-        }
-        if (t == c) sm.bal[1] = e2[1];
-        if (t == 0) {
-          sm.pre[G] = N;
-          sm.xpre[G] = s2[0];
-          sm.bal[0] = T;
-          sm.bal[2] = s2[0];
-        }
-        named_bar_sync(kRedBar, kConsumerThreads);
-        const int dstart = sm.bal[1], xtotal = sm.bal[2];
-        const int keep = min(n_own, T);
-        const int deficit = max(0, T - n_own);
-        const int ntake = max(0, min(dstart + deficit, xtotal) - dstart);
-        for (int q = t; q < keep; q += kConsumerThreads) sm.list_ent[q] = sm.pre[c] + q;
-        for (int q = t; q < ntake; q += kConsumerThreads) {
-          const int x = dstart + q;
-          int lo = 0, hi = G;   // owner o: xpre[o] <= x < xpre[o + 1]
-          while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (sm.xpre[mid] <= x) lo = mid;
-            else hi = mid;
-          }
-          const int k = T + (x - sm.xpre[lo]);
-          const int m = owner_select<NB>(ob, lo, k, nw);
-          const int i = lo + max(m, 0) * G;
-          sm.list[keep + q] = i < f ? i : 0;
-          sm.list_ent[keep + q] = sm.pre[lo] + k;
-          sm.list_bits[keep + q] = (uint8_t)owner_token_bits<NB>(ob, lo, max(m, 0), nw);
-        }
-        nlist = keep + ntake;
-        ntotal = N;
-      }
       if (t == 0) {
         atomicAdd(p.active_total, (unsigned long long)nlist);
         if (p.layer_count) atomicAdd(p.layer_count + l, nlist);
@@ -958,7 +897,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         if (t == 0) atomicExch(p.err, DEV_ERR_INDEX);
         cnt = 0;
       }
-      const int a0 = (int)((long long)c * cnt / G), a1 = (int)((long long)(c + 1) * cnt / G);
+      const int a0 = (int)((unsigned)c * (unsigned)cnt / (unsigned)G);
+      const int a1 = (int)((unsigned)(c + 1) * (unsigned)cnt / (unsigned)G);
       nlist = a1 - a0;
       if (nlist > kMaxList) {
         if (t == 0) atomicExch(p.err, DEV_ERR_LIST);
@@ -970,109 +910,127 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         uint32_t bits = 0;
         for (int b = 0; b < B; ++b) bits |= ((__ldg(p.mask_in + (size_t)b * words + (i >> 5)) >> (i & 31)) & 1u) << b;
         sm.list[e] = i;
-        sm.list_ent[e] = a0 + e;
         sm.list_bits[e] = (uint8_t)bits;
       }
-      if (t == 0) atomicAdd(p.active_total, (unsigned long long)nlist);
+      if (t == 0) {
+        atomicAdd(p.active_total, (unsigned long long)nlist);
+        sm.na = sm.own_cnt = sm.nrec = nlist;
+        mbar_arrive(&sm.list_ready);
+      }
       ntotal = cnt;
+      hid0 = a0;
     }
 
     named_bar_sync(kRedBar, kConsumerThreads);
-    if (t == 0) {
-      if (!signaled_a) {
-        sm.nlist_a = nlist;
-        mbar_arrive(&sm.list_ready);
-      }
-      sm.nlist = nlist;
-      mbar_arrive(&sm.list2_ready);
-    }
     stamp(p, l, 6);
     stamp_val(p, l, 14, nlist);
-    stamp_val(p, l, 15, ntotal);
 
     // ------------------------------------------------------------ down list and copies
     // Chunk k holds the active entries [k*dch, (k+1)*dch) of the layer in owner-major
-    // order (the caller's order for a given list); dlist half k%2 holds their neuron ids
-    // and dbuf half k%2 their units [cu0, cu1).  Each thread copies, and later reads,
-    // only its own slots, so its cp.async groups alone order the copies and the reads.
-    const int nchunks = (ntotal + dch - 1) / dch;
+    // order (the caller's order for a given list); dlist half k%2 holds their neuron ids,
+    // dhid half k%2 the index of their h words (owner o's records publish h from word
+    // o * nown_max on; a caller's list, at its entry index) and dbuf half k%2 their units
+    // [cu0, cu1).  The helper warps build the halves and copy the units (cp.async); the
+    // copies of half j complete a phase of dfull[j].
     const uint8_t* dn = Ld.rec + p.dn_off;
-    auto build_dlist = [&](int k) {
-      const int lo = k * dch, hi = min(ntotal, lo + dch);
+    const int ht = t - kFWarps * 32;   // helper thread index (>= 0 in the helper warps)
+    int woff = 0;                      // helpers: the layer's entries before this thread's mask words
+    // chunks k .. k + nk - 1 (nk = 2 only from an even k: the two halves in order)
+    auto build_dlist = [&](int k, int nk) {
+      const int lo = k * dch, hi = min(ntotal, lo + nk * dch);
       int32_t* dl = dlist + (k & 1) * dch;
+      int32_t* dh = dhid + (k & 1) * dch;
       if (do_pred) {
-        for (int o = t; o < G; o += kConsumerThreads) {
-          const int e0 = sm.pre[o], e1 = e0 + sm.cnt[o];
-          if (e1 <= lo || e0 >= hi) continue;
-          int e = e0;
-          for (int w = 0; w < nw && e < hi; ++w) {
-            uint32_t u = union_word<NB>(ob, o, w, nw);
-            const int n = __popc(u);
-            if (e + n <= lo) { e += n; continue; }
+        // this thread's run of mask words, its first entry at woff: set bits in order
+        int e = woff;
+        int o = wj0 / nw, w = wj0 - o * nw;
+        const uint32_t dla = smem_u32(dl), dha = smem_u32(dh);
+        for (int j = wj0; j < wj1 && e < hi; ++j) {
+          uint32_t u = union_word(ob, o, w, nw, B);
+          const int n = __popc(u);
+          if (e + n > lo) {
+            const int pre_o = sm.pre[o];
             while (u && e < hi) {
               const int bit = __ffs(u) - 1;
               u &= u - 1;
-              if (e >= lo) dl[e - lo] = o + (32 * w + bit) * G;
+              if (e >= lo) {
+                sts_u32(dla + 4u * (uint32_t)(e - lo), (uint32_t)(o + (32 * w + bit) * G));
+                // owner o's h words start at o * nown_max
+                sts_u32(dha + 4u * (uint32_t)(e - lo), (uint32_t)(o * nown_max + (e - pre_o)));
+              }
               ++e;
             }
+          } else {
+            e += n;
+          }
+          if (++w == nw) {
+            w = 0;
+            ++o;
           }
         }
       } else {
-        for (int e = lo + t; e < hi; e += kConsumerThreads) {
+        for (int e = lo + ht; e < hi; e += kHelperThreads) {
           int i = __ldg(p.idx_in + e);
           if (i < 0 || i >= f) i = 0;   // reported above
           dl[e - lo] = i;
+          dh[e - lo] = e;
         }
       }
     };
+    // helper lane mapping of the copies: the F mapping of the down pass over 4 warps
+    const int hde0 = (warp - kFWarps) * epw + lane / lpe;
+    const int hdstep = (kConsumerWarps - kFWarps) * epw;
     auto issue_down = [&](int k) {
-      if (dw < 0) return;
-      const int lo = k * dch, hi = min(ntotal, lo + dch);
-      const int32_t* dl = dlist + (k & 1) * dch;
-      const int half = (k & 1) * dch;
-      for (int e = lo + de0; e < hi; e += dstep) {
-        const int i = dl[e - lo];
-        const uint8_t* row = dn + (size_t)i * p.dn_stride;
-        const uint32_t slot = (uint32_t)((half + e - lo) * pmax + dw);
-        cpa16(dbuf_u + slot * 16u, row + (size_t)(cu0 + dw) * 16);
-        if constexpr (FAM == FAM_Q4) cpa4(dsc_u + slot * 4u, row + (size_t)(d >> 1) + (size_t)((cu0 + dw) >> 1) * 4);
+      if (dw >= 0) {
+        const int lo = k * dch, hi = min(ntotal, lo + dch);
+        const int32_t* dl = dlist + (k & 1) * dch;
+        const int half = (k & 1) * dch;
+        for (int e = lo + hde0; e < hi; e += hdstep) {
+          const int i = dl[e - lo];
+          const uint8_t* row = dn + (size_t)i * p.dn_stride;
+          const uint32_t slot = (uint32_t)((half + e - lo) * pmax + dw);
+          cpa16(dbuf_u + slot * 16u, row + (size_t)(cu0 + dw) * 16);
+          if constexpr (FAM == FAM_Q4)
+            cpa4(dsc_u + slot * 4u, row + (size_t)(d >> 1) + (size_t)((cu0 + dw) >> 1) * 4);
+        }
       }
+      cpa_arrive_noinc(&sm.dfull[k & 1]);
     };
-    build_dlist(0);
-    if (nchunks > 1) build_dlist(1);
-    named_bar_sync(kRedBar, kConsumerThreads);
-    issue_down(0);
-    cpa_commit();
-    if (nchunks > 1) issue_down(1);
-    cpa_commit();
-    stamp(p, l, 7);
 
     // ------------------------------------------------------------ F: records -> h
-    // The 16 consumer warps form groups of KG; group g dots records g, g + 16/KG, ...
-    // with no block barrier: each warp of the group waits for the record to land, dots
-    // its slice of the units with x from shared memory, reduces across its lanes and
-    // posts its partial sums in the record's h slot.  The last warp of the group to post
-    // sums the group's partials in a fixed order, forms h and publishes it.
-    {
+    // Warps below kFWarps form groups of KG; group g dots records g, g + NG, ... in ring
+    // order: each warp of the group waits for the record to land, dots its slice of the
+    // units with x from shared memory, reduces across its lanes and posts its partial
+    // sums in the record's h slot.  The last warp of the group to post sums the group's
+    // partials in a fixed order, forms h and publishes it.  Records past na wait for the
+    // helpers' list (kAssignBar).  The helper warps take the mask exchange, the balanced
+    // assignment, the down list and the down copies meanwhile.
+    if (warp < kFWarps) {
       constexpr int NV = (ACT == PI_REGLU) ? 2 : 1;
       constexpr int NVAL = NB * NV;                 // partial sums per warp and record
       constexpr int V = pow2_ceil(NVAL);
       constexpr int LG = log2_exact(V);
-      constexpr int KG = f_group_warps(FAM, ACT, NB);
-      constexpr int NG = kConsumerWarps / KG;       // records dotted at once
-      static_assert(KG * NVAL <= 16 && kConsumerWarps % KG == 0, "h slot layout");
+      constexpr int KG = f_group_warps(ACT, NB);
+      constexpr int NG = kFWarps / KG;              // records dotted at once
+      static_assert(KG * NVAL <= 16 && kFWarps % KG == 0 && kHr % NG == 0, "h slot layout");
       const uint32_t base = smem_u32(ring.base), xsa = smem_u32(xs);
       const uint32_t item0 = ring.item;
       const int kq = warp % KG;
-      long long f_wait = 0;   // diagnostics: cycles warp 0 waits for records
       uint32_t hd = ring.head;   // ring head before record id (dot cursor)
       int id = 0;
-      for (int e = warp / KG; e < nlist; e += NG) {
+      const int na = sm.na;
+      int nrec = na, own_cnt = na;
+      for (int e = warp / KG;; e += NG) {
+        if (e >= na && nrec == na && own_cnt == na) {
+          named_bar_sync(kAssignBar, kConsumerThreads);   // the rest of the list is in place
+          nrec = sm.nrec;
+          own_cnt = sm.own_cnt;
+          if (nrec == na) own_cnt = -1;   // (no second wait)
+        }
+        if (e >= nrec) break;
         uint32_t pos = 0;
         for (; id <= e; ++id) pos = ring_place(hd, (uint32_t)p.rec_stride, ring.cap);
-        const long long wt0 = diag_clock(p);
         ring_wait_item_warp(item0 + e, sm, p);
-        f_wait += diag_clock(p) - wt0;
         if (e == 0) stamp(p, l, 8);
         float au[NB], ag[NB];
         record_dot<FAM, ACT, NB>(base + pos, xsa, p, nunits, 32 * kq + lane, 32 * KG, au, ag);
@@ -1086,7 +1044,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         }
         const float sw = reduce_scatter<V>(v, lane);   // lane k: value k >> (5 - LG)
         const uint32_t s = (fseq + (uint32_t)e) % kHr;
-        if ((lane & ((32 >> LG) - 1)) == 0 && (lane >> (5 - LG)) < NVAL) sm.hpart[s][kq * NVAL + (lane >> (5 - LG))] = sw;
+        if ((lane & ((32 >> LG) - 1)) == 0 && (lane >> (5 - LG)) < NVAL)
+          sm.hpart[s][kq * NVAL + (lane >> (5 - LG))] = sw;
         const float bi = lds_f32(base + pos + (uint32_t)p.bias_off);
         __syncwarp();
         if (lane == 0) {
@@ -1094,7 +1053,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           if (atomicAdd(&sm.hcnt[s], 1) == KG - 1) {
             __threadfence_block();
             const volatile float* hp = sm.hpart[s];
-            const int ent = sm.list_ent[e];
+            const int ent = e < max(own_cnt, na) ? hid0 + e : sm.list_hid[e];
             const uint32_t bits = sm.list_bits[e];
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
@@ -1122,12 +1081,154 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
         }
         ring_release_item(item0 + e, sm, (uint32_t)(kConsumerWarps / KG));
       }
-      for (int q = 0; q < nlist; ++q) ring_place(ring.head, (uint32_t)p.rec_stride, ring.cap);
-      ring.item = item0 + (uint32_t)nlist;
-      fseq += (uint32_t)nlist;
-      stamp_val(p, l, 19, f_wait);
+      stamp(p, l, 9);
+      if (t == 0) mbar_arrive(&sm.fdone);
+    } else {
+      if (do_pred) {
+        // ---------------------------------------------------------- mask exchange
+        poll_words<8>(p.mx, [](int q) { return (size_t)q; }, G * B * nw, kConsumerWarps - kFWarps, tag_m, ob, sm, p,
+                      kFWarps * 32);
+        named_bar_sync(kHelpBar, kHelperThreads);
+        hstamp(p, l, 5);
+        // The mask words in owner-major order (word j: owner j / nw, word j % nw) are
+        // split into runs of consecutive words, one run a helper thread.  Only bits of
+        // neurons the owner has can be set (a word of an aborted exchange may hold
+        // anything): the rest are cleared in place.
+        int wcnt = 0;
+        for (int j = wj0; j < wj1; ++j) {
+          const int o = j / nw, w = j - o * nw;
+          const int nown_o = o < own_rem ? nown_max : nown_max - 1;
+          const int nv = min(32, max(0, nown_o - 32 * w));
+          const uint32_t valid = nv >= 32 ? 0xFFFFFFFFu : ((1u << nv) - 1u);
+          uint32_t u = 0;
+          for (int b = 0; b < B; ++b) {
+            uint32_t* wp = ob + ((size_t)o * B + b) * nw + w;
+            const uint32_t x = *wp & valid;
+            *wp = x;
+            u |= x;
+          }
+          wcnt += __popc(u);
+        }
+        // the prefix of the counts, then of the excess over T and of the shortfall
+        const int hw = warp - kFWarps;
+        auto helper_scan = [&](int v, int slot, int& total) -> int {   // exclusive prefix over helpers
+          int incl = v;
+#pragma unroll
+          for (int k = 1; k < 32; k <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, incl, k);
+            if (lane >= k) incl += x;
+          }
+          if (lane == 31) sm.wsum[slot][hw] = incl;
+          named_bar_sync(kHelpBar, kHelperThreads);
+          int off = 0;
+          total = 0;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps - kFWarps; ++w) {
+            const int x = sm.wsum[slot][w];
+            off += w < hw ? x : 0;
+            total += x;
+          }
+          return off + incl - v;   // exclusive
+        };
+        int N = 0;
+        woff = helper_scan(wcnt, 0, N);   // entries before this thread's first word
+        {
+          int e = woff;
+          for (int j = wj0; j < wj1; ++j) {
+            const int o = j / nw, w = j - o * nw;
+            if (w == 0) sm.pre[o] = e;
+            e += __popc(union_word(ob, o, w, nw, B));
+          }
+          if (ht == 0) sm.pre[G] = N;
+        }
+        named_bar_sync(kHelpBar, kHelperThreads);
+        int n2[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int o = 2 * ht + i;
+          n2[i] = o < G ? sm.pre[o + 1] - sm.pre[o] : 0;
+        }
+        const int T = max(1, (N + G - 1) / G);
+        // the excess over T and the shortfall below it, scanned together
+        const int x0 = max(0, n2[0] - T), x1 = max(0, n2[1] - T);
+        const int s0 = (2 * ht < G) ? max(0, T - n2[0]) : 0, s1 = (2 * ht + 1 < G) ? max(0, T - n2[1]) : 0;
+        int px, ps, xtotal;
+        {
+          int ix = x0 + x1, is = s0 + s1;
+#pragma unroll
+          for (int k = 1; k < 32; k <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, ix, k), b = __shfl_up_sync(0xffffffffu, is, k);
+            if (lane >= k) {
+              ix += a;
+              is += b;
+            }
+          }
+          if (lane == 31) {
+            sm.wsum[1][hw] = ix;
+            sm.wsum[1][kConsumerWarps / 2 + hw] = is;
+          }
+          named_bar_sync(kHelpBar, kHelperThreads);
+          int ox = 0, os = 0;
+          xtotal = 0;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps - kFWarps; ++w) {
+            const int a = sm.wsum[1][w], b = sm.wsum[1][kConsumerWarps / 2 + w];
+            ox += w < hw ? a : 0;
+            os += w < hw ? b : 0;
+            xtotal += a;
+          }
+          px = ox + ix - (x0 + x1);
+          ps = os + is - (s0 + s1);
+        }
+        sm.xpre[2 * ht] = px;
+        sm.xpre[2 * ht + 1] = px + x0;
+        if (ht == kHelperThreads - 1) sm.xpre[2 * kHelperThreads] = xtotal;
+        if (2 * ht == c) sm.wsum[0][kConsumerWarps - 1] = ps;
+        if (2 * ht + 1 == c) sm.wsum[0][kConsumerWarps - 1] = ps + s0;
+        named_bar_sync(kHelpBar, kHelperThreads);
+        const int n_own = nlist;
+        const int dstart = sm.wsum[0][kConsumerWarps - 1];
+        // this block dots its first own_cnt own records (those already handed to the
+        // producer included) and then the taken ones, listed from entry own_cnt on
+        const int own_cnt = max(min(n_own, T), sm.na);
+        const int deficit = max(0, T - n_own);
+        const int ntake = max(0, min(dstart + deficit, xtotal) - dstart);
+        if (ht == 0) {
+          sm.own_cnt = own_cnt;
+          sm.nrec = own_cnt + ntake;
+        }
+        for (int q = ht; q < ntake; q += kHelperThreads) {
+          const int x = dstart + q;
+          int lo = 0, hi = G;   // owner o: xpre[o] <= x < xpre[o + 1]
+          while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (sm.xpre[mid] <= x) lo = mid;
+            else hi = mid;
+          }
+          const int k = T + (x - sm.xpre[lo]);
+          const int m = owner_select(ob, lo, k, nw, B);
+          const int i = lo + max(m, 0) * G;
+          sm.list[own_cnt + q] = i < f ? i : 0;
+          sm.list_bits[own_cnt + q] = (uint8_t)(m >= 0 ? owner_token_bits(ob, lo, m, nw, B) : 0u);
+          sm.list_hid[own_cnt + q] = lo * nown_max + k;
+        }
+        ntotal = N;
+      }
+      named_bar_sync(kHelpBar, kHelperThreads);
+      if (ht == 0) mbar_arrive(&sm.list2_ready);          // the producer copies the rest
+      named_bar_arrive(kAssignBar, kConsumerThreads);   // the F warps dot it
+      hstamp(p, l, 29);
+      const int nchunks = (ntotal + dch - 1) / dch;
+      build_dlist(0, 2);
+      named_bar_sync(kHelpBar, kHelperThreads);
+      hstamp(p, l, 23);
+      if (nchunks > 0) issue_down(0);
+      if (nchunks > 1) issue_down(1);
+      hstamp(p, l, 7);
     }
-    stamp(p, l, 9);
+    if (do_pred) ntotal = sm.pre[G];   // every warp: the layer's active count
+    const int nchunks = (ntotal + dch - 1) / dch;
+    stamp_val(p, l, 15, ntotal);
 
     // ------------------------------------------------------------ down: y of the slice
     float acc[NB][PE];
@@ -1136,70 +1237,58 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
 #pragma unroll
       for (int e = 0; e < PE; ++e) acc[b][e] = 0.f;
     long long h_wait = 0;   // diagnostics: cycles thread 0 polls for h
+    // The h words of resident entries (at their dhid words) are polled by every consumer
+    // thread at once (one polling round) into shared memory: chunks 0 and 1 together, later
+    // chunks one at a time.  Entry e of chunk k sits in slot e - (k - k % 2) * dch.
+    auto poll_h = [&](int e_lo, int e_hi, int slot0) {
+      const long long wt0 = diag_clock(p);
+      const int32_t* hid = dhid + slot0;
+      poll_words<8>(p.hx, [&](int q) { return (size_t)hid[q / B] * B + (size_t)(q % B); }, (e_hi - e_lo) * B,
+                    kConsumerWarps, tag_h, reinterpret_cast<uint32_t*>(hs) + (size_t)slot0 * B, sm, p);
+      h_wait += diag_clock(p) - wt0;
+    };
+    // every warp is past F and the down list halves 0 and 1 are built
+    named_bar_sync(kRedBar, kConsumerThreads);
+    {
+      // the ring past this layer's records (every consumer keeps the same ring state)
+      const int nr = sm.nrec;
+      for (int q = 0; q < nr; ++q) ring_place(ring.head, (uint32_t)p.rec_stride, ring.cap);
+      ring.item += (uint32_t)nr;
+      fseq += (uint32_t)nr;
+    }
     for (int k = 0; k < nchunks; ++k) {
-      cpa_wait_but_newest();   // this thread's copies of chunk k have landed
+      const int lo = k * dch, hi = min(ntotal, lo + dch);
+      if (k == 0) poll_h(0, min(ntotal, 2 * dch), 0);
+      else if (k >= 2) poll_h(lo, hi, (k & 1) * dch);
+      if (k == 0) stamp(p, l, 25);
+      if (k != 1) named_bar_sync(kRedBar, kConsumerThreads);
+      if (k == 0) stamp(p, l, 26);
+      bar_wait(&sm.dfull[k & 1], dphase[k & 1] & 1u, sm, p);   // the copies of chunk k have landed
+      ++dphase[k & 1];
+      if (k == 0) stamp(p, l, 27);
       if (dw >= 0) {
-        const int lo = k * dch, hi = min(ntotal, lo + dch);
-        const int32_t* dl = dlist + (k & 1) * dch;
         const int half = (k & 1) * dch;
-        constexpr int HB = NB == 1 ? 8 : NB == 2 ? 4 : 2;   // entries whose h words one polling round reads
-        for (int eb = lo + de0; eb < hi; eb += HB * dstep) {
-          uint64_t hw[HB][NB];
-          uint32_t need = 0;
+        for (int e = lo + de0; e < hi; e += dstep) {
+          float h[NB];
 #pragma unroll
-          for (int q = 0; q < HB; ++q)
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-              hw[q][b] = 0;
-              if (eb + q * dstep < hi && b < B) need |= 1u << (q * NB + b);
-            }
-          const long long wt0 = diag_clock(p);
-          bool started = false;
-          uint64_t tp0 = 0;
-          while (need) {
-#pragma unroll
-            for (int q = 0; q < HB; ++q)
-#pragma unroll
-              for (int b = 0; b < NB; ++b)
-                if (need >> (q * NB + b) & 1u) hw[q][b] = ld_tag(p.hx + (size_t)(eb + q * dstep) * B + b);
-#pragma unroll
-            for (int q = 0; q < HB; ++q)
-#pragma unroll
-              for (int b = 0; b < NB; ++b)
-                if ((need >> (q * NB + b) & 1u) && tag_ok(hw[q][b], tag_h)) need &= ~(1u << (q * NB + b));
-            if (!need || aborted(sm)) break;
-            if (!started) { tp0 = wait_start(); started = true; }
-            else if (timed_out(tp0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
-            if (p.poll_ns) __nanosleep(p.poll_ns);
+          for (int b = 0; b < NB; ++b) h[b] = b < B ? hs[(size_t)(half + e - lo) * B + b] : 0.f;
+          const uint32_t slot = (uint32_t)((half + e - lo) * pmax + dw);
+          float sc = 0.f;
+          if constexpr (FAM == FAM_Q4) {
+            const uint32_t sw = lds_u32(dsc_u + slot * 4u);
+            sc = __half2float(__ushort_as_half((unsigned short)(((cu0 + dw) & 1) ? (sw >> 16) : (sw & 0xFFFFu))));
           }
-          h_wait += diag_clock(p) - wt0;
-#pragma unroll
-          for (int q = 0; q < HB; ++q) {
-            const int e = eb + q * dstep;
-            if (e < hi) {
-              float h[NB];
-#pragma unroll
-              for (int b = 0; b < NB; ++b) h[b] = b < B ? tag_val(hw[q][b]) : 0.f;
-              const uint32_t slot = (uint32_t)((half + e - lo) * pmax + dw);
-              float sc = 0.f;
-              if constexpr (FAM == FAM_Q4) {
-                const uint32_t sw = lds_u32(dsc_u + slot * 4u);
-                sc = __half2float(__ushort_as_half((unsigned short)(((cu0 + dw) & 1) ? (sw >> 16) : (sw & 0xFFFFu))));
-              }
-              down_unit_fma<FAM, NB>(dbuf_u + slot * 16u, sc, h, acc);
-            }
-          }
+          down_unit_fma<FAM, NB>(dbuf_u + slot * 16u, sc, h, acc);
         }
       }
       if (k + 2 < nchunks) {
-        named_bar_sync(kRedBar, kConsumerThreads);   // every thread is done with dlist half k%2
-        build_dlist(k + 2);
-        named_bar_sync(kRedBar, kConsumerThreads);
-        issue_down(k + 2);
+        named_bar_sync(kRedBar, kConsumerThreads);   // every thread is done with dlist, hs and dbuf half k%2
+        if (warp >= kFWarps) build_dlist(k + 2, 1);
+        named_bar_sync(kRedBar, kConsumerThreads);   // chunk k + 2's dlist and dhid are in place
+        if (warp >= kFWarps) issue_down(k + 2);
       }
-      cpa_commit();
     }
-    cpa_wait_all();
+    stamp(p, l, 28);
     stamp_val(p, l, 17, h_wait);
     stamp(p, l, 10);
 
@@ -1223,158 +1312,84 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const FusedParams p)
           for (int e = 0; e < PE; ++e) dred[(warp * pmax + dw) * V + b * PE + e] = acc[b][e];
       }
       named_bar_sync(kRedBar, kConsumerThreads);
-      float* vsl = dred + kConsumerWarps * pmax * V;   // [NB][ncol] v of the slice
-      if (t < B * ncol) {
-        const int b = t / ncol, q = t % ncol, w = q / PE, e = q % PE;
-        float y = 0.f;
-        for (int k = 0; k < kConsumerWarps; ++k) y += dred[(k * pmax + w) * V + b * PE + e];
-        const int col = col0 + q;
+      // warp b forms token b's slice: y, v = x + y and its (sum, sum of squares), which
+      // follow v in the exchange array
+      if (warp < B) {
+        const int b = warp;
+        float s = 0.f, s2 = 0.f;
+        for (int q = lane; q < ncol; q += 32) {
+          const int w = q / PE, e = q % PE;
+          float y = 0.f;
+          for (int k = 0; k < kConsumerWarps; ++k) y += dred[(k * pmax + w) * V + b * PE + e];
+          const int col = col0 + q;
+          if (do_glue) {
+            const float v = xs_val<FAM>(xs, b * d + col) + y;
+            st_tag(p.vx + (size_t)b * d + col, v, tag_v);
+            if (p.trace.y) p.trace.y[((size_t)l * B + b) * d + col] = y;
+            s += v;
+            s2 += v * v;
+          } else {
+            p.y_out[(size_t)b * d + col] = y;
+          }
+        }
         if (do_glue) {
-          const float v = xs_val<FAM>(xs, b * d + col) + y;
-          vsl[b * ncol + q] = v;
-          st_tag(p.vx + (size_t)b * d + col, v, tag_v);
-          if (p.trace.y) p.trace.y[((size_t)l * B + b) * d + col] = y;
-        } else {
-          p.y_out[(size_t)b * d + col] = y;
+          s = warp_sum(s);
+          s2 = warp_sum(s2);
+          if (lane == 0) {
+            st_tag(p.vx + (size_t)B * d + ((size_t)b * G + c) * 2, s, tag_v);
+            st_tag(p.vx + (size_t)B * d + ((size_t)b * G + c) * 2 + 1, s2, tag_v);
+          }
         }
       }
       if (!do_glue) break;
-      named_bar_sync(kRedBar, kConsumerThreads);
-      if (warp < NB) {
-        float s = 0.f, s2 = 0.f;
-        if (warp < B)
-          for (int q = lane; q < ncol; q += 32) {
-            const float v = vsl[warp * ncol + q];
-            s += v;
-            s2 += v * v;
-          }
-        s = warp_sum(s);
-        s2 = warp_sum(s2);
-        if (lane == 0 && warp < B) {
-          st_tag(p.sx + ((size_t)warp * G + c) * 2, s, tag_v);
-          st_tag(p.sx + ((size_t)warp * G + c) * 2 + 1, s2, tag_v);
-        }
-      }
     }
     stamp(p, l, 11);
 
     // ------------------------------------------------------------ glue: x' = (v - mean) / sd
-    // One polling round reads every v and every slice's (sum, sum of squares).
+    // The consumer threads poll every slice's (sum, sum of squares), which follow v in the
+    // same array, and then all of v into the down buffers (free now); the moments give
+    // each token's mean and 1 / sd, and every thread forms its elements of x'.
     {
-      const int npairs = B * d / 2;
-      const int nmom = 2 * G * B;
-      constexpr int MQ = (2 * kMaxGrid * 4 + kConsumerThreads - 1) / kConsumerThreads;
-      uint64_t w0[8], w1[8], wm[MQ];
-      uint32_t need = 0, needm = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        w0[k] = w1[k] = 0;
-        if (t + k * kConsumerThreads < npairs) need |= 1u << k;
-      }
-#pragma unroll
-      for (int i = 0; i < MQ; ++i) {
-        wm[i] = 0;
-        if (t + i * kConsumerThreads < nmom) needm |= 1u << i;
-      }
-      {
-        bool started = false;
-        uint64_t tp0 = 0;
-        while (need | needm) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if (need >> k & 1u) ld_tag2(p.vx + 2 * (size_t)(t + k * kConsumerThreads), w0[k], w1[k]);
-#pragma unroll
-          for (int i = 0; i < MQ; ++i)
-            if (needm >> i & 1u) wm[i] = ld_tag(p.sx + t + i * kConsumerThreads);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if ((need >> k & 1u) && tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
-#pragma unroll
-          for (int i = 0; i < MQ; ++i)
-            if ((needm >> i & 1u) && tag_ok(wm[i], tag_v)) needm &= ~(1u << i);
-          if (!(need | needm) || aborted(sm)) break;
-          if (!started) { tp0 = wait_start(); started = true; }
-          else if (timed_out(tp0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
-          if (p.poll_ns) __nanosleep(p.poll_ns);
-        }
-      }
-      named_bar_sync(kRedBar, kConsumerThreads);   // nobody reads vsl or xs any more
-      stamp(p, l, 12);
-      float* mom = dred;                            // [B][G][2]
-#pragma unroll
-      for (int i = 0; i < MQ; ++i)
-        if (t + i * kConsumerThreads < nmom) mom[t + i * kConsumerThreads] = tag_val(wm[i]);
+      float* gbuf = reinterpret_cast<float*>(dsmem + p.off_dlist);   // [B][d] v, then [B][G][2]
+      // the moments, published after v, first: the repeated polls then touch only the
+      // few lines they sit in, and v is usually complete at the first look
+      poll_linear<8>(p.vx + (size_t)B * d, 2 * B * G, kConsumerWarps, tag_v,
+                     reinterpret_cast<uint32_t*>(gbuf) + (size_t)B * d, sm, p);
+      poll_linear<16>(p.vx, B * d, kConsumerWarps, tag_v, reinterpret_cast<uint32_t*>(gbuf), sm, p);
       named_bar_sync(kRedBar, kConsumerThreads);
-      if (warp < NB) {
+      stamp(p, l, 12);
+      if (warp < B) {
+        const float* mom = gbuf + (size_t)B * d + (size_t)warp * G * 2;
         float s = 0.f, s2 = 0.f;
-        if (warp < B)
-          for (int cq = lane; cq < G; cq += 32) {
-            s += mom[(warp * G + cq) * 2];
-            s2 += mom[(warp * G + cq) * 2 + 1];
-          }
+        for (int cq = lane; cq < G; cq += 32) {
+          s += mom[2 * cq];
+          s2 += mom[2 * cq + 1];
+        }
         const float sum = warp_sum(s);
         s2 = warp_sum(s2);
         if (lane == 0) {
           const float mean = sum / (float)d;
           const float var = fmaxf(s2 / (float)d - mean * mean, 0.f);
           sm.gmean[warp] = mean;
-          sm.gsd[warp] = sqrtf(var + kNormEps);
+          sm.gsd[warp] = 1.0f / sqrtf(var + kNormEps);   // one division per token; elements multiply
         }
       }
       named_bar_sync(kRedBar, kConsumerThreads);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int pr = t + k * kConsumerThreads;
-        if (pr < npairs) {
-          const int idx = 2 * pr, b = idx / d;
-          const float mean = sm.gmean[b], sd = sm.gsd[b];
-          xs[idx] = XT(round_act<FAM>((tag_val(w0[k]) - mean) / sd));
-          xs[idx + 1] = XT(round_act<FAM>((tag_val(w1[k]) - mean) / sd));
-        }
-      }
-      // pairs past the first chunk (wide layers or several tokens): published already
-      for (int base = 8 * kConsumerThreads; base < npairs; base += 8 * kConsumerThreads) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) w0[k] = w1[k] = 0;
-        need = 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          if (base + t + k * kConsumerThreads < npairs) need |= 1u << k;
-        bool started = false;
-        uint64_t tp0 = 0;
-        while (need) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if (need >> k & 1u) ld_tag2(p.vx + 2 * (size_t)(base + t + k * kConsumerThreads), w0[k], w1[k]);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if ((need >> k & 1u) && tag_ok(w0[k], tag_v) && tag_ok(w1[k], tag_v)) need &= ~(1u << k);
-          if (!need || aborted(sm)) break;
-          if (!started) { tp0 = wait_start(); started = true; }
-          else if (timed_out(tp0, p.wait_cycles)) { set_abort(sm, p.err, DEV_ERR_GRID_TIMEOUT); break; }
-          if (p.poll_ns) __nanosleep(p.poll_ns);
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int pr = base + t + k * kConsumerThreads;
-          if (pr < npairs) {
-            const int idx = 2 * pr, b = idx / d;
-            const float mean = sm.gmean[b], sd = sm.gsd[b];
-            xs[idx] = XT(round_act<FAM>((tag_val(w0[k]) - mean) / sd));
-            xs[idx + 1] = XT(round_act<FAM>((tag_val(w1[k]) - mean) / sd));
-          }
-        }
+      for (int b = 0; b < B; ++b) {
+        const float mean = sm.gmean[b], inv = sm.gsd[b];
+        for (int j = t; j < d; j += kConsumerThreads)
+          xs[b * d + j] = XT(round_act<FAM>((gbuf[b * d + j] - mean) * inv));
       }
       named_bar_sync(kRedBar, kConsumerThreads);
       // every block writes its own columns of the trace and of the output
       if (p.trace.x || l == p.L - 1)
-        for (int q = t; q < B * ncol; q += kConsumerThreads) {
-          const int b = q / ncol;
-          const size_t j = (size_t)b * d + col0 + q % ncol;
-          const float xv = xs_val<FAM>(xs, (int)j);
-          if (p.trace.x) store_act<FAM>(p.trace.x, (size_t)(l + 1) * B * d + j, xv);
-          if (l == p.L - 1) store_act<FAM>(p.x_out, j, xv);
-        }
+        for (int b = 0; b < B; ++b)
+          for (int q = t; q < ncol; q += kConsumerThreads) {
+            const int j = b * d + col0 + q;
+            const float xv = xs_val<FAM>(xs, j);
+            if (p.trace.x) store_act<FAM>(p.trace.x, (size_t)(l + 1) * B * d + j, xv);
+            if (l == p.L - 1) store_act<FAM>(p.x_out, (size_t)j, xv);
+          }
     }
     stamp(p, l, 13);
   }
@@ -1513,16 +1528,22 @@ bool fused_plan_smem(FusedParams& p, int family, size_t budget, size_t& smem_byt
   const long long max_p2_item = std::max((long long)p.p2_item_bytes, (long long)p.p2_stride);
   const long long max_item = std::max({(long long)p.rec_stride, (long long)p.p1_rows_per_item * p.p1_row,
                                        max_p2_item});
-  const size_t dred_floats = std::max((size_t)(kConsumerWarps + 1) * p.pmax * nb * pe, (size_t)nb * G * 2);
+  const size_t dred_floats = (size_t)kConsumerWarps * p.pmax * nb * pe;
   size_t off = round_up(sizeof(Smem), 128);
   const size_t fixed_tail = round_up((size_t)nb * p.d * xbytes, 16) + round_up((size_t)nb * p.r * 4, 16) +
                             round_up((size_t)G * nb * p.nw * 4, 16) + round_up(dred_floats * 4, 16);
-  // per chunk entry: its dlist slot and its units (plus a scale word per Q4_0 unit), twice
-  const size_t entry_bytes = 2 * (4 + (size_t)p.pmax * 16 + (family == FAM_Q4 ? (size_t)p.pmax * 4 : 0));
+  // per chunk entry: its dlist and dhid slots and its units (plus a scale word per Q4_0
+  // unit), twice
+  const size_t entry_bytes = 2 * (8 + (size_t)nb * 4 + (size_t)p.pmax * 16 + (family == FAM_Q4 ? (size_t)p.pmax * 4 : 0));
   const size_t ring_min = std::max((size_t)112 * 1024, (size_t)(2 * max_item));
   if (budget < off + fixed_tail + ring_min + 64 * entry_bytes + 256) return false;
   size_t dch = (budget - off - fixed_tail - ring_min - 256) / entry_bytes;
   dch = std::min(dch, (size_t)kMaxDch);
+  p.dch = (int)dch;
+  // the glue reuses the down region (dlist .. hs) for all of v and the slice moments
+  const size_t glue_bytes = ((size_t)nb * p.d + 2 * (size_t)nb * G) * 4;
+  if (dch * entry_bytes < glue_bytes) dch = std::min((size_t)kMaxDch, (glue_bytes + entry_bytes - 1) / entry_bytes);
+  if (dch * entry_bytes < glue_bytes) return false;
   p.dch = (int)dch;
   const size_t down_bytes = round_up(dch * entry_bytes, 128);
   p.ring_bytes = (int)((budget - off - fixed_tail - down_bytes - 256) / 128 * 128);
@@ -1538,11 +1559,13 @@ bool fused_plan_smem(FusedParams& p, int family, size_t budget, size_t& smem_byt
   p.off_dred = (int)off;
   off += round_up(dred_floats * 4, 16);
   p.off_dlist = (int)off;
-  off += round_up((size_t)2 * dch * 4, 16);
+  off += round_up((size_t)4 * dch * 4, 16);
   p.off_dbuf = (int)off;
   off += (size_t)2 * dch * p.pmax * 16;
   p.off_dsc = (int)off;
   off += family == FAM_Q4 ? (size_t)2 * dch * p.pmax * 4 : 0;
+  p.off_hs = (int)off;
+  off += (size_t)2 * dch * nb * 4;
   smem_bytes = round_up(off, 128);
   return smem_bytes <= budget;
 }

@@ -92,9 +92,8 @@ struct pi_workspace {
   int device;
   uint64_t* ux;      // [B_max][r_max]          tagged u
   uint64_t* mx;      // [grid][4][kMaxOwnWords] tagged own mask words
-  uint64_t* hx;      // [f_max][B_max]          tagged h of the active neurons
-  uint64_t* vx;      // [B_max][d_max]          tagged x + y
-  uint64_t* sx;      // [B_max][grid][2]        tagged column-slice sums and sums of squares
+  uint64_t* hx;      // [f_max + grid][B_max]   tagged h: owner o's records from word o * nown_max on
+  uint64_t* vx;      // [B][d] tagged x + y, then [B][grid][2] the column slices' sums and sums of squares
   uint32_t* bar;     // [0] probe barrier count, [1] exit count, [2] launch epoch (tags)
   int* err;          // device error word
   unsigned long long* active_total;  // running sum of active-list lengths (all calls)
@@ -139,7 +138,7 @@ struct FusedParams {
   int pmax;            // most down units one block owns: ceil(dunits / grid), <= kMaxPieces
   int dch;             // active entries per down chunk (each chunk's rows fit one half of dbuf)
   // dynamic shared-memory layout (byte offsets)
-  int off_ring, off_xs, off_us, off_ob, off_dlist, off_dbuf, off_dsc, off_dred;
+  int off_ring, off_xs, off_us, off_ob, off_dlist, off_dbuf, off_dsc, off_dred, off_hs;
   LayerDev layers[kMaxLayers];
   // inputs / outputs
   const void* x_in;          // [B][d] activation dtype
@@ -155,8 +154,7 @@ struct FusedParams {
   uint64_t* ux;
   uint64_t* mx;
   uint64_t* hx;
-  uint64_t* vx;
-  uint64_t* sx;
+  uint64_t* vx;        // [B][d] v, then [B][grid][2] slice moments
   uint32_t* bar;
   int* err;
   unsigned long long* active_total;

@@ -50,7 +50,9 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* b, uint32_t parity) {
 // Blocking form for wait loops: the thread may be suspended until the phase completes or
 // about `hint_ns` pass, instead of spinning and taking issue slots from the warps that
 // share its scheduler.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity);
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* b, uint32_t parity, uint32_t hint_ns) {
+  if (hint_ns == 0) return mbar_try_wait(b, parity);
   uint32_t ok;
   asm volatile(
       "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n"
@@ -82,9 +84,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
       "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
-__device__ __forceinline__ void prefetch_l2_bulk(const void* src_gmem, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src_gmem), "r"(bytes) : "memory");
-}
 
 // ---------------------------------------------------------------- global sync
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
@@ -96,9 +95,14 @@ __device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Named barrier among the first `nthreads` threads (a multiple of 32).
+// Named barrier `id`: completes once `nthreads` threads (a multiple of 32) have arrived.
+// named_bar_sync arrives and waits; named_bar_arrive (a producer's side) arrives without
+// waiting, its earlier writes visible to the threads the barrier releases.
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------- conversions
@@ -123,4 +127,9 @@ __device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_gro
 // every group but the newest one has landed
 __device__ __forceinline__ void cpa_wait_but_newest() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cpa_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// The mbarrier at `bar` counts one arrival once every cp.async this thread issued so far
+// has landed (its expected count already includes this arrival).
+__device__ __forceinline__ void cpa_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 }  // namespace pi

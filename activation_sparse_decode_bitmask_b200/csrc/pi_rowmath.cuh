@@ -57,6 +57,9 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
   return v;
 }
+__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
 __device__ __forceinline__ float lds_f32(uint32_t a) {
   float v;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
@@ -65,6 +68,19 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
 __device__ __forceinline__ float lds_h2f(uint32_t a) {
   unsigned short v;
   asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return __half2float(__ushort_as_half(v));
+}
+// Read-only streaming loads from global memory (weights that no kernel writes meanwhile)
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+__device__ __forceinline__ float ldg_h2f(const void* p) {
+  unsigned short v;
+  asm("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
   return __half2float(__ushort_as_half(v));
 }
 __device__ __forceinline__ float4 u4f(uint4 v) {
@@ -121,19 +137,26 @@ __device__ __forceinline__ uint32_t q4_pair(uint32_t codes) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// acc[b] += (unit q of a weight row) . xu[b]
+// Byte offset, within a weight row, of the 16 bytes unit q reads: the unit itself, or
+// for Q4_0 the code block it is one half of.
+template <int FAM>
+__device__ __forceinline__ uint32_t unit_byte(int q) {
+  return FAM == FAM_Q4 ? 16u * (uint32_t)(q >> 1) : 16u * (uint32_t)q;
+}
+
+// acc[b] += (unit q of a weight row) . xu[b], from the unit's 16 bytes w (and for Q4_0
+// the block's fp16 scale sc)
 template <int FAM, int NB>
-__device__ __forceinline__ void unit_dot(uint32_t row, int d, int q, const uint32_t (&xu)[NB][Fam<FAM>::XW],
-                                         float (&acc)[NB]) {
+__device__ __forceinline__ void unit_dot_w(const uint4 w, float sc, int q, const uint32_t (&xu)[NB][Fam<FAM>::XW],
+                                           float (&acc)[NB]) {
   if constexpr (FAM == FAM_F32) {
-    const float4 w = u4f(lds128(row + 16u * q));
+    const float4 v = u4f(w);
 #pragma unroll
     for (int b = 0; b < NB; ++b)
-      acc[b] = fmaf(w.w, __uint_as_float(xu[b][3]),
-                    fmaf(w.z, __uint_as_float(xu[b][2]),
-                         fmaf(w.y, __uint_as_float(xu[b][1]), fmaf(w.x, __uint_as_float(xu[b][0]), acc[b]))));
+      acc[b] = fmaf(v.w, __uint_as_float(xu[b][3]),
+                    fmaf(v.z, __uint_as_float(xu[b][2]),
+                         fmaf(v.y, __uint_as_float(xu[b][1]), fmaf(v.x, __uint_as_float(xu[b][0]), acc[b]))));
   } else if constexpr (FAM == FAM_F16) {
-    const uint4 w = lds128(row + 16u * q);
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       float s = acc[b], s2 = 0.f;
@@ -144,12 +167,9 @@ __device__ __forceinline__ void unit_dot(uint32_t row, int d, int q, const uint3
       acc[b] = s + s2;
     }
   } else {
-    const int blk = q >> 1;
-    const uint4 nb = lds128(row + 16u * blk);
-    const float sc = lds_h2f(row + (uint32_t)(d >> 1) + 2u * blk);
     const int sh = (q & 1) * 4;
-    const uint32_t wv[4] = {(nb.x >> sh) & 0x0F0F0F0Fu, (nb.y >> sh) & 0x0F0F0F0Fu, (nb.z >> sh) & 0x0F0F0F0Fu,
-                            (nb.w >> sh) & 0x0F0F0F0Fu};
+    const uint32_t wv[4] = {(w.x >> sh) & 0x0F0F0F0Fu, (w.y >> sh) & 0x0F0F0F0Fu, (w.z >> sh) & 0x0F0F0F0Fu,
+                            (w.w >> sh) & 0x0F0F0F0Fu};
     uint32_t wp[8];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -164,6 +184,15 @@ __device__ __forceinline__ void unit_dot(uint32_t row, int d, int q, const uint3
       acc[b] = fmaf(sc, s + s2, acc[b]);
     }
   }
+}
+
+// The same with the row in shared memory (row: shared address; d: the row's length)
+template <int FAM, int NB>
+__device__ __forceinline__ void unit_dot(uint32_t row, int d, int q, const uint32_t (&xu)[NB][Fam<FAM>::XW],
+                                         float (&acc)[NB]) {
+  const uint4 w = lds128(row + unit_byte<FAM>(q));
+  const float sc = FAM == FAM_Q4 ? lds_h2f(row + (uint32_t)(d >> 1) + 2u * (uint32_t)(q >> 1)) : 0.f;
+  unit_dot_w<FAM, NB>(w, sc, q, xu, acc);
 }
 
 // acc[b] += (unit q of a predictor row in the p dtype: fp32 for the fp32 family, else

@@ -207,17 +207,18 @@ pi_status pi_workspace_layer_counts(pi_workspace* ws, int32_t* host_out, int L);
 pi_status pi_diag_barrier_timeout(pi_workspace* ws, long long timeout_ns, cudaStream_t stream);
 
 /* Diagnostic: with `on`, every later pi_decode_stack on this workspace records each
- * block's SM cycle counter at up to 64 points of every layer. Consumer warps: 0 layer
+ * block's SM cycle counter at up to 64 points of every layer. Consumer warp 0: 0 layer
  * start, 1 u rows published, 2 u received, 3 logits done, 4 own list and mask words
- * published, 5 every block's mask words received, 6 assignment done (list handed to the
- * producer), 7 down-row copies issued, 8 first record landed, 9 gate/up dots done,
- * 10 down slice summed, 11 v and moments published, 12 every v and moment received,
- * 13 glue done. Producer warp: 20 waits for the list, 21 list received, 22 all records
- * issued. Slot 14 holds the block's record count, 15 the layer's active count, 17 the
- * cycles thread 0 polls for h, 18 the cycles spent waiting for P2 rows and 19 those
- * warp 0 waits for records to land. With `on` = 2 the stamps come from the GPU's global
- * nanosecond timer instead, so blocks can be compared with one another. With `on` = 0
- * recording stops and the buffer is freed. */
+ * published, 6 list barrier passed, 8 first record landed, 9 gate/up dots done, 25 h
+ * words of the first chunks received, 26 every warp past the h barrier, 27 the down
+ * copies of chunk 0 landed, 28 down products done, 10 down slice summed, 11 v and
+ * moments published, 12 every v and moment received, 13 glue done. First helper thread:
+ * 5 every block's mask words received, 29 the rest of the list handed over, 23 down
+ * list built, 7 down copies issued. Slot 14 holds the block's own active count, 15 the
+ * layer's active count, 17 the cycles thread 0 polls for h and 18 the cycles spent
+ * waiting for P2 rows. With `on` = 2 the stamps come from the GPU's global nanosecond
+ * timer instead, so blocks can be compared with one another. With `on` = 0 recording
+ * stops and the buffer is freed. */
 pi_status pi_diag_phase_clocks_enable(pi_workspace* ws, int on);
 
 /* Copy the first n stamps ([grid][L_max][64], int64) to host memory (synchronous). */

@@ -352,7 +352,7 @@ def test_allocation_failure_is_reported():
 
 
 # ----------------------------------------------------------------- per-layer predictor rank
-W_MIXED_RANK = S.scaled(S.LLAMA2_7B, "reglu_f16_mixed_rank", 3, 1024, 4192, 192, layer_rank=(128, 64, 192))
+W_MIXED_RANK = S.scaled(S.LLAMA2_7B, "reglu_f16_mixed_rank", 3, 1024, 4192, 384, layer_rank=(256, 128, 384))
 
 
 @pytest.mark.parametrize("B", [1, 2, 8])
@@ -360,7 +360,7 @@ def test_decode_stack_mixed_rank(B):
     """Layers of one stack with different predictor ranks (unite.ai "PowerInfer: Mesin
     Inferensi LLM Cepat dengan GPU Konsumen", §"Prediktor Kepadatan Adaptif": each layer's
     predictor is sized on its own) run in one call and match the oracle layer by layer."""
-    assert [W_MIXED_RANK.at_layer(l).rank for l in range(3)] == [128, 64, 192]
+    assert [W_MIXED_RANK.at_layer(l).rank for l in range(3)] == [256, 128, 384]
     flips, resyncs = _stack_check(W_MIXED_RANK, B, 3, stream_id=600 + B)
     print(f"mixed-rank stack B={B}: in-band flips {flips}, re-syncs {resyncs}")
 
