@@ -12,18 +12,19 @@
 //         bit = logit > 0.  The block lists its own active neurons, publishes its bit
 //         words and hands the first na of the list (a floor set from the firing
 //         frequencies) to the producer at once.
-//   F     warps 0..11 dot records as they land (a group of warps per record):
+//   F     warps 0..7 dot records as they land (a group of warps per record):
 //           ReLU : h = max(0, w_up_i . x + b_i)    ReGLU: max(0, w_gate_i . x + b_i) * (w_up_i . x)
 //           squared ReLU: h = max(0, w_up_i . x + b_i)^2
 //           h[b] = 0 where token b's bit is 0
 //         -> h exchange: owner o's k-th active neuron publishes h at word o * nown_max + k
-//   help  meanwhile warps 12..15 poll every block's bit words, count them, and derive the
+//   help  meanwhile warps 8..15 poll every block's bit words, count them, and derive the
 //         same balanced assignment in every block: target T = ceil(N / G); a block dots
 //         at most max(T, na) of its own records and takes the excess of the blocks above
 //         T in block order.  They list the rest of the block's records for the producer
 //         and the F warps, build the layer's down list (all N active neurons in owner-major
 //         order with their h words) and copy the block's slice of every listed down row
-//         into shared memory (cp.async, completing on an mbarrier).
+//         into shared memory (cp.async, completing on an mbarrier).  Down-list chunks past
+//         the second are built and copied by every consumer thread during the down pass.
 //   down  block c owns a slice of the d output columns: once the h words are in,
 //         y[slice] = sum over the active neurons of h_i * W_down[i][slice], in a fixed
 //         order, and v = x + y with the slice's sum and sum of squares -> v exchange
@@ -58,8 +59,9 @@ constexpr int kItems = 32;          // ring items in flight (mbarrier pairs)
 constexpr int kHr = 48;             // F h slots: more than kItems, so a slot is free before its reuse
 constexpr uint32_t kSleepNs = 20000;  // suspend hint of blocking mbarrier waits (wakes on completion)
 constexpr int kMaxDch = 1024;       // entries per down chunk
-constexpr int kFWarps = 12;         // consumer warps that dot records; the others help
+constexpr int kFWarps = 8;          // consumer warps that dot records; the others help
 constexpr int kHelperThreads = (kConsumerWarps - kFWarps) * 32;
+static_assert(2 * kHelperThreads >= kMaxGrid, "the helpers take two owners a thread");
 constexpr int kAssignBar = 2;       // F warps + helpers: the taken records are listed
 constexpr int kHelpBar = 3;         // helpers only
 
@@ -83,7 +85,8 @@ struct Smem {
   uint8_t own_bits[kMaxOwn];
   int32_t pre[kMaxGrid + 1];    // exclusive prefix of cnt: entries in owner-major order
   int32_t xpre[kMaxGrid + 1];   // exclusive prefix of the owners' excess over the target
-  int32_t wsum[2][kConsumerWarps];   // block scans: the warps' totals
+  int32_t wsum[2][kConsumerWarps];   // helper scans: the warps' totals
+  int32_t wall[kConsumerWarps]; // block scan of the consumer threads' word runs
   uint64_t list_ready;          // the first na records of the list are in place
   uint64_t list2_ready;         // all nrec records of the list are in place
   int na;                       // records handed to the producer before the mask exchange
@@ -500,8 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     mbar_init(&sm.fdone, 1);
     mbar_init(&sm.list_ready, 1);
     mbar_init(&sm.list2_ready, 1);
-    mbar_init(&sm.dfull[0], kHelperThreads);
-    mbar_init(&sm.dfull[1], kHelperThreads);
+    mbar_init(&sm.dfull[0], kConsumerThreads);
+    mbar_init(&sm.dfull[1], kConsumerThreads);
     sm.abort_flag = 0;
     mbar_fence_init();
   }
@@ -936,16 +939,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     const int ht = t - kFWarps * 32;   // helper thread index (>= 0 in the helper warps)
     int woff = 0;                      // helpers: the layer's entries before this thread's mask words
     // chunks k .. k + nk - 1 (nk = 2 only from an even k: the two halves in order)
-    auto build_dlist = [&](int k, int nk) {
+    // Word runs: the helpers' (one run a helper thread, its first entry at woff) and, for
+    // chunks past the second, every consumer thread's (wa0, wa1, aoff).
+    auto build_dlist = [&](int k, int nk, int rj0, int rj1, int roff, int tid, int nthr) {
       const int lo = k * dch, hi = min(ntotal, lo + nk * dch);
       int32_t* dl = dlist + (k & 1) * dch;
       int32_t* dh = dhid + (k & 1) * dch;
       if (do_pred) {
-        // this thread's run of mask words, its first entry at woff: set bits in order
-        int e = woff;
-        int o = wj0 / nw, w = wj0 - o * nw;
+        // this thread's run of mask words, its first entry at roff: set bits in order
+        int e = roff;
+        int o = rj0 / nw, w = rj0 - o * nw;
         const uint32_t dla = smem_u32(dl), dha = smem_u32(dh);
-        for (int j = wj0; j < wj1 && e < hi; ++j) {
+        for (int j = rj0; j < rj1 && e < hi; ++j) {
           uint32_t u = union_word(ob, o, w, nw, B);
           const int n = __popc(u);
           if (e + n > lo) {
@@ -969,7 +974,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
           }
         }
       } else {
-        for (int e = lo + ht; e < hi; e += kHelperThreads) {
+        for (int e = lo + tid; e < hi; e += nthr) {
           int i = __ldg(p.idx_in + e);
           if (i < 0 || i >= f) i = 0;   // reported above
           dl[e - lo] = i;
@@ -980,12 +985,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     // helper lane mapping of the copies: the F mapping of the down pass over 4 warps
     const int hde0 = (warp - kFWarps) * epw + lane / lpe;
     const int hdstep = (kConsumerWarps - kFWarps) * epw;
-    auto issue_down = [&](int k) {
+    auto issue_down = [&](int k, int ef, int es) {
       if (dw >= 0) {
         const int lo = k * dch, hi = min(ntotal, lo + dch);
         const int32_t* dl = dlist + (k & 1) * dch;
         const int half = (k & 1) * dch;
-        for (int e = lo + hde0; e < hi; e += hdstep) {
+        for (int e = lo + ef; e < hi; e += es) {
           const int i = dl[e - lo];
           const uint8_t* row = dn + (size_t)i * p.dn_stride;
           const uint32_t slot = (uint32_t)((half + e - lo) * pmax + dw);
@@ -1180,9 +1185,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
           px = ox + ix - (x0 + x1);
           ps = os + is - (s0 + s1);
         }
-        sm.xpre[2 * ht] = px;
-        sm.xpre[2 * ht + 1] = px + x0;
-        if (ht == kHelperThreads - 1) sm.xpre[2 * kHelperThreads] = xtotal;
+        if (2 * ht < G) sm.xpre[2 * ht] = px;
+        if (2 * ht + 1 < G) sm.xpre[2 * ht + 1] = px + x0;
+        if (ht == 0) sm.xpre[G] = xtotal;
         if (2 * ht == c) sm.wsum[0][kConsumerWarps - 1] = ps;
         if (2 * ht + 1 == c) sm.wsum[0][kConsumerWarps - 1] = ps + s0;
         named_bar_sync(kHelpBar, kHelperThreads);
@@ -1219,11 +1224,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
       named_bar_arrive(kAssignBar, kConsumerThreads);   // the F warps dot it
       hstamp(p, l, 29);
       const int nchunks = (ntotal + dch - 1) / dch;
-      build_dlist(0, 2);
+      build_dlist(0, 2, wj0, wj1, woff, ht, kHelperThreads);
       named_bar_sync(kHelpBar, kHelperThreads);
       hstamp(p, l, 23);
-      if (nchunks > 0) issue_down(0);
-      if (nchunks > 1) issue_down(1);
+      if (nchunks > 0) issue_down(0, hde0, hdstep);
+      if (nchunks > 1) issue_down(1, hde0, hdstep);
       hstamp(p, l, 7);
     }
     if (do_pred) ntotal = sm.pre[G];   // every warp: the layer's active count
@@ -1249,6 +1254,34 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     };
     // every warp is past F and the down list halves 0 and 1 are built
     named_bar_sync(kRedBar, kConsumerThreads);
+    if (warp < kFWarps) {   // the F warps' arrivals on the copies of chunks 0 and 1 (none)
+      if (nchunks > 0) cpa_arrive_noinc(&sm.dfull[0]);
+      if (nchunks > 1) cpa_arrive_noinc(&sm.dfull[1]);
+    }
+    // chunks past the second are built and copied by every consumer thread: each takes a
+    // run of the mask words, its first entry from a block scan of the runs' counts
+    int wa0 = 0, wa1 = 0, aoff = 0;
+    if (do_pred && nchunks > 2) {
+      const int wpa = (G * nw + kConsumerThreads - 1) / kConsumerThreads;
+      wa0 = min(G * nw, t * wpa);
+      wa1 = min(G * nw, wa0 + wpa);
+      int cnt = 0;
+      for (int j = wa0; j < wa1; ++j) {
+        const int o = j / nw;
+        cnt += __popc(union_word(ob, o, j - o * nw, nw, B));
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int k = 1; k < 32; k <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, incl, k);
+        if (lane >= k) incl += x;
+      }
+      if (lane == 31) sm.wall[warp] = incl;
+      named_bar_sync(kRedBar, kConsumerThreads);
+      int off = 0;
+      for (int w = 0; w < warp; ++w) off += sm.wall[w];
+      aoff = off + incl - cnt;
+    }
     {
       // the ring past this layer's records (every consumer keeps the same ring state)
       const int nr = sm.nrec;
@@ -1283,9 +1316,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
       }
       if (k + 2 < nchunks) {
         named_bar_sync(kRedBar, kConsumerThreads);   // every thread is done with dlist, hs and dbuf half k%2
-        if (warp >= kFWarps) build_dlist(k + 2, 1);
+        build_dlist(k + 2, 1, wa0, wa1, aoff, t, kConsumerThreads);
         named_bar_sync(kRedBar, kConsumerThreads);   // chunk k + 2's dlist and dhid are in place
-        if (warp >= kFWarps) issue_down(k + 2);
+        issue_down(k + 2, de0, dstep);
       }
     }
     stamp(p, l, 28);
