@@ -112,7 +112,7 @@ pi_status plan_fused(const pi_layer* L, int B, const pi_workspace* ws, FusedPara
   if (!fused_supported(L->family, B, d.d_model)) return PI_ERR_UNSUPPORTED;
   if (!fused_plan_smem(p, L->family, (size_t)smem_optin(ws->device), smem)) return PI_ERR_UNSUPPORTED;
   // ws fields
-  p.ux = ws->ux; p.mx = ws->mx; p.hx = ws->hx; p.vx = ws->vx;
+  p.ux = ws->ux; p.mx = ws->mx; p.hx = ws->hx; p.vx = ws->vx; p.yx = ws->yx;
   p.bar = ws->bar; p.err = ws->err; p.active_total = ws->active_total;
   p.layer_count = nullptr;
   p.barrier_timeout_ns = kDefaultWaitNs;
@@ -413,6 +413,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
             dmalloc(&ws->mx, mx_bytes) == cudaSuccess &&
             dmalloc(&ws->hx, hx_bytes) == cudaSuccess &&
             dmalloc(&ws->vx, (Bm * d_max + 2 * Bm * G) * 8) == cudaSuccess &&
+            dmalloc(&ws->yx, G * (size_t)d_max * 8) == cudaSuccess &&
             dmalloc(&ws->bar, 64) == cudaSuccess &&
             dmalloc(&ws->err, 16) == cudaSuccess &&
             dmalloc(&ws->active_total, 16) == cudaSuccess &&
@@ -433,6 +434,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
     ok = cudaMemset(ws->ux, 0, Bm * r_max * 8) == cudaSuccess && cudaMemset(ws->mx, 0, mx_bytes) == cudaSuccess &&
          cudaMemset(ws->hx, 0, hx_bytes) == cudaSuccess &&
          cudaMemset(ws->vx, 0, (Bm * d_max + 2 * Bm * G) * 8) == cudaSuccess &&
+         cudaMemset(ws->yx, 0, G * (size_t)d_max * 8) == cudaSuccess &&
          cudaMemset(ws->bar, 0, 64) == cudaSuccess &&
          cudaMemcpy(ws->bar, bar0, sizeof(bar0), cudaMemcpyHostToDevice) == cudaSuccess &&
          cudaMemset(ws->err, 0, 16) == cudaSuccess && cudaMemset(ws->active_total, 0, 16) == cudaSuccess &&
@@ -449,7 +451,7 @@ pi_status pi_workspace_create(int d_max, int f_max, int r_max, int B_max, int L_
 
 void pi_workspace_free(pi_workspace* ws) {
   if (!ws) return;
-  cudaFree(ws->ux); cudaFree(ws->mx); cudaFree(ws->hx); cudaFree(ws->vx);
+  cudaFree(ws->ux); cudaFree(ws->mx); cudaFree(ws->hx); cudaFree(ws->vx); cudaFree(ws->yx);
   cudaFree(ws->bar); cudaFree(ws->err); cudaFree(ws->active_total);
   cudaFree(ws->layer_count); cudaFree(ws->x_dev); cudaFree(ws->phase_clk);
   cudaFree(ws->u_hi); cudaFree(ws->u_lo); cudaFree(ws->bmask); cudaFree(ws->bidx); cudaFree(ws->bcount);

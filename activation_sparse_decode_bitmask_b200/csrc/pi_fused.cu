@@ -65,7 +65,11 @@ static_assert(2 * kHelperThreads >= kMaxGrid, "the helpers take two owners a thr
 constexpr int kAssignBar = 2;       // F warps + helpers: the taken records are listed
 constexpr int kHelpBar = 3;         // helpers only
 
-enum Exchange : int { EX_U = 0, EX_M = 1, EX_H = 2, EX_V = 3 };
+enum Exchange : int { EX_U = 0, EX_M = 1, EX_H = 2, EX_V = 3, EX_Y = 4 };
+
+// Row-owned down pass (one token, layers whose active list exceeds two down chunks): each
+// thread keeps the partial y of the down units t, t + 512, ... (at most kRoUnits of them).
+__host__ __device__ constexpr int ro_units(int fam) { return fam == FAM_Q4 ? 1 : 3; }
 
 struct Smem {
   uint64_t full[kItems];
@@ -92,6 +96,9 @@ struct Smem {
   int na;                       // records handed to the producer before the mask exchange
   int own_cnt;                  // own records this block dots (list entries [0, own_cnt))
   int nrec;                     // records this block dots: own_cnt own ones, then taken ones
+  int keep_t;                   // own records whose down rows this block takes (row-owned pass)
+  int ro;                       // this layer's down pass is row-owned
+  float hrec[kMaxList];         // h of each dotted record (one token)
   uint64_t dfull[2];            // down chunk copies of each half landed
   uint64_t fdone;               // the layer's neuron records are dotted (the producer's gate)
 };
@@ -624,6 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
         const int n1 = do_pred ? (k1 - k0 + p.p1_rows_per_item - 1) / p.p1_rows_per_item : 0;
         const int n2 = do_pred ? (nown + p2_rows - 1) / p2_rows : 0;
         int na = 0, n = 0;   // records: handed over first, in all (known once listed)
+        int nd = 0, keep_t = 0, own_c = 0;   // row-owned layers: down rows after the records
         for (int it = 0; ok; ++it) {
           const uint8_t* src;
           uint32_t bytes;
@@ -645,10 +653,22 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
             if (e == na && n == na) {
               if (!(ok = wait_list(&sm.list2_ready, (uint32_t)(l & 1)))) break;
               n = sm.nrec;
+              if (sm.ro) {
+                keep_t = sm.keep_t;
+                own_c = sm.own_cnt;
+                nd = keep_t + (n - own_c);
+              }
             }
-            if (e >= n) break;
-            src = Ld.rec + (size_t)sm.list[e] * p.rec_stride;
-            bytes = (uint32_t)p.rec_stride;
+            if (e < n) {
+              src = Ld.rec + (size_t)sm.list[e] * p.rec_stride;
+              bytes = (uint32_t)p.rec_stride;
+            } else {
+              const int j = e - n;   // down row j: own entries below T, then the taken ones
+              if (j >= nd) break;
+              const int ent = j < keep_t ? j : own_c + (j - keep_t);
+              src = Ld.rec + p.dn_off + (size_t)sm.list[ent] * p.dn_stride;
+              bytes = (uint32_t)p.dn_stride;
+            }
           }
           uint8_t* dst;
           uint64_t* fb;
@@ -695,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     const int p2_stride = p2_stride_of(r, PB);
     const int p2_rows = max(1, min(p.nown_max, p.p2_item_bytes / p2_stride));
     const uint32_t tag_u = tag_of(epoch, l, EX_U), tag_m = tag_of(epoch, l, EX_M), tag_h = tag_of(epoch, l, EX_H),
-                   tag_v = tag_of(epoch, l, EX_V);
+                   tag_v = tag_of(epoch, l, EX_V), tag_y = tag_of(epoch, l, EX_Y);
     int nlist = 0;      // records this block dots
     int ntotal = 0;     // active entries of the layer (the down list)
     int hid0 = 0;       // h word of the block's first record: records publish h in list order
@@ -918,6 +938,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
       if (t == 0) {
         atomicAdd(p.active_total, (unsigned long long)nlist);
         sm.na = sm.own_cnt = sm.nrec = nlist;
+        sm.ro = 0;
         mbar_arrive(&sm.list_ready);
       }
       ntotal = cnt;
@@ -1079,6 +1100,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
                   if (p.act_square) a *= a;
                 }
                 st_tag(p.hx + (size_t)ent * B + b, ((bits >> b) & 1u) ? a : 0.f, tag_h);
+                if (b == 0) sm.hrec[e] = (bits & 1u) ? a : 0.f;
               }
             }
             sm.hcnt[s] = 0;
@@ -1201,6 +1223,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
         if (ht == 0) {
           sm.own_cnt = own_cnt;
           sm.nrec = own_cnt + ntake;
+          // more active neurons than two down chunks hold: the row-owned down pass (one
+          // token), each block over the down rows of the records it dots, own ones past T
+          // left to their takers
+          sm.ro = (B == 1 && N > 2 * dch && p.dunits <= kConsumerThreads * ro_units(FAM) &&
+                   G * PE * 4 <= 32 * dch) ? 1 : 0;
+          sm.keep_t = min(n_own, T);
         }
         for (int q = ht; q < ntake; q += kHelperThreads) {
           const int x = dstart + q;
@@ -1223,7 +1251,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
       if (ht == 0) mbar_arrive(&sm.list2_ready);          // the producer copies the rest
       named_bar_arrive(kAssignBar, kConsumerThreads);   // the F warps dot it
       hstamp(p, l, 29);
-      const int nchunks = (ntotal + dch - 1) / dch;
+      const int nchunks = sm.ro ? 0 : (ntotal + dch - 1) / dch;
       build_dlist(0, 2, wj0, wj1, woff, ht, kHelperThreads);
       named_bar_sync(kHelpBar, kHelperThreads);
       hstamp(p, l, 23);
@@ -1232,7 +1260,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
       hstamp(p, l, 7);
     }
     if (do_pred) ntotal = sm.pre[G];   // every warp: the layer's active count
-    const int nchunks = (ntotal + dch - 1) / dch;
+    const bool ro = sm.ro != 0;
+    const int nchunks = ro ? 0 : (ntotal + dch - 1) / dch;
     stamp_val(p, l, 15, ntotal);
 
     // ------------------------------------------------------------ down: y of the slice
@@ -1289,6 +1318,43 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
       ring.item += (uint32_t)nr;
       fseq += (uint32_t)nr;
     }
+    if (ro) {
+      // ------------------------------------------------------------ row-owned down pass
+      // The down rows of the records this block dotted follow them in the ring; thread t
+      // adds h times its units t, t + 512, ... of each row, in list order, and publishes
+      // its partial y (tagged words, d a block).
+      constexpr int RU = ro_units(FAM);
+      const int keep_t = sm.keep_t, own_c = sm.own_cnt;
+      const int nd = keep_t + (sm.nrec - own_c);
+      const uint32_t base = smem_u32(ring.base);
+      float ra[RU][1][PE];
+#pragma unroll
+      for (int u = 0; u < RU; ++u)
+#pragma unroll
+        for (int e = 0; e < PE; ++e) ra[u][0][e] = 0.f;
+      for (int j = 0; j < nd; ++j) {
+        const uint32_t pos = ring_place(ring.head, (uint32_t)p.dn_stride, ring.cap);
+        ring_wait_item_warp(ring.item, sm, p);
+        const float h1[1] = {sm.hrec[j < keep_t ? j : own_c + (j - keep_t)]};
+#pragma unroll
+        for (int u = 0; u < RU; ++u) {
+          const int unit = t + u * kConsumerThreads;
+          if (unit < p.dunits) {
+            float sc = 0.f;
+            if constexpr (FAM == FAM_Q4) sc = lds_h2f(base + pos + (uint32_t)(d >> 1) + 2u * (uint32_t)unit);
+            down_unit_fma<FAM, 1>(base + pos + 16u * (uint32_t)unit, sc, h1, ra[u]);
+          }
+        }
+        ring_release_item(ring.item++, sm);
+      }
+#pragma unroll
+      for (int u = 0; u < RU; ++u) {
+        const int unit = t + u * kConsumerThreads;
+        if (unit < p.dunits)
+#pragma unroll
+          for (int e = 0; e < PE; ++e) st_tag(p.yx + (size_t)c * d + (size_t)unit * PE + e, ra[u][0][e], tag_y);
+      }
+    }
     for (int k = 0; k < nchunks; ++k) {
       const int lo = k * dch, hi = min(ntotal, lo + dch);
       if (k == 0) poll_h(0, min(ntotal, 2 * dch), 0);
@@ -1338,12 +1404,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
           for (int o = lpe; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
           acc[b][e] = v;
         }
-      if (lane < lpe && dw >= 0) {
+      if (lane < lpe && dw >= 0 && !ro) {
 #pragma unroll
         for (int b = 0; b < NB; ++b)
 #pragma unroll
           for (int e = 0; e < PE; ++e) dred[(warp * pmax + dw) * V + b * PE + e] = acc[b][e];
       }
+      // row-owned layers: every block's partial y of this block's columns
+      float* ybuf = reinterpret_cast<float*>(dsmem + p.off_dbuf);   // [G][ncol]
+      if (ro)
+        poll_words<8>(p.yx, [&](int q) { const int g = q / ncol; return (size_t)g * d + col0 + (q - g * ncol); },
+                      G * ncol, kConsumerWarps, tag_y, reinterpret_cast<uint32_t*>(ybuf), sm, p);
       named_bar_sync(kRedBar, kConsumerThreads);
       // warp b forms token b's slice: y, v = x + y and its (sum, sum of squares), which
       // follow v in the exchange array
@@ -1353,7 +1424,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
         for (int q = lane; q < ncol; q += 32) {
           const int w = q / PE, e = q % PE;
           float y = 0.f;
-          for (int k = 0; k < kConsumerWarps; ++k) y += dred[(k * pmax + w) * V + b * PE + e];
+          if (ro)
+            for (int g = 0; g < G; ++g) y += ybuf[g * ncol + q];
+          else
+            for (int k = 0; k < kConsumerWarps; ++k) y += dred[(k * pmax + w) * V + b * PE + e];
           const int col = col0 + q;
           if (do_glue) {
             const float v = xs_val<FAM>(xs, b * d + col) + y;
@@ -1375,6 +1449,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
         }
       }
       if (!do_glue) break;
+      if (ro) named_bar_sync(kRedBar, kConsumerThreads);   // ybuf is read before the glue reuses it
     }
     stamp(p, l, 11);
 

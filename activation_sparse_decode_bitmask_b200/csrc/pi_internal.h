@@ -94,6 +94,7 @@ struct pi_workspace {
   uint64_t* mx;      // [grid][4][kMaxOwnWords] tagged own mask words
   uint64_t* hx;      // [f_max + grid][B_max]   tagged h: owner o's records from word o * nown_max on
   uint64_t* vx;      // [B][d] tagged x + y, then [B][grid][2] the column slices' sums and sums of squares
+  uint64_t* yx;      // [grid][d_max] tagged partial y of each block (row-owned down pass, one token)
   uint32_t* bar;     // [0] probe barrier count, [1] exit count, [2] launch epoch (tags)
   int* err;          // device error word
   unsigned long long* active_total;  // running sum of active-list lengths (all calls)
@@ -155,6 +156,7 @@ struct FusedParams {
   uint64_t* mx;
   uint64_t* hx;
   uint64_t* vx;        // [B][d] v, then [B][grid][2] slice moments
+  uint64_t* yx;        // [G][d] partial y of every block (row-owned down pass)
   uint32_t* bar;
   int* err;
   unsigned long long* active_total;
