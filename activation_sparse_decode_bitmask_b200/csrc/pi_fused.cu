@@ -28,6 +28,11 @@
 //   down  block c owns a slice of the d output columns: once the h words are in,
 //         y[slice] = sum over the active neurons of h_i * W_down[i][slice], in a fixed
 //         order, and v = x + y with the slice's sum and sum of squares -> v exchange
+//         With one token and more active neurons than three down-list chunks hold, the down
+//         pass is row-owned instead: each block reads the full down rows of the records it
+//         dotted (bulk copies after the records), adds h times its units of each row into
+//         registers, publishes its partial y (d words), and sums its column slice over all
+//         blocks' partials (small scattered slice copies would limit it otherwise).
 //   glue  x' = (v - mean(v)) / sqrt(var(v) + 1e-6) from every slice's v and moments,
 //         rounded to the activation dtype
 // The down projection is column-owned: a block reads only its slice of each active down
@@ -67,7 +72,7 @@ constexpr int kHelpBar = 3;         // helpers only
 
 enum Exchange : int { EX_U = 0, EX_M = 1, EX_H = 2, EX_V = 3, EX_Y = 4 };
 
-// Row-owned down pass (one token, layers whose active list exceeds two down chunks): each
+// Row-owned down pass (one token, layers whose active list exceeds three down chunks): each
 // thread keeps the partial y of the down units t, t + 512, ... (at most kRoUnits of them).
 __host__ __device__ constexpr int ro_units(int fam) { return fam == FAM_Q4 ? 1 : 3; }
 
@@ -98,7 +103,6 @@ struct Smem {
   int nrec;                     // records this block dots: own_cnt own ones, then taken ones
   int keep_t;                   // own records whose down rows this block takes (row-owned pass)
   int ro;                       // this layer's down pass is row-owned
-  float hrec[kMaxList];         // h of each dotted record (one token)
   uint64_t dfull[2];            // down chunk copies of each half landed
   uint64_t fdone;               // the layer's neuron records are dotted (the producer's gate)
 };
@@ -466,6 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
   int32_t* dlist = reinterpret_cast<int32_t*>(dsmem + p.off_dlist);  // [2][dch] neuron of each chunk entry
   int32_t* dhid = dlist + 2 * p.dch;                                  // [2][dch] its h word (per token)
   float* dred = reinterpret_cast<float*>(dsmem + p.off_dred);        // down reduction / v slice / moments
+  float* hrec = dred;   // h of each dotted record, one token (read by a row-owned down pass,
+                        // which leaves dred unused; F writes it before any slice reduction)
   const uint32_t dbuf_u = smem_u32(dsmem + p.off_dbuf);              // [2][dch][pmax] 16-byte down units
   const uint32_t dsc_u = smem_u32(dsmem + p.off_dsc);                // Q4_0: [2][dch][pmax] scale words
   float* hs = reinterpret_cast<float*>(dsmem + p.off_hs);            // [2 * dch][B] h of the resident entries
@@ -1100,7 +1106,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
                   if (p.act_square) a *= a;
                 }
                 st_tag(p.hx + (size_t)ent * B + b, ((bits >> b) & 1u) ? a : 0.f, tag_h);
-                if (b == 0) sm.hrec[e] = (bits & 1u) ? a : 0.f;
+                if (b == 0) hrec[e] = (bits & 1u) ? a : 0.f;
               }
             }
             sm.hcnt[s] = 0;
@@ -1223,10 +1229,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
         if (ht == 0) {
           sm.own_cnt = own_cnt;
           sm.nrec = own_cnt + ntake;
-          // more active neurons than two down chunks hold: the row-owned down pass (one
+          // more active neurons than three down chunks hold: the row-owned down pass (one
           // token), each block over the down rows of the records it dots, own ones past T
           // left to their takers
-          sm.ro = (B == 1 && N > 2 * dch && p.dunits <= kConsumerThreads * ro_units(FAM) &&
+          sm.ro = (B == 1 && N > 3 * dch && p.dunits <= kConsumerThreads * ro_units(FAM) &&
                    G * PE * 4 <= 32 * dch) ? 1 : 0;
           sm.keep_t = min(n_own, T);
         }
@@ -1335,7 +1341,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
       for (int j = 0; j < nd; ++j) {
         const uint32_t pos = ring_place(ring.head, (uint32_t)p.dn_stride, ring.cap);
         ring_wait_item_warp(ring.item, sm, p);
-        const float h1[1] = {sm.hrec[j < keep_t ? j : own_c + (j - keep_t)]};
+        const float h1[1] = {hrec[j < keep_t ? j : own_c + (j - keep_t)]};
 #pragma unroll
         for (int u = 0; u < RU; ++u) {
           const int unit = t + u * kConsumerThreads;
@@ -1636,7 +1642,7 @@ bool fused_plan_smem(FusedParams& p, int family, size_t budget, size_t& smem_byt
   const long long max_p2_item = std::max((long long)p.p2_item_bytes, (long long)p.p2_stride);
   const long long max_item = std::max({(long long)p.rec_stride, (long long)p.p1_rows_per_item * p.p1_row,
                                        max_p2_item});
-  const size_t dred_floats = (size_t)kConsumerWarps * p.pmax * nb * pe;
+  const size_t dred_floats = std::max((size_t)kConsumerWarps * p.pmax * nb * pe, (size_t)kMaxList);
   size_t off = round_up(sizeof(Smem), 128);
   const size_t fixed_tail = round_up((size_t)nb * p.d * xbytes, 16) + round_up((size_t)nb * p.r * 4, 16) +
                             round_up((size_t)G * nb * p.nw * 4, 16) + round_up(dred_floats * 4, 16);
