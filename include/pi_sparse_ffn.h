@@ -178,10 +178,12 @@ void pi_free_layer(pi_layer* layer);
 
 /* Scratch for the kernels: the cross-block exchange words (the predictor vector u,
  * every block's mask words, h of the active neurons, the stack's x + y and its
- * moments), the launch words, the device error word, and the multi-launch path's mask,
- * index and partial-sum buffers. It is sized for the largest shapes it will serve: calls with larger d_model,
- * d_ff, rank, B or L return PI_ERR_ARG. A workspace serves one stream at a time. Calls
- * that overlap on the device and share a workspace race. */
+ * moments, and every block's partial y for the row-owned down pass: grid x d_model_max
+ * words of 8 bytes), the launch words, the device error word, and the multi-launch
+ * path's mask, index and partial-sum buffers. It is sized for the largest shapes it
+ * will serve: calls with larger d_model, d_ff, rank, B or L return PI_ERR_ARG. A
+ * workspace serves one stream at a time. Calls that overlap on the device and share a
+ * workspace race. */
 pi_status pi_workspace_create(int d_model_max, int d_ff_max, int rank_max, int B_max,
                               int L_max, pi_workspace** out);
 void pi_workspace_free(pi_workspace* ws);
