@@ -376,3 +376,21 @@ def test_decode_stack_rejects_other_shapes():
     with pytest.raises(pi.PiError) as e:
         pi.decode_stack([ga[0], gb[0]], x, 1, ws)
     assert e.value.status == 1
+
+
+# ----------------------------------------------------------------- row-owned down pass
+# d = 1024 keeps a down-list chunk at its 1024-entry cap; ~4900 active neurons a layer
+# (15 % of 32768) exceed three chunks, so one token takes the row-owned down pass.
+W_ROW_OWNED = [S.scaled(S.FALCON_40B, "relu_f16_row_owned", 2, 1024, 32768, 128, mean_p=0.15),
+               S.scaled(S.LLAMA2_70B_Q4, "reglu_q4_row_owned", 2, 1024, 32768, 128, mean_p=0.15)]
+
+
+@pytest.mark.parametrize("wl", W_ROW_OWNED, ids=lambda w: w.name)
+def test_decode_stack_row_owned_down(wl):
+    """A stack whose layers are past three down-list chunks (each block sums the full down
+    rows of the records it dots and the blocks exchange partial y) matches the oracle
+    layer by layer, as the column-owned pass does (the down projection is the same sum,
+    KPD "PowerInfer: Fast Large Language Model Serving with a Consumer-grade GPU",
+    §"Метод": only the active neurons' rows and columns are read)."""
+    flips, resyncs = _stack_check(wl, 1, wl.n_layers, stream_id=700)
+    print(f"{wl.name}: in-band flips {flips}, re-syncs {resyncs}")
